@@ -24,7 +24,12 @@ class OrOut(C.Structure):
     _fields_ = [("hidden_out", C.c_void_p), ("h_out", C.c_void_p), ("route_ids", C.c_void_p),
                 ("route_w", C.c_void_p), ("route_gap", C.c_void_p), ("logits", C.c_void_p),
                 ("attn_out", C.c_void_p), ("k_new", C.c_void_p), ("v_new", C.c_void_p),
-                ("s_max_minus_bound", C.c_void_p), ("n_distinct", C.c_void_p)]
+                ("s_max_minus_bound", C.c_void_p), ("n_distinct", C.c_void_p), ("k_pre", C.c_void_p),
+                ("v_pre", C.c_void_p)]
+
+
+class OrForce(C.Structure):
+    _fields_ = [("ids", C.c_void_p), ("k", C.c_void_p), ("v", C.c_void_p)]
 
 
 _lib = None
@@ -35,8 +40,8 @@ def lib():
     if _lib is None:
         L = C.CDLL(_build.build())
         P = C.c_void_p
-        L.msk_oracle_step.argtypes = [C.POINTER(OrCfg), P, C.c_int, C.c_int, P, P, P, P, C.c_int,
-                                      C.POINTER(OrOut)]
+        L.msk_oracle_step.argtypes = [C.POINTER(OrCfg), P, C.c_int, C.c_int, P, P, P, C.POINTER(OrForce),
+                                      C.c_int, C.POINTER(OrOut)]
         L.msk_oracle_step.restype = C.c_int
         L.msk_or_e2m1_decode.argtypes = [C.c_int]
         L.msk_or_e2m1_decode.restype = C.c_double
@@ -69,9 +74,12 @@ def cfg_struct(w):
     return c
 
 
-def step(w, source_ptr, hidden_in, positions, seq_ids=None, forced_ids=None, threads=None):
+def step(w, source_ptr, hidden_in, positions, seq_ids=None, forced_ids=None, forced_k=None, forced_v=None,
+         threads=None):
     """Run one oracle step.  hidden_in: uint16 [T][d] bf16 bits; positions:
-    int [n_seqs][tps].  Returns a dict of numpy outputs."""
+    int [n_seqs][tps]; forced_*: optional replacements (-1 = oracle's own
+    decision) of near-tied routing [L][T][k] and of fp8 KV codes at rounding
+    midpoints [L][T][Hkv*hd].  Returns a dict of numpy outputs."""
     positions = np.ascontiguousarray(positions, np.int32)
     n_seqs, tps = positions.shape
     T = n_seqs * tps
@@ -84,17 +92,20 @@ def step(w, source_ptr, hidden_in, positions, seq_ids=None, forced_ids=None, thr
         "route_gap": np.zeros((L, T)), "logits": np.zeros((L, T, E)),
         "attn_out": np.zeros((L, T, qd)), "k_new": np.zeros((L, T, kvd), np.uint8),
         "v_new": np.zeros((L, T, kvd), np.uint8), "s_max_minus_bound": np.zeros(L),
-        "n_distinct": np.zeros(L, np.int32),
+        "n_distinct": np.zeros(L, np.int32), "k_pre": np.zeros((L, T, kvd)), "v_pre": np.zeros((L, T, kvd)),
     }
     out = OrOut(*[o[f].ctypes.data for f, _ in OrOut._fields_])
     sid = None if seq_ids is None else np.ascontiguousarray(seq_ids, np.int32)
     fr = None if forced_ids is None else np.ascontiguousarray(forced_ids, np.int16).reshape(L, T, k)
+    fk = None if forced_k is None else np.ascontiguousarray(forced_k, np.int16).reshape(L, T, kvd)
+    fv = None if forced_v is None else np.ascontiguousarray(forced_v, np.int16).reshape(L, T, kvd)
+    force = OrForce(None if fr is None else fr.ctypes.data, None if fk is None else fk.ctypes.data,
+                    None if fv is None else fv.ctypes.data)
     cfg = cfg_struct(w)
     nt = threads if threads else min(64, os.cpu_count() or 1)
     rc = lib().msk_oracle_step(C.byref(cfg), source_ptr, n_seqs, tps,
                                None if sid is None else sid.ctypes.data, positions.ctypes.data,
-                               hidden_in.ctypes.data, None if fr is None else fr.ctypes.data, nt,
-                               C.byref(out))
+                               hidden_in.ctypes.data, C.byref(force), nt, C.byref(out))
     if rc:
         raise RuntimeError(f"msk_oracle_step failed: {rc}")
     return o

@@ -310,7 +310,8 @@ static void expert_one(void* p, int64_t ui) {
 /* ---- the step ------------------------------------------------------------------ */
 int msk_oracle_step(const msk_or_cfg* g, const msk_source* src, int n_seqs, int tps,
                     const int32_t* seq_ids, const int32_t* positions, const uint16_t* hidden_in,
-                    const int16_t* forced_ids, int n_threads, msk_or_out* out) {
+                    const msk_or_force* force, int n_threads, msk_or_out* out) {
+  const int16_t* forced_ids = force ? force->ids : NULL;
   pthread_once(&g_tab_once, build_tables);
   const int L = g->n_layers, d = g->d_model, hq = g->n_q_heads, hkv = g->n_kv_heads, hd = g->head_dim;
   const int E = g->n_experts, k = g->top_k, f = g->expert_dim;
@@ -374,7 +375,11 @@ int msk_oracle_step(const msk_or_cfg* g, const msk_source* src, int n_seqs, int 
     for (int64_t i = 0; i < (int64_t)T * kvd; ++i) {
       knew[i] = (uint8_t)msk_or_e4m3_encode(kk[i]);
       vnew[i] = (uint8_t)msk_or_e4m3_encode(vv[i]);
+      if (force && force->k && force->k[(int64_t)l * T * kvd + i] >= 0) knew[i] = (uint8_t)force->k[(int64_t)l * T * kvd + i];
+      if (force && force->v && force->v[(int64_t)l * T * kvd + i] >= 0) vnew[i] = (uint8_t)force->v[(int64_t)l * T * kvd + i];
     }
+    if (out->k_pre) memcpy(out->k_pre + (int64_t)l * T * kvd, kk, sizeof(double) * (size_t)T * kvd);
+    if (out->v_pre) memcpy(out->v_pre + (int64_t)l * T * kvd, vv, sizeof(double) * (size_t)T * kvd);
     if (out->k_new) memcpy(out->k_new + (int64_t)l * T * kvd, knew, (size_t)T * kvd);
     if (out->v_new) memcpy(out->v_new + (int64_t)l * T * kvd, vnew, (size_t)T * kvd);
 

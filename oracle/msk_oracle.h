@@ -36,16 +36,27 @@ typedef struct msk_or_out {
   uint8_t* v_new;
   double* s_max_minus_bound; /* [L] max score minus sqrt(hd) max|g_q| max|g_k| */
   int32_t* n_distinct;       /* [L] distinct experts selected */
+  double* k_pre;             /* [L][T][Hkv][hd] K after QK-norm, before fp8 */
+  double* v_pre;             /* [L][T][Hkv][hd] V before fp8 */
 } msk_or_out;
+
+/* Optional replacements for decisions with two valid answers (NULL = none).
+ *  ids[L][T][k]:   a token's expert set where ids[..][0] >= 0 (near-tied
+ *                  routing); weights are the softmax of those experts' logits
+ *  k, v[L][T][Hkv*hd]: an fp8 code where >= 0 (a value at an e4m3 rounding
+ *                  midpoint, up to the compared implementation's error) */
+typedef struct msk_or_force {
+  const int16_t* ids;
+  const int16_t* k;
+  const int16_t* v;
+} msk_or_force;
 
 /* One step.  positions[n_seqs][tps] must be contiguous per sequence; keys
  * below a sequence's first position come from src->past_kv with sequence id
- * seq_ids[b] (or b if seq_ids is NULL).  forced_ids[L][T][k], if given,
- * replaces a token's routing where its first entry is >= 0 (weights are then
- * the softmax of the forced experts' logits). */
+ * seq_ids[b] (or b if seq_ids is NULL).  `force` may be NULL. */
 int msk_oracle_step(const msk_or_cfg* cfg, const msk_source* src, int n_seqs, int tps,
                     const int32_t* seq_ids, const int32_t* positions, const uint16_t* hidden_in,
-                    const int16_t* forced_ids, int n_threads, msk_or_out* out);
+                    const msk_or_force* force, int n_threads, msk_or_out* out);
 
 /* building blocks, exported for the pin tests */
 double msk_or_e2m1_decode(int nib);

@@ -13,7 +13,7 @@ import os
 import numpy as np
 
 from . import build as _build
-from .configs import WORKLOADS, Workload  # noqa: F401
+from .configs import PROFILE_WORKLOADS, WORKLOADS, Workload  # noqa: F401
 
 MAX_LAYERS = 64
 ROLES = {"wq": 0, "wk": 1, "wv": 2, "wo": 3, "w_gate": 4, "w_up": 5, "w_down": 6}

@@ -61,3 +61,8 @@ WORKLOADS = {
     # 16 layers (3 sliding : 1 full), d=4096, 32/4 heads, f 1024, 16 x 4 tokens, 128K past
     "large": Workload("large", 16, 4096, 32, 4, 128, 1024, [1, 1, 1, 0] * 4, 16, 4, 131072, 0x5EED + 4),
 }
+# profiling stand-in for the largest workload: its layer shapes and batch,
+# two layers (sliding, full) and 8K past tokens, a few GB on the device
+PROFILE_WORKLOADS = {
+    "large2": Workload("large2", 2, 4096, 32, 4, 128, 1024, [1, 0], 16, 4, 8192, 0x5EED + 4),
+}

@@ -1,0 +1,171 @@
+"""GPU parity: the CUDA step (through the C ABI) against the fp64 oracle.
+
+Tolerances are the target's: routing sets identical unless the oracle's
+8th-9th logit gap is below 1e-3 (then the oracle is replayed with the GPU's
+routing for that token), final hidden states max-abs <= 2e-2 and rel-L2 <=
+1e-2, per-layer attention outputs rel-L2 <= 5e-3.  Sizes: the tiny, 8-layer
+decode and 8-layer verify workloads in full; a ragged multi-sequence case
+(different past lengths, an empty past, a window shorter than the context,
+chunk boundaries crossed); the long-context and largest workloads at full
+size in the benchmark's launch configuration, with the oracle on sampled
+sequences.
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import synth.gpu as sg
+import verify_step_megakernel_b200 as msk
+from synth.configs import Workload
+from tests._gpu import Engine
+from tests._parity import assert_parity, bf16_to_f64, run_parity
+
+pytestmark = pytest.mark.gpu
+
+
+def _report(name, rep):
+    print(f"\n[{name}] attn_rel max {max(rep['attn_rel']):.2e}  h_abs {rep['h_abs']:.2e}  h_rel {rep['h_rel']:.2e}"
+          f"  dh_rel {rep['dh_rel']:.2e}  route exempt {rep['n_exempt']} forced {rep['forced']}"
+          f"  kv midpoint {rep['forced_kv']}/{rep['kv_codes']} invalid {rep['kv_invalid']}")
+
+
+def _kv_written_match(w, eng, ref, positions, seqs):
+    """The fp8 K/V this step wrote equal the oracle's codes up to one e4m3
+    step where the fp32 and fp64 values straddle a rounding boundary."""
+    tps = len(positions[0])
+    kvd = w.n_kv_heads * w.head_dim
+    tot = same = 0
+    for l in range(w.n_layers):
+        for i, b in enumerate(seqs):
+            k, v = eng.read_kv(l, b, positions[b][0], tps)
+            for arr, key in ((k, "k_new"), (v, "v_new")):
+                want = ref[key][l, i * tps:(i + 1) * tps].reshape(tps, kvd)
+                tot += want.size
+                same += int((arr == want).sum())
+                a = torch.from_numpy(arr).view(torch.float8_e4m3fn).double().numpy()
+                bb = torch.from_numpy(want).view(torch.float8_e4m3fn).double().numpy()
+                assert np.all(np.abs(a - bb) <= np.maximum(np.abs(bb), 2.0 ** -6) * 0.125 + 1e-12)
+    assert same / tot > 0.9, same / tot
+
+
+@pytest.mark.parametrize("name", ["tiny", "dec8", "ver8"])
+def test_parity_workload(name):
+    w = synth.WORKLOADS[name]
+    eng = Engine(w)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    pos = w.positions()
+    rep, gpu, ref = run_parity(w, eng, hid, pos)
+    _report(name, rep)
+    assert_parity(rep)
+    _kv_written_match(w, eng, ref, pos, list(range(w.n_seqs)))
+    eng.close()
+
+
+RAGGED = Workload("ragged", 3, 256, 4, 2, 64, 128, [1, 0, 1], 3, 3, 0, 0x5EED + 40, n_experts=32, top_k=4,
+                  window=100)
+
+
+def test_parity_ragged_sequences():
+    w = RAGGED
+    past = [0, 130, 517]  # empty past, a chunk boundary crossed, window < context
+    eng = Engine(w, past_per_seq=past)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    pos = [[p + i for i in range(w.tokens_per_seq)] for p in past]
+    rep, gpu, ref = run_parity(w, eng, hid, pos)
+    _report("ragged", rep)
+    assert_parity(rep)
+    _kv_written_match(w, eng, ref, pos, [0, 1, 2])
+    eng.close()
+
+
+def test_hd128_window_edge_and_single_token_window():
+    # window 1: each query sees only itself; 128-wide heads, GQA group 4
+    w = Workload("w1", 2, 512, 8, 2, 128, 256, [1, 1], 2, 2, 300, 0x5EED + 41, n_experts=64, top_k=8, window=1)
+    eng = Engine(w)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions())
+    _report("w1", rep)
+    assert_parity(rep)
+    eng.close()
+
+
+def test_step_is_deterministic_and_repeatable():
+    w = synth.WORKLOADS["ver8"].with_(n_layers=2, sliding=[1, 0])
+    eng = Engine(w)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    a = eng.step(hid, w.positions())
+    b = eng.step(hid, w.positions())
+    assert a["status"] == 0 and b["status"] == 0
+    assert np.array_equal(a["hidden_out"], b["hidden_out"])
+    assert np.array_equal(a["attn_out"], b["attn_out"])
+    eng.close()
+
+
+def test_bad_positions_are_reported():
+    w = synth.WORKLOADS["tiny"].with_(n_seqs=1, tokens_per_seq=2)
+    eng = Engine(w)
+    hid = sg.hidden(w)
+    r = eng.step(hid, [[5, 7]])  # not contiguous
+    assert r["status"] == msk.MskError(6, "").code
+    r = eng.step(hid, [[w.past + 100, w.past + 101]])  # beyond the (rounded-up) capacity
+    assert r["status"] == 6
+    r = eng.step(hid, [[3, 4]])
+    assert r["status"] == 0
+    eng.close()
+
+
+def test_invalid_arguments_and_bound():
+    w = synth.WORKLOADS["tiny"]
+    wts = sg.DeviceWeights(w)
+    from tests._gpu import config_struct, layer_structs
+    cfg = config_struct(w)
+    cfg.head_dim = 96
+    with pytest.raises(msk.MskError) as e:
+        msk.msk_create(cfg, layer_structs(wts), 0)
+    assert e.value.code == 2
+    cfg = config_struct(w)
+    layers = layer_structs(wts)
+    big = torch.full((w.head_dim,), 2.0, dtype=torch.float32, device="cuda")  # M = 8*2*2 = 32: 2M = 64 ok
+    layers[0].q_norm_g = big.data_ptr()
+    h = msk.msk_create(cfg, layers, 0)
+    msk.msk_destroy(h)
+    bigger = torch.full((w.head_dim,), 2.5, dtype=torch.float32, device="cuda")  # M = 50: 2M >= 80
+    layers[0].q_norm_g = bigger.data_ptr()
+    layers[0].k_norm_g = bigger.data_ptr()
+    with pytest.raises(msk.MskError) as e:
+        msk.msk_create(cfg, layers, 0)
+    assert e.value.code == 5
+    layers = layer_structs(wts)
+    layers[1].wq.codes = layers[1].wq.codes + 1  # misaligned
+    with pytest.raises(msk.MskError) as e:
+        msk.msk_create(cfg, layers, 0)
+    assert e.value.code == 1
+
+
+@pytest.mark.slow
+def test_parity_long_context_sampled():
+    w = synth.WORKLOADS["long"]
+    eng = Engine(w)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions())
+    _report("long", rep)
+    assert_parity(rep)
+    eng.close()
+
+
+@pytest.mark.slow
+def test_parity_largest_sampled():
+    w = synth.WORKLOADS["large"]
+    eng = Engine(w)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions(), seqs=[0, 15])
+    _report("large", rep)
+    assert_parity(rep)
+    eng.close()

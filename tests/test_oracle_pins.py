@@ -290,3 +290,21 @@ def test_lazy_source_equals_arrays(mini):
     b = oracle.step(w, src.src.ptr, hid, w.positions(), threads=2)
     assert np.array_equal(a["h_out"], b["h_out"])
     assert np.array_equal(a["hidden_out"], b["hidden_out"])
+
+
+def test_forced_kv_code_is_used():
+    # uniform attention (W_q = 0): forcing the new token's v codes changes the
+    # mean by exactly the forced values' share
+    w, weights, pk, pv, rng = _hand()
+    h = bf16_bits(rng.standard_normal((1, 16)) + 0.5)
+    m = HandModel(w, weights, [[[pk]]], [[[pv]]])
+    a = oracle.step(w, m.src.ptr, h, w.positions(), threads=1)
+    fv = np.full((1, 1, 16), -1, np.int16)
+    fv[0, 0, 3] = 0x40  # 2.0
+    b = oracle.step(w, m.src.ptr, h, w.positions(), forced_v=fv, threads=1)
+    n = w.past + 1
+    delta = (2.0 - e4m3_values(a["v_new"][0, 0, 3:4])[0]) / n
+    assert b["attn_out"][0, 0, 3] == pytest.approx(a["attn_out"][0, 0, 3] + delta, rel=1e-13)
+    assert np.array_equal(np.delete(b["attn_out"][0, 0], 3), np.delete(a["attn_out"][0, 0], 3))
+    assert b["v_new"][0, 0, 3] == 0x40
+    assert np.allclose(a["v_pre"][0, 0], rmsnorm_ref(bf16_values(h), weights["attn_norm_g"], w.rms_eps)[0])

@@ -1,0 +1,508 @@
+/*
+ * msk_api.cu -- the C ABI declared in include/msk.h: argument checks,
+ * scratch allocation, the KV cache object with its tensor map, and the
+ * cooperative launch of the step kernel.
+ */
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <new>
+
+#include "msk_internal.h"
+
+extern "C" size_t msk_kernel_smem_bytes();
+extern "C" cudaError_t msk_kernel_setup(int hd, int* ctas_per_sm);
+extern "C" cudaError_t msk_kernel_launch(int hd, const MskParams* P_dev, const MskStep* st, const CUtensorMap* map,
+                                         int ncta, cudaStream_t stream);
+
+struct msk_handle {
+  int device;
+  int ncta;
+  msk_config_t cfg;
+  msk_layer_weights_t layers[MSK_MAX_LAYERS];
+  MskParams host;   /* mirror of the device copy */
+  MskParams* dev;   /* device copy */
+  void* scratch;    /* one allocation for every scratch buffer */
+  CUtensorMap* emaps; /* [L][6] expert tensor maps (device) */
+  size_t scratch_bytes;
+  uint32_t* words;  /* ctrl + status */
+  msk_debug_t dbg;
+  int have_last;
+};
+
+struct msk_kv {
+  msk_handle_t* h;
+  int n_seqs;
+  int64_t cap;
+  int64_t half_rows;
+  uint8_t* base;
+  CUtensorMap map;
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = (EncodeTiledFn)p;
+  }
+  return fn;
+}
+
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+static msk_status_t check_nv(const msk_nvfp4_t& w) {
+  if (!w.codes || !w.scales || !aligned16(w.codes) || !aligned16(w.scales)) return MSK_ERR_INVALID_ARG;
+  if (!(w.global_scale > 0.0f) || !isfinite(w.global_scale)) return MSK_ERR_INVALID_ARG;
+  return MSK_OK;
+}
+
+static msk_status_t check_config(const msk_config_t* c) {
+  if (c->n_layers < 1 || c->n_layers > MSK_MAX_LAYERS) return MSK_ERR_INVALID_ARG;
+  if (c->head_dim != 64 && c->head_dim != 128) return MSK_ERR_UNSUPPORTED;
+  if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads) return MSK_ERR_INVALID_ARG;
+  const int qd = c->n_q_heads * c->head_dim;
+  if (c->d_model < 128 || c->d_model % 128 || c->d_model > 4096) return MSK_ERR_UNSUPPORTED;
+  if (qd % 128 || qd > 4096) return MSK_ERR_UNSUPPORTED;
+  if (c->expert_dim < 128 || c->expert_dim % 128 || c->expert_dim > 4096) return MSK_ERR_UNSUPPORTED;
+  /* expert tiles stream K in chunks of 512 or 256: longer rows must split evenly */
+  if ((c->d_model > 512 && c->d_model % 256) || (c->expert_dim > 512 && c->expert_dim % 256))
+    return MSK_ERR_UNSUPPORTED;
+  if (c->n_experts < 32 || c->n_experts % 32 || c->n_experts > 256) return MSK_ERR_UNSUPPORTED;
+  if (c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return MSK_ERR_INVALID_ARG;
+  if (c->window < 1) return MSK_ERR_INVALID_ARG;
+  if (!(c->rms_eps >= 0.0f)) return MSK_ERR_INVALID_ARG;
+  if (c->max_seqs < 1 || c->max_tokens_per_seq < 1) return MSK_ERR_INVALID_ARG;
+  if (c->max_seqs * c->max_tokens_per_seq > MSK_MAX_TOKENS) return MSK_ERR_UNSUPPORTED;
+  if (c->max_tokens_per_seq * (c->n_q_heads / c->n_kv_heads) > 64) return MSK_ERR_UNSUPPORTED;
+  if (c->max_seqs * c->n_kv_heads > MSK_MAX_PAIRS) return MSK_ERR_UNSUPPORTED;
+  if (c->wait_timeout_us < 0) return MSK_ERR_INVALID_ARG;
+  return MSK_OK;
+}
+
+extern "C" {
+
+const char* msk_status_string(msk_status_t s) {
+  switch (s) {
+    case MSK_OK: return "ok";
+    case MSK_ERR_INVALID_ARG: return "invalid argument";
+    case MSK_ERR_UNSUPPORTED: return "unsupported device or shape";
+    case MSK_ERR_OOM: return "out of device memory";
+    case MSK_ERR_CUDA: return "CUDA error";
+    case MSK_ERR_BOUND: return "softmax bound 2M >= 80";
+    case MSK_ERR_KV_RANGE: return "positions outside the KV cache or not contiguous";
+    case MSK_ERR_TIMEOUT: return "device wait timed out";
+    case MSK_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* layers, int device,
+                        msk_handle_t** out) {
+  if (!config || !layers || !out) return MSK_ERR_INVALID_ARG;
+  *out = nullptr;
+  msk_status_t st = check_config(config);
+  if (st) return st;
+  for (int l = 0; l < config->n_layers; ++l) {
+    const msk_layer_weights_t& w = layers[l];
+    if (!w.attn_norm_g || !w.q_norm_g || !w.k_norm_g || !w.moe_norm_g || !w.router) return MSK_ERR_INVALID_ARG;
+    if (!aligned16(w.attn_norm_g) || !aligned16(w.moe_norm_g) || !aligned16(w.router) || !aligned16(w.q_norm_g) ||
+        !aligned16(w.k_norm_g))
+      return MSK_ERR_INVALID_ARG;
+    const msk_nvfp4_t* nvs[7] = {&w.wq, &w.wk, &w.wv, &w.wo, &w.w_gate, &w.w_up, &w.w_down};
+    for (auto* nv : nvs)
+      if ((st = check_nv(*nv))) return st;
+  }
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || device < 0 || device >= ndev) return MSK_ERR_UNSUPPORTED;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (cudaSetDevice(device) != cudaSuccess) return MSK_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) { cudaSetDevice(prev); return MSK_ERR_CUDA; }
+  if (prop.major != 10 || !prop.cooperativeLaunch) { cudaSetDevice(prev); return MSK_ERR_UNSUPPORTED; }
+  int per_sm = 0;
+  if (msk_kernel_setup(config->head_dim, &per_sm) != cudaSuccess || per_sm < 1) { cudaSetDevice(prev); return MSK_ERR_UNSUPPORTED; }
+
+  msk_handle_t* h = new (std::nothrow) msk_handle_t();
+  if (!h) { cudaSetDevice(prev); return MSK_ERR_OOM; }
+  h->device = device;
+  h->ncta = prop.multiProcessorCount; /* one persistent CTA per SM */
+  h->cfg = *config;
+  memcpy(h->layers, layers, sizeof(msk_layer_weights_t) * config->n_layers);
+
+  MskParams& P = h->host;
+  memset(&P, 0, sizeof P);
+  const msk_config_t& c = *config;
+  P.L = c.n_layers; P.d = c.d_model; P.hq = c.n_q_heads; P.hkv = c.n_kv_heads; P.hd = c.head_dim;
+  P.E = c.n_experts; P.k = c.top_k; P.f = c.expert_dim; P.W = c.window; P.G = c.n_q_heads / c.n_kv_heads;
+  P.qd = P.hq * P.hd; P.kvd = P.hkv * P.hd;
+  P.ncta = h->ncta;
+  P.max_T = c.max_seqs * c.max_tokens_per_seq;
+  P.eps = c.rms_eps;
+  P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)P.hd));
+  P.timeout_ns = (int64_t)(c.wait_timeout_us ? c.wait_timeout_us : 2000000) * 1000;
+  P.flags = c.flags;
+
+  /* the fixed softmax shift of each layer, from its QK-norm gains */
+  float* gq = (float*)malloc(sizeof(float) * P.hd);
+  float* gk = (float*)malloc(sizeof(float) * P.hd);
+  st = MSK_OK;
+  for (int l = 0; l < P.L && st == MSK_OK; ++l) {
+    if (cudaMemcpy(gq, layers[l].q_norm_g, sizeof(float) * P.hd, cudaMemcpyDeviceToHost) != cudaSuccess ||
+        cudaMemcpy(gk, layers[l].k_norm_g, sizeof(float) * P.hd, cudaMemcpyDeviceToHost) != cudaSuccess) {
+      st = MSK_ERR_CUDA;
+      break;
+    }
+    double mq = 0, mk = 0;
+    for (int i = 0; i < P.hd; ++i) { mq = fmax(mq, fabs(gq[i])); mk = fmax(mk, fabs(gk[i])); }
+    const double M = sqrt((double)P.hd) * mq * mk;
+    if (!(2.0 * M < 80.0)) st = MSK_ERR_BOUND;
+    MskLayer& Ly = P.layers[l];
+    const msk_layer_weights_t& w = layers[l];
+    Ly.g_attn = w.attn_norm_g; Ly.g_q = w.q_norm_g; Ly.g_k = w.k_norm_g; Ly.g_moe = w.moe_norm_g; Ly.router = w.router;
+    auto nv = [](const msk_nvfp4_t& x) { MskNv r; r.codes = x.codes; r.scales = x.scales; r.gs = x.global_scale; r.pad = 0; return r; };
+    Ly.wq = nv(w.wq); Ly.wk = nv(w.wk); Ly.wv = nv(w.wv); Ly.wo = nv(w.wo);
+    Ly.wg = nv(w.w_gate); Ly.wu = nv(w.w_up); Ly.wd = nv(w.w_down);
+    Ly.bound_log2 = (float)(M * 1.4426950408889634);
+    Ly.sliding = c.layer_is_sliding[l] ? 1 : 0;
+  }
+  free(gq);
+  free(gk);
+  if (st) { delete h; cudaSetDevice(prev); return st; }
+
+  /* scratch */
+  const size_t T = (size_t)P.max_T, d = P.d, qd = P.qd, kvd = P.kvd;
+  const size_t R_max = (size_t)c.max_tokens_per_seq * P.G;
+  P.part_stride = (int32_t)(R_max * (P.hd + 4));
+  const size_t slots = (size_t)h->ncta + (size_t)c.max_seqs * P.hkv;
+  size_t sizes[] = {
+      T * d * 4,                 /* h */
+      T * d * 2,                 /* x */
+      T * (qd + 2 * kvd) * 4,    /* qkv */
+      T * qd * 2,                /* qs */
+      slots * P.part_stride * 4, /* part */
+      T * qd * 2,                /* o */
+      T * d * 4,                 /* x2f */
+      T * d * 2,                 /* x2h */
+      T * P.E * 4,               /* logits */
+      T * P.k * P.f * 2,         /* u */
+      T * P.k * d * 4,           /* y */
+      (CTRL_WORDS + ST_WORDS) * 4,
+      (size_t)P.L * 4,           /* n_distinct */
+      (2 + MSK_MAX_TOKENS) * 4,  /* last_shape */
+  };
+  const int nbuf = sizeof(sizes) / sizeof(sizes[0]);
+  size_t off[16], total = 0;
+  for (int i = 0; i < nbuf; ++i) { off[i] = total; total += (sizes[i] + 255) & ~(size_t)255; }
+  if (cudaMalloc(&h->scratch, total) != cudaSuccess) { delete h; cudaSetDevice(prev); return MSK_ERR_OOM; }
+  cudaMemset(h->scratch, 0, total);
+  h->scratch_bytes = total;
+  uint8_t* b = (uint8_t*)h->scratch;
+  P.h = (float*)(b + off[0]);
+  P.x = (uint16_t*)(b + off[1]);
+  P.qkv = (float*)(b + off[2]);
+  P.qs = (uint16_t*)(b + off[3]);
+  P.part = (float*)(b + off[4]);
+  P.o = (uint16_t*)(b + off[5]);
+  P.x2f = (float*)(b + off[6]);
+  P.x2h = (uint16_t*)(b + off[7]);
+  P.logits = (float*)(b + off[8]);
+  P.u = (uint16_t*)(b + off[9]);
+  P.y = (float*)(b + off[10]);
+  P.ctrl = (uint32_t*)(b + off[11]);
+  P.status = P.ctrl + CTRL_WORDS;
+  P.n_distinct = (int32_t*)(b + off[12]);
+  P.last_shape = (int32_t*)(b + off[13]);
+  h->words = P.ctrl;
+  /* tensor maps of the expert tensors, for the K-chunked expert tiles */
+  {
+    EncodeTiledFn enc = encode_fn();
+    CUtensorMap* hm = (CUtensorMap*)calloc((size_t)P.L * 6, sizeof(CUtensorMap));
+    bool ok = enc != nullptr && hm != nullptr && cudaMalloc(&h->emaps, sizeof(CUtensorMap) * 6 * P.L) == cudaSuccess;
+    for (int l = 0; l < P.L && ok; ++l) {
+      const msk_layer_weights_t& w = layers[l];
+      const msk_nvfp4_t* mats[3] = {&w.w_gate, &w.w_up, &w.w_down};
+      for (int m = 0; m < 3 && ok; ++m) {
+        const int64_t K = m < 2 ? P.d : P.f, rows = (int64_t)P.E * (m < 2 ? P.f : P.d);
+        const int KC = K <= 512 ? (int)K : (K % 512 == 0 ? 512 : 256);
+        for (int part = 0; part < 2 && ok; ++part) {
+          /* whole-row chunks use plain bulk copies; the map is left zero */
+          if (K <= 512) continue;
+          const int64_t width = part == 0 ? K / 2 : K / 16;
+          cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+          cuuint64_t strides[1] = {(cuuint64_t)width};
+          cuuint32_t box[2] = {(cuuint32_t)(part == 0 ? KC / 2 : KC / 16), 16};
+          cuuint32_t estr[2] = {1, 1};
+          void* base = (void*)(part == 0 ? mats[m]->codes : mats[m]->scales);
+          ok = enc(&hm[l * 6 + m * 2 + part], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        }
+      }
+      P.layers[l].emap = h->emaps + l * 6;
+    }
+    if (ok) ok = cudaMemcpy(h->emaps, hm, sizeof(CUtensorMap) * 6 * P.L, cudaMemcpyHostToDevice) == cudaSuccess;
+    free(hm);
+    if (!ok) {
+      if (h->emaps) cudaFree(h->emaps);
+      cudaFree(h->scratch);
+      delete h;
+      cudaSetDevice(prev);
+      return MSK_ERR_CUDA;
+    }
+  }
+  if (cudaMalloc(&h->dev, sizeof(MskParams)) != cudaSuccess) {
+    cudaFree(h->emaps);
+    cudaFree(h->scratch);
+    delete h;
+    cudaSetDevice(prev);
+    return MSK_ERR_OOM;
+  }
+  if (cudaMemcpy(h->dev, &P, sizeof(MskParams), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(h->dev);
+    cudaFree(h->emaps);
+    cudaFree(h->scratch);
+    delete h;
+    cudaSetDevice(prev);
+    return MSK_ERR_CUDA;
+  }
+  cudaSetDevice(prev);
+  *out = h;
+  return MSK_OK;
+}
+
+void msk_destroy(msk_handle_t* h) {
+  if (!h) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  cudaFree(h->dev);
+  cudaFree(h->scratch);
+  cudaFree(h->emaps);
+  cudaSetDevice(prev);
+  delete h;
+}
+
+msk_status_t msk_kv_create(msk_handle_t* h, int n_seqs, int64_t capacity, msk_kv_t** out) {
+  if (!h || !out || n_seqs < 1 || capacity < 1) return MSK_ERR_INVALID_ARG;
+  *out = nullptr;
+  if (n_seqs > h->cfg.max_seqs) return MSK_ERR_INVALID_ARG;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return MSK_ERR_CUDA;
+  const MskParams& P = h->host;
+  const int64_t cap = (capacity + 15) / 16 * 16;
+  const int64_t half_rows = (int64_t)P.L * n_seqs * P.hkv * cap;
+  if (2 * half_rows >= ((int64_t)1 << 31)) return MSK_ERR_UNSUPPORTED; /* tensor-copy coordinates are int32 */
+  const size_t bytes = (size_t)(2 * half_rows) * P.hd;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  msk_kv_t* kv = new (std::nothrow) msk_kv_t();
+  if (!kv) { cudaSetDevice(prev); return MSK_ERR_OOM; }
+  kv->h = h;
+  kv->n_seqs = n_seqs;
+  kv->cap = cap;
+  kv->half_rows = half_rows;
+  if (cudaMalloc(&kv->base, bytes) != cudaSuccess) { delete kv; cudaSetDevice(prev); return MSK_ERR_OOM; }
+  /* zero: unwritten positions must decode to finite values (masked keys
+   * still pass through the tensor-core tile as 0 * v) */
+  if (cudaMemset(kv->base, 0, bytes) != cudaSuccess || cudaDeviceSynchronize() != cudaSuccess) {
+    cudaFree(kv->base);
+    delete kv;
+    cudaSetDevice(prev);
+    return MSK_ERR_CUDA;
+  }
+  const int C = P.hd == 128 ? 128 : 256;
+  cuuint64_t dims[2] = {(cuuint64_t)P.hd, (cuuint64_t)(2 * half_rows)};
+  cuuint64_t strides[1] = {(cuuint64_t)P.hd};
+  cuuint32_t box[2] = {(cuuint32_t)P.hd, (cuuint32_t)C};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&kv->map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->base, dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   P.hd == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  cudaSetDevice(prev);
+  if (r != CUDA_SUCCESS) {
+    cudaFree(kv->base);
+    delete kv;
+    return MSK_ERR_CUDA;
+  }
+  *out = kv;
+  return MSK_OK;
+}
+
+void msk_kv_destroy(msk_kv_t* kv) {
+  if (!kv) return;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(kv->h->device);
+  cudaDeviceSynchronize();
+  cudaFree(kv->base);
+  cudaSetDevice(prev);
+  delete kv;
+}
+
+static int64_t kv_row(const msk_kv_t* kv, int layer, int seq, int head, int64_t pos) {
+  const MskParams& P = kv->h->host;
+  return (((int64_t)layer * kv->n_seqs + seq) * P.hkv + head) * kv->cap + pos;
+}
+
+msk_status_t msk_kv_append(msk_handle_t* h, msk_kv_t* kv, int layer, int seq, int64_t pos0, int64_t n,
+                           const uint8_t* k_fp8, const uint8_t* v_fp8, void* stream) {
+  if (!h || !kv || kv->h != h || !k_fp8 || !v_fp8) return MSK_ERR_INVALID_ARG;
+  const MskParams& P = h->host;
+  if (layer < 0 || layer >= P.L || seq < 0 || seq >= kv->n_seqs || pos0 < 0 || n < 0) return MSK_ERR_INVALID_ARG;
+  if (pos0 + n > kv->cap) return MSK_ERR_KV_RANGE;
+  if (n == 0) return MSK_OK;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaSuccess;
+  for (int hh = 0; hh < P.hkv && e == cudaSuccess; ++hh) {
+    for (int kvsel = 0; kvsel < 2 && e == cudaSuccess; ++kvsel) {
+      uint8_t* dst = kv->base + (kv_row(kv, layer, seq, hh, pos0) + (kvsel ? kv->half_rows : 0)) * P.hd;
+      const uint8_t* src = (kvsel ? v_fp8 : k_fp8) + (size_t)hh * P.hd;
+      e = cudaMemcpy2DAsync(dst, P.hd, src, (size_t)P.hkv * P.hd, P.hd, (size_t)n, cudaMemcpyDefault,
+                            (cudaStream_t)stream);
+    }
+  }
+  cudaSetDevice(prev);
+  return e == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
+}
+
+msk_status_t msk_kv_read(msk_handle_t* h, msk_kv_t* kv, int layer, int seq, int64_t pos0, int64_t n, uint8_t* k_out,
+                         uint8_t* v_out) {
+  if (!h || !kv || kv->h != h || !k_out || !v_out) return MSK_ERR_INVALID_ARG;
+  const MskParams& P = h->host;
+  if (layer < 0 || layer >= P.L || seq < 0 || seq >= kv->n_seqs || pos0 < 0 || n < 0) return MSK_ERR_INVALID_ARG;
+  if (pos0 + n > kv->cap) return MSK_ERR_KV_RANGE;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  for (int hh = 0; hh < P.hkv && e == cudaSuccess; ++hh) {
+    for (int kvsel = 0; kvsel < 2 && e == cudaSuccess; ++kvsel) {
+      const uint8_t* src = kv->base + (kv_row(kv, layer, seq, hh, pos0) + (kvsel ? kv->half_rows : 0)) * P.hd;
+      uint8_t* dst = (kvsel ? v_out : k_out) + (size_t)hh * P.hd;
+      e = cudaMemcpy2D(dst, (size_t)P.hkv * P.hd, src, P.hd, P.hd, (size_t)n, cudaMemcpyDefault);
+    }
+  }
+  cudaSetDevice(prev);
+  return e == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
+}
+
+msk_status_t msk_step(msk_handle_t* h, const uint16_t* hidden_in, const int32_t* positions, int n_seqs,
+                      int tokens_per_seq, msk_kv_t* kv, uint16_t* hidden_out, void* stream) {
+  if (!h || !hidden_in || !positions || !kv || !hidden_out || kv->h != h) return MSK_ERR_INVALID_ARG;
+  if (n_seqs < 1 || tokens_per_seq < 1 || n_seqs > h->cfg.max_seqs || tokens_per_seq > h->cfg.max_tokens_per_seq ||
+      n_seqs > kv->n_seqs)
+    return MSK_ERR_INVALID_ARG;
+  if (!aligned16(hidden_in) || !aligned16(hidden_out) || ((uintptr_t)positions & 3u)) return MSK_ERR_INVALID_ARG;
+  const MskParams& P = h->host;
+  MskStep st;
+  st.hidden_in = hidden_in;
+  st.positions = positions;
+  st.hidden_out = hidden_out;
+  st.kv_base = kv->base;
+  st.kv_cap = kv->cap;
+  st.kv_half_rows = kv->half_rows;
+  st.kv_seqs = kv->n_seqs;
+  st.S = n_seqs;
+  st.Tq = tokens_per_seq;
+  st.T = n_seqs * tokens_per_seq;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != h->device) cudaSetDevice(h->device);
+  cudaError_t e = cudaMemsetAsync(P.ctrl, 0, CTRL_WORDS * 4, (cudaStream_t)stream);
+  if (e == cudaSuccess) e = msk_kernel_launch(P.hd, h->dev, &st, &kv->map, h->ncta, (cudaStream_t)stream);
+  if (prev != h->device) cudaSetDevice(prev);
+  h->have_last = 1;
+  return e == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
+}
+
+msk_status_t msk_step_status(msk_handle_t* h) {
+  if (!h) return MSK_ERR_INVALID_ARG;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  uint32_t w[ST_WORDS];
+  cudaError_t e = cudaMemcpy(w, h->host.status, sizeof w, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(h->host.status, 0, sizeof w);
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) return MSK_ERR_CUDA;
+  return (msk_status_t)w[ST_CODE];
+}
+
+msk_status_t msk_set_debug(msk_handle_t* h, const msk_debug_t* dbg) {
+  if (!h) return MSK_ERR_INVALID_ARG;
+  MskParams& P = h->host;
+  msk_debug_t z;
+  memset(&z, 0, sizeof z);
+  const msk_debug_t& d = dbg ? *dbg : z;
+  P.dbg_ids = d.route_ids;
+  P.dbg_w = d.route_w;
+  P.dbg_logits = d.logits;
+  P.dbg_attn = d.attn_out;
+  P.dbg_trace = d.trace;
+  h->dbg = d;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaMemcpy(h->dev, &P, sizeof(MskParams), cudaMemcpyHostToDevice);
+  cudaSetDevice(prev);
+  return e == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
+}
+
+msk_status_t msk_query(msk_handle_t* h, msk_stats_t* out) {
+  if (!h || !out) return MSK_ERR_INVALID_ARG;
+  memset(out, 0, sizeof *out);
+  const MskParams& P = h->host;
+  out->n_layers = P.L;
+  out->scratch_bytes = (int64_t)h->scratch_bytes;
+  if (!h->have_last) return MSK_OK;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  cudaSetDevice(h->device);
+  cudaError_t e = cudaDeviceSynchronize();
+  int32_t shape[2 + MSK_MAX_TOKENS];
+  if (e == cudaSuccess) e = cudaMemcpy(out->n_distinct, P.n_distinct, sizeof(int32_t) * P.L, cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemcpy(shape, P.last_shape, sizeof shape, cudaMemcpyDeviceToHost);
+  cudaSetDevice(prev);
+  if (e != cudaSuccess) return MSK_ERR_CUDA;
+  /* bytes the step must move at least once: each weight it uses, each KV
+   * position it attends (the union over a sequence's rows) and writes, and
+   * the hidden states in and out */
+  const int64_t d = P.d, qd = P.qd, kvd = P.kvd, f = P.f;
+  auto nvb = [](int64_t n) { return n / 2 + n / 16; }; /* NVFP4 bytes of n values */
+  int64_t wbytes = 0, kvbytes = 0;
+  const int S = shape[0], Tq = shape[1], T = S * Tq;
+  for (int l = 0; l < P.L; ++l) {
+    wbytes += nvb(qd * d) + 2 * nvb(kvd * d) + nvb(d * qd) + (int64_t)P.E * d * 4;
+    wbytes += (int64_t)out->n_distinct[l] * (3 * nvb(d * f));
+    for (int b_ = 0; b_ < S; ++b_) {
+      const int64_t p0 = shape[2 + b_], last = p0 + Tq - 1;
+      int64_t lo = 0;
+      if (P.layers[l].sliding) { lo = p0 - P.W + 1; if (lo < 0) lo = 0; }
+      kvbytes += P.hkv * (last - lo + 1) * 2 * P.hd; /* K and V read */
+    }
+    kvbytes += (int64_t)T * 2 * kvd; /* K and V written */
+  }
+  out->weight_bytes = wbytes;
+  out->kv_bytes = kvbytes;
+  out->algorithmic_bytes = wbytes + kvbytes + (int64_t)T * d * 2 * 2;
+  return MSK_OK;
+}
+
+}  // extern "C"

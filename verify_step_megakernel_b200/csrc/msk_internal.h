@@ -1,0 +1,92 @@
+/*
+ * msk_internal.h -- structures shared by the host launcher and the
+ * persistent step kernel (not part of the public ABI).
+ */
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "../../include/msk.h"
+
+/* CTA shape: warpgroup 0 is the producer (one thread issues the bulk/TMA
+ * copies into the ring; the group gives its registers back), warpgroups 1-2
+ * are MSK_NCW consumer warps (tensor-core tiles, norms, routing). */
+#define MSK_NCW 8
+#define MSK_NTHREADS ((MSK_NCW + 4) * 32)
+#define MSK_NST 5            /* ring stages */
+#define MSK_STAGE 36864      /* bytes per stage: 16 rows x 4096 NVFP4 + scales */
+#define MSK_SCR 32768        /* consumer scratch: split-K / key-split reductions */
+#define MSK_NT_DENSE 8       /* n-tiles of 8 tokens: dense projections, T <= 64 */
+#define MSK_UNIT_TOK 8       /* tokens of an expert unit (one 8-column n-tile) */
+#define MSK_MAX_UNITS 512    /* expert units per layer (T*k <= 512) */
+#define MSK_MAX_PAIRS 64     /* (sequence, kv-head) attention pairs */
+
+/* per-step control words (zeroed before every launch) */
+enum { CTRL_BARRIER = 0, CTRL_ABORT = 1, CTRL_WORDS = 32 };
+/* persistent status words (cleared by msk_step_status) */
+enum { ST_CODE = 0, ST_WHERE = 1, ST_WORDS = 4 };
+
+typedef struct MskNv {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  float gs;
+  int32_t pad;
+} MskNv;
+
+typedef struct MskLayer {
+  const float* g_attn;
+  const float* g_q;
+  const float* g_k;
+  const float* g_moe;
+  const float* router;
+  MskNv wq, wk, wv, wo, wg, wu, wd;
+  /* 2-D tensor maps of the expert tensors for K-chunked tiles (device):
+   * gate codes, gate scales, up codes, up scales, down codes, down scales */
+  const CUtensorMap* emap;
+  float bound_log2; /* M * log2(e), M = sqrt(hd) max|g_q| max|g_k| */
+  int32_t sliding;
+} MskLayer;
+
+typedef struct MskParams {
+  int32_t L, d, hq, hkv, hd, E, k, f, W, G, qd, kvd;
+  int32_t ncta, max_T;
+  float eps, scale_log2; /* 1/sqrt(hd) * log2(e) */
+  int64_t timeout_ns;
+  uint32_t flags;
+  /* scratch (device) */
+  float* h;         /* [T][d] residual */
+  uint16_t* x;      /* [T][d] f16 attention-norm input of the projections */
+  float* qkv;       /* [T][qd + 2 kvd] raw projections */
+  uint16_t* qs;     /* [T][qd] f16 normalised queries */
+  float* part;      /* [slots][R_max][hd + 4] attention partials */
+  uint16_t* o;      /* [T][qd] f16 attention output */
+  float* x2f;       /* [T][d] moe-norm output, fp32 (router) */
+  uint16_t* x2h;    /* [T][d] same, f16 (experts) */
+  float* logits;    /* [T][E] */
+  uint16_t* u;      /* [T*k][f] f16 SwiGLU activations */
+  float* y;         /* [T*k][d] expert outputs */
+  uint32_t* ctrl;   /* CTRL_WORDS, zeroed per step */
+  uint32_t* status; /* ST_WORDS */
+  int32_t* n_distinct; /* [L] */
+  int32_t* last_shape; /* [2 + MSK_MAX_TOKENS]: S, Tq, first position of each sequence */
+  int32_t part_stride; /* floats per partial slot */
+  /* debug capture (may be null) */
+  int16_t* dbg_ids;
+  float* dbg_w;
+  float* dbg_logits;
+  float* dbg_attn;
+  uint64_t* dbg_trace;
+  MskLayer layers[MSK_MAX_LAYERS];
+} MskParams;
+
+typedef struct MskStep {
+  const uint16_t* hidden_in;
+  const int32_t* positions;
+  uint16_t* hidden_out;
+  uint8_t* kv_base;        /* K region; V region starts kv_half_rows rows later */
+  int64_t kv_cap;
+  int64_t kv_half_rows;    /* L * kv_seqs * hkv * cap */
+  int32_t kv_seqs;
+  int32_t S, Tq, T;
+} MskStep;

@@ -1,0 +1,1448 @@
+/*
+ * msk_kernel.cu -- the persistent, cooperative decode/verify-step kernel.
+ *
+ * One launch runs every layer of the step (the pages' "one program replaces
+ * many kernel boundaries"): one CTA per SM, each with one producer warp that
+ * streams weight tiles (cp.async.bulk) and KV chunks (2-D tensor copies,
+ * 128-byte swizzle) into a ring of shared-memory stages guarded by
+ * mbarriers, and eight consumer warps that run the math.  The producer runs
+ * ahead across phase and layer boundaries: the next phase's dense weights
+ * and the past keys are in flight while the consumers wait at a grid
+ * barrier; expert tiles are issued as soon as this CTA has resolved the
+ * top-k routing (the pages' "dense weights are streamed through a ring of
+ * tiles, selected expert weights are requested as soon as routing
+ * finishes").
+ *
+ * Per layer (grid barriers marked |):
+ *   QKV projection | QK-norm + fp8 KV write | split-sequence attention with
+ *   the fixed softmax bound | chunk combine | W_o + residual | MoE RMSNorm |
+ *   router logits | top-k (every CTA, redundantly) + gate/up + SwiGLU |
+ *   down projection | weighted combine + next RMSNorm |
+ * NVFP4 products run on the tensor cores (mma.sync m16n8k16, f16 operands,
+ * fp32 accumulate): each e2m1 code times its e4m3 block scale is exact in
+ * f16, the fp32 global scale is applied to the accumulator.
+ *
+ * Every wait is bounded by params.timeout_ns; a wait that gives up records
+ * MSK_ERR_TIMEOUT and sets an abort word every other wait polls, so the
+ * kernel always returns.
+ */
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "msk_device.cuh"
+#include "msk_internal.h"
+
+namespace {
+
+constexpr int NCW = MSK_NCW;
+constexpr int NCT = MSK_NCW * 32;  /* consumer threads */
+constexpr int BAR_CONS = 1;        /* named barrier of the consumer warps */
+constexpr int CONS_WARP0 = 4;      /* warpgroup 0 produces, warpgroups 1-2 consume */
+constexpr int CONS0 = CONS_WARP0 * 32;
+/* registers per thread after the split; 128*40 + 256*224 must not exceed
+ * the launch pool 384 * (launch registers), checked by the host */
+constexpr int REGS_PRODUCER = 40;
+constexpr int REGS_CONSUMER = 224;
+
+enum Phase {
+  PH_IN = 0, PH_QKV, PH_QKNORM, PH_ATT, PH_ATTC, PH_WO, PH_MOENORM, PH_ROUTER, PH_TOPK, PH_GU, PH_DN, PH_COMB
+};
+
+struct Route {
+  int n_units, n_distinct;
+  int16_t ids[MSK_MAX_TOKENS * 8];
+  float w[MSK_MAX_TOKENS * 8];
+  int16_t cnt[256];
+  int16_t start[257];
+  int16_t pairs[MSK_MAX_TOKENS * 8];  /* (token*k + slot), grouped by expert */
+  int16_t unit_e[MSK_MAX_UNITS];
+  int16_t unit_start[MSK_MAX_UNITS];  /* into pairs[] */
+  int16_t unit_n[MSK_MAX_UNITS];
+};
+
+constexpr int WKC_MAX = 512;                              /* K chunk of a per-warp expert tile */
+constexpr int NWS = 2;                                    /* per-warp expert ring depth */
+constexpr int WSLOT = 2 * 16 * (WKC_MAX / 2 + WKC_MAX / 16); /* gate+up 16-row chunk: 9216 B */
+static_assert(MSK_NCW * NWS * WSLOT <= MSK_NST * MSK_STAGE, "per-warp expert rings live in the stage ring");
+
+struct Smem {
+  uint64_t full[MSK_NST];
+  uint64_t empty[MSK_NST];
+  uint64_t wfull[MSK_NCW][NWS]; /* per consumer warp: expert chunk landed */
+  volatile int kv_ready;    /* layer+1 whose KV writes all CTAs finished */
+  volatile int route_ready; /* layer+1 whose routing this CTA resolved */
+  volatile int ring_free;   /* layer+1 whose expert phases released the ring */
+  volatile int abort;
+  int pos0[MSK_MAX_TOKENS];
+  float lbuf[4][32][2];
+  Route route;
+};
+
+constexpr size_t SMEM_BYTES = 1024 + (size_t)MSK_NST * MSK_STAGE + MSK_SCR + sizeof(Smem);
+
+/* ---- context ---------------------------------------------------------------------- */
+struct Ctx {
+  const MskParams* P;
+  MskStep st;
+  const CUtensorMap* kvmap;
+  uint8_t* ring;
+  float* scr;
+  Smem* S;
+  int cta, ncta;
+  uint32_t nbar; /* grid barriers passed */
+};
+
+MSK_DEV bool aborted(const Ctx& c) {
+  return c.S->abort || ld_volatile_u32(&c.P->ctrl[CTRL_ABORT]) != 0;
+}
+
+MSK_DEV void raise_err(const Ctx& c, uint32_t code, int layer, int phase) {
+  if (atomicCAS(&c.P->status[ST_CODE], 0u, code) == 0u)
+    c.P->status[ST_WHERE] = ((uint32_t)layer << 16) | ((uint32_t)phase << 8) | (uint32_t)(c.cta & 0xFF);
+  atomicExch(&c.P->ctrl[CTRL_ABORT], 1u);
+  c.S->abort = 1;
+}
+
+/* bounded mbarrier wait; false on timeout or abort */
+MSK_DEV bool wait_bar(const Ctx& c, uint64_t* bar, uint32_t parity, int layer, int phase) {
+  if (mbar_try(bar, parity)) return true;
+  uint64_t t0 = gtimer();
+  for (uint32_t it = 0;; ++it) {
+    if (mbar_try(bar, parity)) return true;
+    if ((it & 63) == 0) {
+      if (aborted(c)) return false;
+      if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+        raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
+        return false;
+      }
+    }
+  }
+}
+
+/* consumer-only grid barrier; false if the step is being aborted */
+MSK_DEV bool grid_sync(Ctx& c, int layer, int phase) {
+  named_sync(BAR_CONS, NCT);
+  __shared__ int s_ok;
+  if (threadIdx.x == CONS0) {
+    int ok = !c.S->abort;
+    if (ok) {
+      __threadfence();
+      atomicAdd(&c.P->ctrl[CTRL_BARRIER], 1u);
+      uint32_t target = (c.nbar + 1) * (uint32_t)c.ncta;
+      uint64_t t0 = gtimer();
+      while (ld_acquire_u32(&c.P->ctrl[CTRL_BARRIER]) < target) {
+        if (ld_volatile_u32(&c.P->ctrl[CTRL_ABORT])) { ok = 0; break; }
+        if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+          raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+      __threadfence();
+    }
+    if (!ok) c.S->abort = 1;
+    s_ok = ok;
+  }
+  named_sync(BAR_CONS, NCT);
+  c.nbar++;
+  if (c.P->dbg_trace && c.cta == 0 && threadIdx.x == CONS0 && layer >= 0)
+    c.P->dbg_trace[layer * 16 + phase] = gtimer();
+  return s_ok != 0;
+}
+
+/* ---- schedule: which stages this CTA streams, in order ---------------------------- */
+MSK_DEV int rows_per_stage(int K) {
+  int m = MSK_STAGE / (16 * (K / 2 + K / 16));
+  return 16 * (m < 1 ? 1 : (m > 8 ? 8 : m));
+}
+
+struct WStage { /* a weight stage: nrows x K NVFP4 rows starting at row0 */
+  const uint8_t* codes;
+  const uint8_t* scales;
+  int nrows, K;
+  int mat;  /* QKV: 0 q, 1 k, 2 v; GU: 0 gate, 1 up */
+  int row0; /* row within the (expert's) matrix */
+  int unit; /* expert unit (GU / DN) */
+  float gs;
+};
+
+MSK_DEV int qkv_stages(const MskParams* P, int* sQ, int* sK) {
+  int r = rows_per_stage(P->d);
+  *sQ = (P->qd + r - 1) / r;
+  *sK = (P->kvd + r - 1) / r;
+  return *sQ + 2 * *sK;
+}
+
+MSK_DEV WStage qkv_stage(const MskParams* P, const MskLayer& Ly, int j, int sQ, int sK) {
+  int r = rows_per_stage(P->d);
+  WStage s;
+  const MskNv* nv;
+  int rows;
+  if (j < sQ) { s.mat = 0; nv = &Ly.wq; rows = P->qd; }
+  else if (j < sQ + sK) { s.mat = 1; nv = &Ly.wk; j -= sQ; rows = P->kvd; }
+  else { s.mat = 2; nv = &Ly.wv; j -= sQ + sK; rows = P->kvd; }
+  s.row0 = j * r;
+  s.nrows = min(r, rows - s.row0);
+  s.K = P->d;
+  s.codes = nv->codes + (int64_t)s.row0 * (P->d / 2);
+  s.scales = nv->scales + (int64_t)s.row0 * (P->d / 16);
+  s.gs = nv->gs;
+  s.unit = 0;
+  return s;
+}
+
+MSK_DEV WStage wo_stage(const MskParams* P, const MskLayer& Ly, int j) {
+  int r = rows_per_stage(P->qd);
+  WStage s;
+  s.mat = 0;
+  s.row0 = j * r;
+  s.nrows = min(r, P->d - s.row0);
+  s.K = P->qd;
+  s.codes = Ly.wo.codes + (int64_t)s.row0 * (P->qd / 2);
+  s.scales = Ly.wo.scales + (int64_t)s.row0 * (P->qd / 16);
+  s.gs = Ly.wo.gs;
+  s.unit = 0;
+  return s;
+}
+
+/* expert stages: items = unit x row block, contiguous ranges per CTA */
+MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
+  *a = (int)((int64_t)n * cta / ncta);
+  *b = (int)((int64_t)n * (cta + 1) / ncta);
+}
+
+/* attention key space of one layer: pairs (seq, kv head) in order, each
+ * with the union of its rows' key ranges; CTA c owns [c N / n, (c+1) N / n) */
+struct AttGeo {
+  int npairs;
+  int nparts; /* CTAs that take part: each gets >= 2 stages of keys when possible */
+  int64_t N;
+  int64_t lo[MSK_MAX_PAIRS];  /* first key position of the pair */
+  int64_t off[MSK_MAX_PAIRS + 1]; /* prefix sums of key counts */
+};
+MSK_DEV void att_geo(const Ctx& c, int layer, AttGeo& g) {
+  const MskParams* P = c.P;
+  g.npairs = c.st.S * P->hkv;
+  g.off[0] = 0;
+  for (int p = 0; p < g.npairs; ++p) {
+    int b = p / P->hkv;
+    int64_t first = c.S->pos0[b];
+    int64_t last = first + c.st.Tq - 1;
+    int64_t lo = 0;
+    if (P->layers[layer].sliding) { lo = first - P->W + 1; if (lo < 0) lo = 0; }
+    g.lo[p] = lo;
+    g.off[p + 1] = g.off[p] + (last - lo + 1);
+  }
+  g.N = g.off[g.npairs];
+  const int64_t C = P->hd == 128 ? 128 : 256;
+  int64_t parts = (g.N + 2 * C - 1) / (2 * C);
+  g.nparts = (int)(parts < 1 ? 1 : (parts > c.ncta ? c.ncta : parts));
+}
+MSK_DEV int att_owner(const AttGeo& g, int64_t x) {
+  return (int)(((x + 1) * (int64_t)g.nparts - 1) / g.N);
+}
+MSK_DEV int att_keys_per_stage(int hd) { return hd == 128 ? 128 : 256; }
+
+/* Calls f(pair, slot, key0, nkeys, first_of_segment, last_of_segment) for
+ * this CTA's attention stages. */
+template <class F>
+MSK_DEV void for_each_att_stage(const Ctx& c, const AttGeo& g, F&& f) {
+  const int C = att_keys_per_stage(c.P->hd);
+  if (c.cta >= g.nparts) return;
+  int64_t A = g.N * c.cta / g.nparts, B = g.N * (c.cta + 1) / g.nparts;
+  for (int p = 0; p < g.npairs; ++p) {
+    int64_t a = max(A, g.off[p]), b = min(B, g.off[p + 1]);
+    if (a >= b) continue;
+    int64_t k0 = g.lo[p] + (a - g.off[p]), k1 = g.lo[p] + (b - g.off[p]);
+    for (int64_t x = k0; x < k1; x += C) {
+      int n = (int)min((int64_t)C, k1 - x);
+      if (!f(p, c.cta + p, x, n, x == k0, x + C >= k1)) return;
+    }
+  }
+}
+
+/* ---- producer ---------------------------------------------------------------------- */
+struct Prod {
+  Ctx* c;
+  uint32_t it;
+  uint32_t last_parity_for_slot[MSK_NST];
+  bool ok;
+};
+
+MSK_DEV bool prod_acquire(Prod& p, int layer, int phase, uint8_t** stg, uint64_t** bar) {
+  Ctx& c = *p.c;
+  uint32_t slot = p.it % MSK_NST, round = p.it / MSK_NST;
+  if (round > 0 && !wait_bar(c, &c.S->empty[slot], (round - 1) & 1, layer, phase)) return false;
+  *stg = c.ring + (size_t)slot * MSK_STAGE;
+  *bar = &c.S->full[slot];
+  p.last_parity_for_slot[slot] = round & 1;
+  p.it++;
+  return true;
+}
+
+MSK_DEV bool prod_weights(Prod& p, const WStage& s, int layer, int phase) {
+  uint8_t* stg;
+  uint64_t* bar;
+  if (!prod_acquire(p, layer, phase, &stg, &bar)) return false;
+  uint32_t cb = (uint32_t)s.nrows * (s.K / 2), sb = (uint32_t)s.nrows * (s.K / 16);
+  mbar_arrive_tx(bar, cb + sb);
+  bulk_g2s(stg, s.codes, cb, bar);
+  bulk_g2s(stg + cb, s.scales, sb, bar);
+  return true;
+}
+
+MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, int phase) {
+  uint64_t t0 = gtimer();
+  for (uint32_t it = 0; *flag < want; ++it) {
+    if ((it & 15) == 0) {
+      if (aborted(c)) return false;
+      if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+        raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
+        return false;
+      }
+    }
+    __nanosleep(32);
+  }
+  __threadfence_block();
+  return true;
+}
+
+MSK_DEV void producer(Ctx& c) {
+  const MskParams* P = c.P;
+  Prod p;
+  p.c = &c;
+  p.it = 0;
+  p.ok = true;
+  const int hd = P->hd;
+  const int C = att_keys_per_stage(hd);
+  for (int l = 0; l < P->L && p.ok; ++l) {
+    const MskLayer& Ly = P->layers[l];
+    /* QKV weights: round-robin stages */
+    int sQ, sK, nq = qkv_stages(P, &sQ, &sK);
+    for (int j = c.cta; j < nq && p.ok; j += c.ncta) p.ok = prod_weights(p, qkv_stage(P, Ly, j, sQ, sK), l, PH_QKV);
+    /* attention: past keys stream at once, chunks holding this step's keys
+     * wait until every CTA has written them */
+    AttGeo g;
+    att_geo(c, l, g);
+    for_each_att_stage(c, g, [&](int pr, int slot, int64_t k0, int n, bool, bool) {
+      int b = pr / P->hkv, h = pr % P->hkv;
+      if (k0 + C > c.S->pos0[b]) {
+        if (!wait_flag(c, &c.S->kv_ready, l + 1, l, PH_ATT)) { p.ok = false; return false; }
+        fence_proxy_async_global();
+      }
+      uint8_t* stg;
+      uint64_t* bar;
+      if (!prod_acquire(p, l, PH_ATT, &stg, &bar)) { p.ok = false; return false; }
+      int64_t row = (((int64_t)l * c.st.kv_seqs + b) * P->hkv + h) * c.st.kv_cap + k0;
+      mbar_arrive_tx(bar, (uint32_t)(2 * C * hd));
+      tma_2d_g2s(stg, c.kvmap, 0, (int32_t)row, bar);
+      tma_2d_g2s(stg + C * hd, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), bar);
+      (void)slot;
+      (void)n;
+      return true;
+    });
+    if (!p.ok) break;
+    int nwo = (P->d + rows_per_stage(P->qd) - 1) / rows_per_stage(P->qd);
+    for (int j = c.cta; j < nwo && p.ok; j += c.ncta) p.ok = prod_weights(p, wo_stage(P, Ly, j), l, PH_WO);
+    if (!p.ok) break;
+    /* the consumer warps stream the selected experts through their own
+     * slices of the ring; meanwhile pull this CTA's next-layer dense tiles
+     * into L2 */
+    if (l + 1 < P->L) {
+      const MskLayer& Ln = P->layers[l + 1];
+      for (int j = c.cta; j < nq; j += c.ncta) {
+        WStage ws = qkv_stage(P, Ln, j, sQ, sK);
+        prefetch_l2(ws.codes, (uint32_t)ws.nrows * (ws.K / 2));
+        prefetch_l2(ws.scales, (uint32_t)ws.nrows * (ws.K / 16));
+      }
+      for (int j = c.cta; j < nwo; j += c.ncta) {
+        WStage ws = wo_stage(P, Ln, j);
+        prefetch_l2(ws.codes, (uint32_t)ws.nrows * (ws.K / 2));
+        prefetch_l2(ws.scales, (uint32_t)ws.nrows * (ws.K / 16));
+      }
+    }
+    if (!wait_flag(c, &c.S->ring_free, l + 1, l, PH_DN)) { p.ok = false; break; }
+  }
+  if (!p.ok) {
+    /* let every copy already issued land before the CTA may exit */
+    uint32_t n = p.it < MSK_NST ? p.it : MSK_NST;
+    for (uint32_t i = p.it - n; i < p.it; ++i) {
+      uint32_t slot = i % MSK_NST;
+      uint64_t t0 = gtimer();
+      while (!mbar_try(&c.S->full[slot], (i / MSK_NST) & 1)) {
+        if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+      }
+    }
+  }
+}
+
+/* ---- consumer: weight stages on the tensor cores ----------------------------------- */
+struct Cons {
+  Ctx* c;
+  uint32_t it;
+};
+
+MSK_DEV uint8_t* cons_wait(Cons& q, int layer, int phase, uint32_t* slot_out) {
+  Ctx& c = *q.c;
+  uint32_t slot = q.it % MSK_NST, round = q.it / MSK_NST;
+  if (!wait_bar(c, &c.S->full[slot], round & 1, layer, phase)) return nullptr;
+  *slot_out = slot;
+  q.it++;
+  return c.ring + (size_t)slot * MSK_STAGE;
+}
+MSK_DEV void cons_release(Cons& q, uint32_t slot) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&q.c->S->empty[slot]);
+}
+
+/* split of a weight stage over the consumer warps: mt m-tiles x ks K-slices */
+MSK_DEV void stage_split(int nrows, int K, int* mt, int* ks) {
+  int m = nrows / 16;
+  int mp = 1;
+  while (mp < m) mp <<= 1;
+  int k = NCW / mp;
+  if (k < 1) k = 1;
+  while (k > 1 && ((K / 64) % k) != 0) k >>= 1;
+  *mt = m;
+  *ks = k;
+}
+
+/*
+ * One weight stage (nrows x K NVFP4 in smem) times ncols activation columns.
+ * Columns are rows of an f16 matrix: bcol(j) gives the row pointer of column j
+ * (j < ncols).  K is split into windows of 64*BPT; inside a window lane
+ * (g, c) owns NVFP4 blocks c*BPT .. c*BPT+BPT-1 of rows g and g+8, so its
+ * A-fragment bytes are contiguous; the same k permutation is applied to the
+ * B fragments, which leaves the dot products unchanged.
+ */
+template <int NT, int BPT>
+MSK_DEV void gemm_warp(const uint8_t* stg, int nrows, int K, int ks, int mi, int ki, int ntl,
+                       const uint16_t* const* bp, float (*acc)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const int Kr = K / ks;
+  const int nwin = Kr / (64 * BPT);
+  const int r0 = mi * 16 + g;
+  const uint32_t sbase = smem_u32(stg);
+  const uint32_t cbase0 = sbase + r0 * (K / 2), cbase1 = cbase0 + 8 * (K / 2);
+  const uint32_t scb = sbase + nrows * (K / 2);
+  const uint32_t sbase0 = scb + r0 * (K / 16), sbase1 = sbase0 + 8 * (K / 16);
+  for (int win = 0; win < nwin; ++win) {
+    const int kw = ki * Kr + win * 64 * BPT;
+    const uint32_t coff = kw / 2 + cq * BPT * 8;
+    const uint32_t soff = kw / 16 + cq * BPT;
+    uint32_t w0[2 * BPT], w1[2 * BPT];
+    if (BPT == 4) {
+      uint4 a = lds128(cbase0 + coff), b = lds128(cbase0 + coff + 16);
+      uint4 d = lds128(cbase1 + coff), e = lds128(cbase1 + coff + 16);
+      w0[0] = a.x; w0[1] = a.y; w0[2] = a.z; w0[3] = a.w; w0[4 % (2 * BPT)] = b.x; w0[5 % (2 * BPT)] = b.y;
+      w0[6 % (2 * BPT)] = b.z; w0[7 % (2 * BPT)] = b.w;
+      w1[0] = d.x; w1[1] = d.y; w1[2] = d.z; w1[3] = d.w; w1[4 % (2 * BPT)] = e.x; w1[5 % (2 * BPT)] = e.y;
+      w1[6 % (2 * BPT)] = e.z; w1[7 % (2 * BPT)] = e.w;
+    } else if (BPT == 2) {
+      uint4 a = lds128(cbase0 + coff), d = lds128(cbase1 + coff);
+      w0[0] = a.x; w0[1] = a.y; w0[2 % (2 * BPT)] = a.z; w0[3 % (2 * BPT)] = a.w;
+      w1[0] = d.x; w1[1] = d.y; w1[2 % (2 * BPT)] = d.z; w1[3 % (2 * BPT)] = d.w;
+    } else {
+      uint2 a = lds64(cbase0 + coff), d = lds64(cbase1 + coff);
+      w0[0] = a.x; w0[1 % (2 * BPT)] = a.y;
+      w1[0] = d.x; w1[1 % (2 * BPT)] = d.y;
+    }
+    uint32_t sw0, sw1; /* BPT scale bytes of rows g and g+8 */
+    if (BPT == 4) {
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw0) : "r"(sbase0 + soff));
+      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw1) : "r"(sbase1 + soff));
+    } else if (BPT == 2) {
+      asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw0) : "r"(sbase0 + soff));
+      asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw1) : "r"(sbase1 + soff));
+    } else {
+      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw0) : "r"(sbase0 + soff));
+      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw1) : "r"(sbase1 + soff));
+    }
+#pragma unroll
+    for (int qb = 0; qb < BPT; ++qb) {
+      const uint32_t s0 = (sw0 >> (8 * qb)) & 0xFF, s1 = (sw1 >> (8 * qb)) & 0xFF;
+      const uint32_t sc0 = e4m3x2_to_f16x2(s0 | (s0 << 8)), sc1 = e4m3x2_to_f16x2(s1 | (s1 << 8));
+      const int kb = kw + 16 * (cq * BPT + qb);
+      uint4 bl[NT][2];
+#pragma unroll
+      for (int j = 0; j < NT; ++j) {
+        if (j < ntl && bp[j]) {
+          bl[j][0] = ldg128(bp[j] + kb);
+          bl[j][1] = ldg128(bp[j] + kb + 8);
+        } else {
+          bl[j][0] = bl[j][1] = make_uint4(0, 0, 0, 0);
+        }
+      }
+#pragma unroll
+      for (int s = 0; s < 4; ++s) {
+        const uint32_t x0 = w0[2 * qb + (s >> 1)] >> (16 * (s & 1));
+        const uint32_t x1 = w1[2 * qb + (s >> 1)] >> (16 * (s & 1));
+        uint32_t a[4];
+        a[0] = hmul2(e2m1x2_to_f16x2(x0 & 0xFF), sc0);
+        a[1] = hmul2(e2m1x2_to_f16x2(x1 & 0xFF), sc1);
+        a[2] = hmul2(e2m1x2_to_f16x2((x0 >> 8) & 0xFF), sc0);
+        a[3] = hmul2(e2m1x2_to_f16x2((x1 >> 8) & 0xFF), sc1);
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          if (j < ntl) {
+            const uint4& lo = bl[j][s >> 1];
+            const uint32_t b0 = (s & 1) ? lo.z : lo.x, b1 = (s & 1) ? lo.w : lo.y;
+            mma_f16(acc[j], a, b0, b1);
+          }
+        }
+      }
+    }
+  }
+}
+
+template <int NT, class BCol, class Epi>
+MSK_DEV bool gemm_stage(Cons& q, const WStage& ws, int ncols, BCol bcol, Epi epi, int layer, int phase) {
+  Ctx& c = *q.c;
+  uint32_t slot;
+  /* on a failed wait the warp skips the math but keeps the barrier sequence,
+   * so no sibling is left waiting in a named barrier */
+  const uint8_t* stg = cons_wait(q, layer, phase, &slot);
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2;
+  const int K = ws.K, nrows = ws.nrows;
+  int mt, ks;
+  stage_split(nrows, K, &mt, &ks);
+  const int ntl = (ncols + 7) >> 3;
+  float acc[NT][4];
+#pragma unroll
+  for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
+  const bool active = cw < mt * ks && stg != nullptr;
+  if (active) {
+    const int mi = cw / ks, ki = cw % ks;
+    const int Kr = K / ks;
+    const uint16_t* bp[NT];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int col = j * 8 + g;
+      bp[j] = (j < ntl && col < ncols) ? bcol(col) : nullptr;
+    }
+    if ((Kr / 64) % 4 == 0) gemm_warp<NT, 4>(stg, nrows, K, ks, mi, ki, ntl, bp, acc);
+    else if ((Kr / 64) % 2 == 0) gemm_warp<NT, 2>(stg, nrows, K, ks, mi, ki, ntl, bp, acc);
+    else gemm_warp<NT, 1>(stg, nrows, K, ks, mi, ki, ntl, bp, acc);
+  }
+  if (stg) cons_release(q, slot);
+  /* split-K reduction in fixed order, then the epilogue */
+  float* red = c.scr;
+  if (active) {
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+      if (j < ntl)
+        *reinterpret_cast<float4*>(&red[((cw * NT + j) * 32 + lane) * 4]) =
+            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
+  }
+  named_sync(BAR_CONS, NCT);
+  const int ctid = threadIdx.x - CONS0;
+  for (int idx = ctid; idx < mt * ntl * 32; idx += NCT) {
+    int mi = idx / (ntl * 32), j = (idx / 32) % ntl, ln = idx & 31;
+    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int ki = 0; ki < ks; ++ki) {
+      float4 v = *reinterpret_cast<const float4*>(&red[(((mi * ks + ki) * NT + j) * 32 + ln) * 4]);
+      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+    }
+    int row = mi * 16 + (ln >> 2), col = j * 8 + 2 * (ln & 3);
+    if (col < ncols) { epi(row, col, s.x * ws.gs); epi(row + 8, col, s.z * ws.gs); }
+    if (col + 1 < ncols) { epi(row, col + 1, s.y * ws.gs); epi(row + 8, col + 1, s.w * ws.gs); }
+  }
+  named_sync(BAR_CONS, NCT);
+  return !c.S->abort; /* read after the barrier: the same answer in every warp */
+}
+
+/* ---- consumer: attention stages ------------------------------------------------------ */
+MSK_DEV uint32_t swz(uint32_t off, int hd) {
+  return hd == 128 ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
+}
+
+template <int HD>
+struct AttState {
+  float o[HD / 8][4];
+  float l0, l1;
+  int lo0, hi0, lo1, hi1; /* key window of rows g and g+8 (empty if lo > hi) */
+};
+
+/* Q of the segment's rows as A fragments in the scratch, fragment order:
+ * qf[mi][step][lane] = 16 bytes (a0a1, a2a3, a4a5, a6a7).  Warps with ki == 0
+ * fill their m-tile; every consumer warp passes the barrier. */
+template <int HD>
+MSK_DEV void att_begin(const Ctx& c, AttState<HD>& A, int pair, int mi, bool writer) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const int b = pair / P->hkv, kvh = pair % P->hkv;
+  const int R = c.st.Tq * P->G;
+#pragma unroll
+  for (int j = 0; j < HD / 8; ++j) A.o[j][0] = A.o[j][1] = A.o[j][2] = A.o[j][3] = 0.f;
+  A.l0 = A.l1 = 0.f;
+  uint4* qf = reinterpret_cast<uint4*>(c.scr) + (size_t)mi * (HD / 16) * 32;
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int rho = mi * 16 + g + 8 * half;
+    int lo = 1, hi = 0;
+    uint32_t qw[HD / 8];
+#pragma unroll
+    for (int i = 0; i < HD / 8; ++i) qw[i] = 0;
+    if (rho < R) {
+      const int ti = rho / P->G, h = kvh * P->G + rho % P->G;
+      const int t = b * c.st.Tq + ti;
+      hi = c.S->pos0[b] + ti;
+      lo = 0;
+      if (writer) {
+        const uint16_t* qrow = P->qs + (size_t)t * P->qd + h * HD + cq * (HD / 4);
+#pragma unroll
+        for (int i = 0; i < HD / 32; ++i) {
+          uint4 v = ldg128(qrow + 8 * i);
+          qw[4 * i] = v.x; qw[4 * i + 1] = v.y; qw[4 * i + 2] = v.z; qw[4 * i + 3] = v.w;
+        }
+      }
+    }
+    if (half == 0) { A.lo0 = lo; A.hi0 = hi; } else { A.lo1 = lo; A.hi1 = hi; }
+    if (writer) {
+      /* step s uses q[c*HD/4 + 4s .. +4): words 2s (a0a1 / a2a3) and 2s+1 (a4a5 / a6a7) */
+      uint32_t* qfw = reinterpret_cast<uint32_t*>(qf);
+#pragma unroll
+      for (int s = 0; s < HD / 16; ++s) {
+        qfw[(s * 32 + lane) * 4 + half] = qw[2 * s];
+        qfw[(s * 32 + lane) * 4 + 2 + half] = qw[2 * s + 1];
+      }
+    }
+  }
+  named_sync(BAR_CONS, NCT);
+}
+
+template <int HD>
+MSK_DEV void att_stage(const Ctx& c, AttState<HD>& A, const uint8_t* stg, int64_t k0, int nkeys, int ks, int mi,
+                       int ki, float scale_log2, float bound_log2) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const uint32_t kbase = smem_u32(stg);
+  const int C = (HD == 128) ? 128 : 256;
+  const uint32_t vbase = kbase + C * HD;
+  const uint32_t qfb = smem_u32(c.scr) + (uint32_t)(mi * (HD / 16) * 32 + lane) * 16;
+  const float two120 = 1.329227995784916e36f; /* 2^120 */
+  const int k0i = (int)k0;
+  for (int kb = ki; kb * 16 < nkeys; kb += ks) {
+    float sacc[2][4];
+#pragma unroll
+    for (int n2 = 0; n2 < 2; ++n2) {
+      sacc[n2][0] = sacc[n2][1] = sacc[n2][2] = sacc[n2][3] = 0.f;
+      const uint32_t row = kb * 16 + n2 * 8 + g;
+      uint32_t kw[HD / 16];
+#pragma unroll
+      for (int i = 0; i < HD / 64; ++i) {
+        uint4 v = lds128(kbase + swz(row * HD + cq * (HD / 4) + 16 * i, HD));
+        kw[4 * i] = v.x; kw[4 * i + 1] = v.y; kw[4 * i + 2] = v.z; kw[4 * i + 3] = v.w;
+      }
+#pragma unroll
+      for (int s = 0; s < HD / 16; ++s) {
+        const uint4 qv = lds128(qfb + s * 32 * 16);
+        const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w};
+        mma_f16(sacc[n2], qa, e4m3x2_to_f16x2(kw[s] & 0xFFFF), e4m3x2_to_f16x2(kw[s] >> 16));
+      }
+    }
+    /* p = exp(s - M) under the key windows; l in fp32, P as bf16 scaled by 2^120
+     * to match V's 2^-120 */
+    uint32_t pa[4];
+#pragma unroll
+    for (int n2 = 0; n2 < 2; ++n2) {
+      float p[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kl = kb * 16 + n2 * 8 + 2 * cq + (e & 1);
+        const int kp = k0i + kl;
+        const bool r1 = e >= 2;
+        const bool ok = kl < nkeys && (r1 ? (kp >= A.lo1 && kp <= A.hi1) : (kp >= A.lo0 && kp <= A.hi0));
+        p[e] = ok ? fast_exp2(sacc[n2][e] * scale_log2 - bound_log2) : 0.f;
+      }
+      A.l0 += p[0] + p[1];
+      A.l1 += p[2] + p[3];
+      pa[2 * n2] = f32x2_to_bf16x2(p[0] * two120, p[1] * two120);
+      pa[2 * n2 + 1] = f32x2_to_bf16x2(p[2] * two120, p[3] * two120);
+    }
+    /* V: lane (g, c) holds columns g*HD/8 .. +HD/8 of keys 2c, 2c+1, 2c+8, 2c+9
+     * (the mma k-slots of this lane: keys 2c, 2c+1 from S tile 0, 8+2c, 9+2c
+     * from S tile 1); read 8 columns at a time */
+    const uint32_t rA = kb * 16 + 2 * cq;
+#pragma unroll
+    for (int hv = 0; hv < HD / 64; ++hv) {
+      uint32_t vw[4][2];
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const uint32_t row = rA + (kk & 1) + 8 * (kk >> 1);
+        uint2 v = lds64(vbase + swz(row * HD + g * (HD / 8) + 8 * hv, HD));
+        vw[kk][0] = v.x; vw[kk][1] = v.y;
+      }
+#pragma unroll
+      for (int wi = 0; wi < 2; ++wi) {
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const uint32_t sel = (uint32_t)(j | (j << 4) | ((j + 4) << 8) | ((j + 4) << 12));
+          const uint32_t b0 = e4m3pair_to_bf16x2_scaled(vw[0][wi], vw[1][wi], sel);
+          const uint32_t b1 = e4m3pair_to_bf16x2_scaled(vw[2][wi], vw[3][wi], sel);
+          mma_bf16(A.o[(hv * 2 + wi) * 4 + j], pa, b0, b1);
+        }
+      }
+    }
+  }
+}
+
+/* Reduce the key-split warps of each m-tile (fixed order) and write the
+ * segment's partial (o[rho][0..hd), l at [hd]) to slot `slot`. */
+template <int HD>
+MSK_DEV void att_end(const Ctx& c, AttState<HD>& A, int pair, int slot, int mt, int ks) {
+  const MskParams* P = c.P;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const bool active = cw < mt * ks;
+  const int mi = active ? cw / ks : 0, ki = active ? cw % ks : 0;
+  /* quad-reduce the row sums first (each lane summed its own key columns) */
+  A.l0 += __shfl_xor_sync(0xffffffffu, A.l0, 1);
+  A.l0 += __shfl_xor_sync(0xffffffffu, A.l0, 2);
+  A.l1 += __shfl_xor_sync(0xffffffffu, A.l1, 1);
+  A.l1 += __shfl_xor_sync(0xffffffffu, A.l1, 2);
+  named_sync(BAR_CONS, NCT); /* every warp is done with the Q fragments */
+  float* buf = c.scr;
+  for (int step = ks / 2; step >= 1; step >>= 1) {
+    if (active && ki >= step && ki < 2 * step) {
+      const int bi = mi * step + (ki - step);
+      float* dst = buf + (size_t)bi * (HD / 8) * 128;
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j)
+        *reinterpret_cast<float4*>(&dst[(j * 32 + lane) * 4]) = make_float4(A.o[j][0], A.o[j][1], A.o[j][2], A.o[j][3]);
+      c.S->lbuf[bi][lane][0] = A.l0;
+      c.S->lbuf[bi][lane][1] = A.l1;
+    }
+    named_sync(BAR_CONS, NCT);
+    if (active && ki < step) {
+      const int bi = mi * step + ki;
+      const float* src = buf + (size_t)bi * (HD / 8) * 128;
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) {
+        float4 v = *reinterpret_cast<const float4*>(&src[(j * 32 + lane) * 4]);
+        A.o[j][0] += v.x; A.o[j][1] += v.y; A.o[j][2] += v.z; A.o[j][3] += v.w;
+      }
+      A.l0 += c.S->lbuf[bi][lane][0];
+      A.l1 += c.S->lbuf[bi][lane][1];
+    }
+    named_sync(BAR_CONS, NCT);
+  }
+  if (active && ki == 0) {
+    const int R = c.st.Tq * P->G;
+    float* base = P->part + (size_t)slot * P->part_stride;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int rho = mi * 16 + g + 8 * half;
+      if (rho >= R) continue;
+      float* row = base + (size_t)rho * (HD + 4);
+#pragma unroll
+      for (int j = 0; j < HD / 8; ++j) {
+        /* C-fragment column 2c+e of n-tile j is head dim (2c+e)*HD/8 + j */
+        row[(2 * cq) * (HD / 8) + j] = A.o[j][2 * half];
+        row[(2 * cq + 1) * (HD / 8) + j] = A.o[j][2 * half + 1];
+      }
+      if (cq == 0) row[HD] = half ? A.l1 : A.l0;
+    }
+  }
+}
+
+template <int HD>
+MSK_DEV bool attention_phase(Cons& q, int layer) {
+  Ctx& c = *q.c;
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  AttGeo g;
+  att_geo(c, layer, g);
+  const int R = c.st.Tq * P->G;
+  const int mt = (R + 15) / 16;
+  int mp = 1;
+  while (mp < mt) mp <<= 1;
+  const int ks = NCW / mp;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0;
+  const bool active = cw < mt * ks;
+  const int mi = active ? cw / ks : 0, ki = active ? cw % ks : 0;
+  const int C = att_keys_per_stage(HD);
+  const float scale_log2 = P->scale_log2, bound_log2 = Ly.bound_log2;
+  if (c.cta < g.nparts) {
+    const int64_t A0 = g.N * c.cta / g.nparts, B0 = g.N * (c.cta + 1) / g.nparts;
+    for (int p = 0; p < g.npairs; ++p) {
+      const int64_t a = max(A0, g.off[p]), b = min(B0, g.off[p + 1]);
+      if (a >= b) continue;
+      const int k0 = (int)(g.lo[p] + (a - g.off[p])), k1 = (int)(g.lo[p] + (b - g.off[p]));
+      AttState<HD> A;
+      att_begin<HD>(c, A, p, mi, active && ki == 0);
+      if (Ly.sliding) { /* key windows of this layer */
+        if (A.lo0 <= A.hi0) { A.lo0 = A.hi0 - P->W + 1; if (A.lo0 < 0) A.lo0 = 0; }
+        if (A.lo1 <= A.hi1) { A.lo1 = A.hi1 - P->W + 1; if (A.lo1 < 0) A.lo1 = 0; }
+      }
+      for (int x = k0; x < k1; x += C) {
+        uint32_t sl;
+        const uint8_t* stg = cons_wait(q, layer, PH_ATT, &sl);
+        if (stg) {
+          if (active) att_stage<HD>(c, A, stg, x, min(C, k1 - x), ks, mi, ki, scale_log2, bound_log2);
+          cons_release(q, sl);
+        }
+      }
+      att_end<HD>(c, A, p, c.cta + p, mt, ks);
+    }
+  }
+  named_sync(BAR_CONS, NCT);
+  return !c.S->abort;
+}
+
+/* ---- consumer: small phases (warp per item over the whole grid) --------------------- */
+MSK_DEV int gwarp(const Ctx& c) { return c.cta * NCW + (threadIdx.x >> 5) - CONS_WARP0; }
+MSK_DEV int nwarps(const Ctx& c) { return c.ncta * NCW; }
+
+/* x = f16(rmsnorm(h) * g) for the row of token t (whole warp) */
+MSK_DEV void norm_row(const float* h, const float* gain, int d, float eps, uint16_t* xh, float* xf) {
+  const int lane = threadIdx.x & 31;
+  float ss = 0.f;
+  for (int i = lane * 4; i < d; i += 128) {
+    float4 v = *reinterpret_cast<const float4*>(h + i);
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / d + eps);
+  for (int i = lane * 4; i < d; i += 128) {
+    float4 v = *reinterpret_cast<const float4*>(h + i);
+    float4 gg = *reinterpret_cast<const float4*>(gain + i);
+    float a = v.x * r * gg.x, b = v.y * r * gg.y, cc = v.z * r * gg.z, dd = v.w * r * gg.w;
+    if (xf) *reinterpret_cast<float4*>(xf + i) = make_float4(a, b, cc, dd);
+    *reinterpret_cast<uint2*>(xh + i) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(cc, dd));
+  }
+}
+
+MSK_DEV void phase_in(const Ctx& c) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31;
+  for (int t = gwarp(c); t < c.st.T; t += nwarps(c)) {
+    float* h = P->h + (size_t)t * P->d;
+    const uint16_t* hin = c.st.hidden_in + (size_t)t * P->d;
+    for (int i = lane * 4; i < P->d; i += 128) {
+      uint2 v = *reinterpret_cast<const uint2*>(hin + i);
+      *reinterpret_cast<float4*>(h + i) = make_float4(bf16_to_f32(v.x & 0xFFFF), bf16_to_f32(v.x >> 16),
+                                                      bf16_to_f32(v.y & 0xFFFF), bf16_to_f32(v.y >> 16));
+    }
+    __syncwarp();
+    norm_row(h, P->layers[0].g_attn, P->d, P->eps, P->x + (size_t)t * P->d, nullptr);
+  }
+}
+
+/* QK-norm of q and k heads, fp8 quantisation of k and v into the cache */
+MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const int lane = threadIdx.x & 31;
+  const int hd = P->hd, nh = P->hq + 2 * P->hkv, nqkv = P->qd + 2 * P->kvd;
+  const int per = hd / 32; /* 4 or 2 values per lane */
+  for (int item = gwarp(c); item < c.st.T * nh; item += nwarps(c)) {
+    const int t = item / nh, hh = item % nh;
+    const float* raw = P->qkv + (size_t)t * nqkv + hh * hd + lane * per;
+    float v[4];
+    for (int i = 0; i < per; ++i) v[i] = raw[i];
+    const int b = t / c.st.Tq, ti = t % c.st.Tq;
+    if (hh < P->hq + P->hkv) {
+      float ss = 0.f;
+      for (int i = 0; i < per; ++i) ss += v[i] * v[i];
+      ss = warp_sum(ss);
+      const float r = 1.0f / sqrtf(ss / hd + P->eps);
+      const float* gain = (hh < P->hq ? Ly.g_q : Ly.g_k) + lane * per;
+      for (int i = 0; i < per; ++i) v[i] = v[i] * r * gain[i];
+    }
+    if (hh < P->hq) {
+      uint16_t* dst = P->qs + (size_t)t * P->qd + hh * hd + lane * per;
+      for (int i = 0; i < per; ++i) dst[i] = f32_to_f16(v[i]);
+    } else {
+      const int isv = hh >= P->hq + P->hkv;
+      const int kvh = hh - P->hq - (isv ? P->hkv : 0);
+      const int64_t pos = c.S->pos0[b] + ti;
+      int64_t row = (((int64_t)layer * c.st.kv_seqs + b) * P->hkv + kvh) * c.st.kv_cap + pos;
+      if (isv) row += c.st.kv_half_rows;
+      uint8_t* dst = c.st.kv_base + row * hd + lane * per;
+      if (per == 4) {
+        uint32_t lo = f32x2_to_e4m3x2(v[0], v[1]), hi = f32x2_to_e4m3x2(v[2], v[3]);
+        *reinterpret_cast<uint32_t*>(dst) = lo | (hi << 16);
+      } else {
+        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)f32x2_to_e4m3x2(v[0], v[1]);
+      }
+    }
+  }
+  fence_proxy_async_global();
+}
+
+/* o = sum of partials / sum of l over the pair's segments */
+MSK_DEV void phase_attc(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31, hd = P->hd, per = hd / 32;
+  AttGeo g;
+  att_geo(c, layer, g);
+  for (int item = gwarp(c); item < c.st.T * P->hq; item += nwarps(c)) {
+    const int t = item / P->hq, h = item % P->hq;
+    const int b = t / c.st.Tq, ti = t % c.st.Tq;
+    const int pair = b * P->hkv + h / P->G;
+    const int rho = ti * P->G + h % P->G;
+    const int cf = att_owner(g, g.off[pair]), cl = att_owner(g, g.off[pair + 1] - 1);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+    for (int cc = cf; cc <= cl; ++cc) {
+      const float* row = P->part + (size_t)(cc + pair) * P->part_stride + (size_t)rho * (hd + 4);
+      for (int i = 0; i < per; ++i) acc[i] += row[lane * per + i];
+      l += row[hd];
+    }
+    const float inv = 1.0f / l;
+    uint16_t* dst = P->o + (size_t)t * P->qd + h * hd + lane * per;
+    for (int i = 0; i < per; ++i) dst[i] = f32_to_f16(acc[i] * inv);
+    if (P->dbg_attn) {
+      float* dbg = P->dbg_attn + ((size_t)layer * c.st.T + t) * P->qd + h * hd + lane * per;
+      for (int i = 0; i < per; ++i) dbg[i] = acc[i] * inv;
+    }
+  }
+}
+
+MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  for (int t = gwarp(c); t < c.st.T; t += nwarps(c))
+    norm_row(P->h + (size_t)t * P->d, P->layers[layer].g_moe, P->d, P->eps, P->x2h + (size_t)t * P->d,
+             P->x2f + (size_t)t * P->d);
+}
+
+/* router logits in fp32: items (8 tokens, 8 experts), one expert per warp */
+MSK_DEV void phase_router(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  const float* Wr = P->layers[layer].router;
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - CONS_WARP0;
+  const int ntg = (c.st.T + 7) / 8, neg = P->E / NCW;
+  for (int item = c.cta; item < ntg * neg; item += c.ncta) {
+    const int tg = item / neg, e = (item % neg) * NCW + cw;
+    const int nt = min(8, c.st.T - tg * 8);
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
+    const float* wrow = Wr + (size_t)e * P->d;
+    for (int i = lane * 4; i < P->d; i += 128) {
+      float4 w = *reinterpret_cast<const float4*>(wrow + i);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j < nt) {
+          float4 x = *reinterpret_cast<const float4*>(P->x2f + (size_t)(tg * 8 + j) * P->d + i);
+          acc[j] += w.x * x.x + w.y * x.y + w.z * x.z + w.w * x.w;
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      float s = warp_sum(acc[j]);
+      if (lane == 0 && j < nt) P->logits[(size_t)(tg * 8 + j) * P->E + e] = s;
+    }
+  }
+}
+
+/* top-k of every token (value desc, index asc), softmax weights, and the
+ * expert work list grouped by expert; every CTA computes the same lists */
+MSK_DEV void phase_topk(Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  Route& R = c.S->route;
+  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - CONS_WARP0;
+  const int E = P->E, k = P->k, per = E / 32;
+  for (int t = cw; t < c.st.T; t += NCW) {
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = i < per ? P->logits[(size_t)t * E + lane * per + i] : -INFINITY;
+    uint32_t taken = 0;
+    float sel[8];
+    float vmax = 0.f;
+    for (int s = 0; s < k; ++s) {
+      float bv = -INFINITY;
+      int bi = 0x7FFFFFFF;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (i < per && !(taken >> i & 1) && (v[i] > bv)) { bv = v[i]; bi = lane * per + i; }
+#pragma unroll
+      for (int o = 16; o; o >>= 1) {
+        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+      }
+      if (bi / per == lane) taken |= 1u << (bi % per);
+      if (s == 0) vmax = bv;
+      sel[s] = bv;
+      if (lane == 0) R.ids[t * k + s] = (int16_t)bi;
+    }
+    if (lane == 0) {
+      float sum = 0.f;
+      for (int s = 0; s < k; ++s) { sel[s] = expf(sel[s] - vmax); sum += sel[s]; }
+      for (int s = 0; s < k; ++s) R.w[t * k + s] = sel[s] / sum;
+    }
+  }
+  named_sync(BAR_CONS, NCT);
+  if (cw == 0) {
+    const int np = c.st.T * k;
+    for (int e = lane; e < E; e += 32) R.cnt[e] = 0;
+    __syncwarp();
+    /* rank of each pair among same-expert pairs, in pair order */
+    int16_t rank_local[16];
+    for (int base = 0, ch = 0; base < np; base += 32, ++ch) {
+      const int pi = base + lane;
+      const bool valid = pi < np;
+      const int e = valid ? R.ids[pi] : -1 - lane;
+      const uint32_t peers = __match_any_sync(0xffffffffu, e);
+      const int rank = __popc(peers & ((1u << lane) - 1));
+      const int before = valid ? R.cnt[e] : 0;
+      __syncwarp();
+      if (valid && rank == 0) R.cnt[e] = (int16_t)(before + __popc(peers));
+      __syncwarp();
+      rank_local[ch] = (int16_t)(before + rank);
+    }
+    /* exclusive scan of counts -> start */
+    int run = 0;
+    for (int base = 0; base < E; base += 32) {
+      int v = R.cnt[base + lane], x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      R.start[base + lane] = (int16_t)(run + x - v);
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) R.start[E] = (int16_t)run;
+    __syncwarp();
+    for (int base = 0, ch = 0; base < np; base += 32, ++ch) {
+      const int pi = base + lane;
+      if (pi < np) R.pairs[R.start[R.ids[pi]] + rank_local[ch]] = (int16_t)pi;
+    }
+    /* units: experts with tokens, split into groups of <= MSK_UNIT_TOK */
+    int nu = 0, nd = 0;
+    for (int base = 0; base < E; base += 32) {
+      const int e = base + lane, n = R.cnt[e];
+      const int mine = (n + MSK_UNIT_TOK - 1) / MSK_UNIT_TOK;
+      int x = mine;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      const int first = nu + x - mine;
+      for (int u = 0; u < mine; ++u) {
+        R.unit_e[first + u] = (int16_t)e;
+        R.unit_start[first + u] = (int16_t)(R.start[e] + u * MSK_UNIT_TOK);
+        R.unit_n[first + u] = (int16_t)min(MSK_UNIT_TOK, n - u * MSK_UNIT_TOK);
+      }
+      nu += __shfl_sync(0xffffffffu, x, 31);
+      nd += __popc(__ballot_sync(0xffffffffu, n > 0));
+    }
+    if (lane == 0) { R.n_units = nu; R.n_distinct = nd; }
+  }
+  named_sync(BAR_CONS, NCT);
+  if (c.cta == 0) {
+    const int ctid = threadIdx.x - CONS0;
+    if (ctid == 0) P->n_distinct[layer] = R.n_distinct;
+    const int np = c.st.T * k;
+    for (int i = ctid; i < np; i += NCT) {
+      if (P->dbg_ids) P->dbg_ids[(size_t)layer * np + i] = R.ids[i];
+      if (P->dbg_w) P->dbg_w[(size_t)layer * np + i] = R.w[i];
+    }
+    if (P->dbg_logits)
+      for (int i = ctid; i < c.st.T * E; i += NCT) P->dbg_logits[(size_t)layer * c.st.T * E + i] = P->logits[i];
+  }
+  if (threadIdx.x == CONS0) {
+    __threadfence_block();
+    c.S->route_ready = layer + 1;
+  }
+}
+
+/* h += sum_slot w * y (slot order); then the next layer's attention norm, or
+ * the bf16 output after the last layer */
+MSK_DEV void phase_comb(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  const Route& R = c.S->route;
+  const int lane = threadIdx.x & 31, k = P->k;
+  const bool last = layer == P->L - 1;
+  for (int t = gwarp(c); t < c.st.T; t += nwarps(c)) {
+    float* h = P->h + (size_t)t * P->d;
+    for (int i = lane * 4; i < P->d; i += 128) {
+      float4 acc = *reinterpret_cast<const float4*>(h + i);
+      for (int s = 0; s < k; ++s) {
+        const float w = R.w[t * k + s];
+        float4 y = *reinterpret_cast<const float4*>(P->y + (size_t)(t * k + s) * P->d + i);
+        acc.x += w * y.x; acc.y += w * y.y; acc.z += w * y.z; acc.w += w * y.w;
+      }
+      *reinterpret_cast<float4*>(h + i) = acc;
+      if (last) {
+        uint16_t* out = c.st.hidden_out + (size_t)t * P->d + i;
+        *reinterpret_cast<uint2*>(out) =
+            make_uint2((uint32_t)f32_to_bf16(acc.x) | ((uint32_t)f32_to_bf16(acc.y) << 16),
+                       (uint32_t)f32_to_bf16(acc.z) | ((uint32_t)f32_to_bf16(acc.w) << 16));
+      }
+    }
+    __syncwarp();
+    if (!last) norm_row(h, P->layers[layer + 1].g_attn, P->d, P->eps, P->x + (size_t)t * P->d, nullptr);
+  }
+}
+
+/* ---- consumer: expert tiles, one pipeline per warp ---------------------------------- */
+MSK_DEV int expert_kc(int K) { return K <= WKC_MAX ? K : (K % 512 == 0 ? 512 : 256); }
+
+/* Copies rows [grow, grow+16) x K-chunk kc of an NVFP4 matrix into dst laid
+ * out codes[16][KC/2] then scales[16][KC/16]: whole rows are one contiguous
+ * bulk copy each; chunks of longer rows are one 2-D tensor box each (maps
+ * cmap/smap over codes [rows][K/2] and scales [rows][K/16]). */
+MSK_DEV void warp_copy_rows(uint8_t* dst, const uint8_t* codes, const uint8_t* scales, const CUtensorMap* cmap,
+                            const CUtensorMap* smap, int64_t grow, int K, int kc, int KC, uint64_t* bar) {
+  const int lane = threadIdx.x & 31;
+  const int cb = KC / 2, sb = KC / 16;
+  if (KC == K) {
+    if (lane == 0) bulk_g2s(dst, codes + grow * (K / 2), 16 * cb, bar);
+    else if (lane == 1) bulk_g2s(dst + 16 * cb, scales + grow * (K / 16), 16 * sb, bar);
+  } else {
+    if (lane == 0) tma_2d_g2s(dst, cmap, kc * cb, (int32_t)grow, bar);
+    else if (lane == 1) tma_2d_g2s(dst + 16 * cb, smap, kc * sb, (int32_t)grow, bar);
+  }
+}
+
+/*
+ * NM 16-row NVFP4 tiles (gate and up, or down alone; mstride bytes apart in
+ * smem, each codes[16][K/2] + scales[16][K/16]) times one 8-column
+ * activation tile whose column rows are bp (this lane's column, or null).
+ * Same k permutation as gemm_warp; the activation fragments are loaded once
+ * for all NM matrices and one block ahead of their use.
+ */
+template <int NM, int BPT>
+MSK_DEV void gemm_rows16(const uint8_t* stg, int mstride, int K, const uint16_t* bp, float (*acc)[4]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const int nwin = K / (64 * BPT);
+  const int nblk = nwin * BPT;
+  const uint32_t sb0 = smem_u32(stg);
+  uint4 bn0 = make_uint4(0, 0, 0, 0), bn1 = bn0;
+  if (bp) {
+    const int kb = 16 * (cq * BPT);
+    bn0 = ldg128(bp + kb);
+    bn1 = ldg128(bp + kb + 8);
+  }
+  for (int win = 0; win < nwin; ++win) {
+    const int kw = win * 64 * BPT;
+    const uint32_t coff = kw / 2 + cq * BPT * 8, soff = 16 * (K / 2) + kw / 16 + cq * BPT;
+    uint32_t w0[NM][2 * BPT], w1[NM][2 * BPT], sw0[NM], sw1[NM];
+#pragma unroll
+    for (int m = 0; m < NM; ++m) {
+      const uint32_t mb = sb0 + m * mstride;
+      const uint32_t r0 = mb + g * (K / 2) + coff, r1 = r0 + 8 * (K / 2);
+      if (BPT == 4) {
+        uint4 a = lds128(r0), b = lds128(r0 + 16), d = lds128(r1), e = lds128(r1 + 16);
+        w0[m][0] = a.x; w0[m][1] = a.y; w0[m][2] = a.z; w0[m][3] = a.w;
+        w0[m][4 % (2 * BPT)] = b.x; w0[m][5 % (2 * BPT)] = b.y; w0[m][6 % (2 * BPT)] = b.z; w0[m][7 % (2 * BPT)] = b.w;
+        w1[m][0] = d.x; w1[m][1] = d.y; w1[m][2] = d.z; w1[m][3] = d.w;
+        w1[m][4 % (2 * BPT)] = e.x; w1[m][5 % (2 * BPT)] = e.y; w1[m][6 % (2 * BPT)] = e.z; w1[m][7 % (2 * BPT)] = e.w;
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
+      } else if (BPT == 2) {
+        uint4 a = lds128(r0), d = lds128(r1);
+        w0[m][0] = a.x; w0[m][1] = a.y; w0[m][2 % (2 * BPT)] = a.z; w0[m][3 % (2 * BPT)] = a.w;
+        w1[m][0] = d.x; w1[m][1] = d.y; w1[m][2 % (2 * BPT)] = d.z; w1[m][3 % (2 * BPT)] = d.w;
+        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
+        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
+      } else {
+        uint2 a = lds64(r0), d = lds64(r1);
+        w0[m][0] = a.x; w0[m][1 % (2 * BPT)] = a.y;
+        w1[m][0] = d.x; w1[m][1 % (2 * BPT)] = d.y;
+        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
+        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
+      }
+    }
+#pragma unroll
+    for (int qb = 0; qb < BPT; ++qb) {
+      const uint4 b0 = bn0, b1 = bn1;
+      const int nxt = win * BPT + qb + 1;
+      if (bp && nxt < nblk) {
+        const int kb = (nxt / BPT) * 64 * BPT + 16 * (cq * BPT + nxt % BPT);
+        bn0 = ldg128(bp + kb);
+        bn1 = ldg128(bp + kb + 8);
+      }
+#pragma unroll
+      for (int m = 0; m < NM; ++m) {
+        const uint32_t s0 = (sw0[m] >> (8 * qb)) & 0xFF, s1 = (sw1[m] >> (8 * qb)) & 0xFF;
+        const uint32_t sc0 = e4m3x2_to_f16x2(s0 | (s0 << 8)), sc1 = e4m3x2_to_f16x2(s1 | (s1 << 8));
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t x0 = w0[m][2 * qb + (s >> 1)] >> (16 * (s & 1));
+          const uint32_t x1 = w1[m][2 * qb + (s >> 1)] >> (16 * (s & 1));
+          uint32_t a[4];
+          a[0] = hmul2(e2m1x2_to_f16x2(x0 & 0xFF), sc0);
+          a[1] = hmul2(e2m1x2_to_f16x2(x1 & 0xFF), sc1);
+          a[2] = hmul2(e2m1x2_to_f16x2((x0 >> 8) & 0xFF), sc0);
+          a[3] = hmul2(e2m1x2_to_f16x2((x1 >> 8) & 0xFF), sc1);
+          const uint4& bb = (s >> 1) ? b1 : b0;
+          mma_f16(acc[m], a, (s & 1) ? bb.z : bb.x, (s & 1) ? bb.w : bb.y);
+        }
+      }
+    }
+  }
+}
+
+/* issue chunk j of this warp's expert items into its ring slot */
+template <bool GU>
+MSK_DEV void expert_issue(const Ctx& c, const MskLayer& Ly, const Route& R, uint8_t* wbase, uint64_t* fb,
+                          uint32_t wit0, int j, int a, int cw, int nkc, int tiles, int rows_unit, int K, int KC,
+                          uint32_t bytes) {
+  const int lane = threadIdx.x & 31;
+  const int item = a + cw + (j / nkc) * NCW, kc = j % nkc;
+  const int unit = item / tiles, tile = item % tiles;
+  const int64_t grow = (int64_t)R.unit_e[unit] * rows_unit + tile * 16;
+  const uint32_t gi = wit0 + (uint32_t)j;
+  uint8_t* dst = wbase + (size_t)(gi % NWS) * WSLOT;
+  uint64_t* bar = &fb[gi % NWS];
+  if (lane == 0) mbar_arrive_tx(bar, bytes);
+  __syncwarp();
+  const MskNv& m0 = GU ? Ly.wg : Ly.wd;
+  const CUtensorMap* mp = Ly.emap + (GU ? 0 : 4);
+  warp_copy_rows(dst, m0.codes, m0.scales, mp, mp + 1, grow, K, kc, KC, bar);
+  if (GU)
+    warp_copy_rows(dst + 16 * (KC / 2 + KC / 16), Ly.wu.codes, Ly.wu.scales, Ly.emap + 2, Ly.emap + 3, grow, K, kc,
+                   KC, bar);
+}
+
+/* gate/up (GU) or down projection of the selected experts.  Items are
+ * (expert unit, 16-row tile); a CTA owns a contiguous item range and its
+ * warps take every 8th item, so the warps of a CTA share the unit's
+ * activation rows in L1.  Each warp streams its items' K chunks through a
+ * 2-slot ring of its own and keeps the whole reduction in registers. */
+template <bool GU, int BPT>
+MSK_DEV bool expert_items(Ctx& c, int layer, uint32_t& wit, int a, int b, int K, int KC, int tiles) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const Route& R = c.S->route;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const int phase = GU ? PH_GU : PH_DN;
+  const int nkc = K / KC;
+  const int cb = KC / 2, sb = KC / 16;
+  const int mine = (b - a > cw) ? (b - a - cw + NCW - 1) / NCW : 0;
+  const int total = mine * nkc;
+  const int rows_unit = GU ? P->f : P->d;
+  uint8_t* wbase = c.ring + (size_t)cw * NWS * WSLOT;
+  uint64_t* fb = c.S->wfull[cw];
+  const uint32_t wit0 = wit;
+  const uint32_t bytes = (GU ? 2u : 1u) * 16u * (uint32_t)(cb + sb);
+  for (int j = 0; j < total && j < NWS; ++j)
+    expert_issue<GU>(c, Ly, R, wbase, fb, wit0, j, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
+  float acc[2][4];
+  int j = 0;
+  bool ok = true;
+  for (; j < total; ++j) {
+    const uint32_t gi = wit0 + (uint32_t)j;
+    if (!wait_bar(c, &fb[gi % NWS], (gi / NWS) & 1, layer, phase)) { ok = false; break; }
+    const uint8_t* stg = wbase + (size_t)(gi % NWS) * WSLOT;
+    const int item = a + cw + (j / nkc) * NCW, kc = j % nkc;
+    const int unit = item / tiles, tile = item % tiles;
+    const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+    if (kc == 0) {
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = 0.f;
+    }
+    const uint16_t* bp = nullptr;
+    if (g < n) {
+      const int pair = R.pairs[st0 + g];
+      bp = GU ? P->x2h + (size_t)(pair / P->k) * P->d + (size_t)kc * KC : P->u + (size_t)pair * P->f + (size_t)kc * KC;
+    }
+    gemm_rows16<GU ? 2 : 1, BPT>(stg, 16 * (cb + sb), KC, bp, acc);
+    __syncwarp();
+    if (j + NWS < total)
+      expert_issue<GU>(c, Ly, R, wbase, fb, wit0, j + NWS, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
+    if (kc == nkc - 1) {
+      const MskNv& m0 = GU ? Ly.wg : Ly.wd;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int col = 2 * cq + (e & 1), row = tile * 16 + g + 8 * (e >> 1);
+        if (col < n) {
+          const int pair = R.pairs[st0 + col];
+          if (GU) {
+            const float gv = acc[0][e] * m0.gs, uv = acc[1][e] * Ly.wu.gs;
+            P->u[(size_t)pair * P->f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
+          } else {
+            P->y[(size_t)pair * P->d + row] = acc[0][e] * m0.gs;
+          }
+        }
+      }
+    }
+  }
+  if (!ok) { /* let the copies in flight land before anything reuses the slots */
+    for (int jj = j; jj < total && jj < j + NWS; ++jj) {
+      const uint32_t gi = wit0 + (uint32_t)jj;
+      uint64_t t0 = gtimer();
+      while (!mbar_try(&fb[gi % NWS], (gi / NWS) & 1))
+        if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+    }
+  }
+  wit = wit0 + (uint32_t)total;
+  return ok;
+}
+
+template <bool GU>
+MSK_DEV bool expert_phase(Ctx& c, int layer, uint32_t& wit) {
+  const MskParams* P = c.P;
+  const Route& R = c.S->route;
+  const int K = GU ? P->d : P->f;
+  const int tiles = (GU ? P->f : P->d) / 16;
+  const int KC = expert_kc(K);
+  int a, b;
+  item_range(R.n_units * tiles, c.cta, c.ncta, &a, &b);
+  const int q = (KC / 64) % 4 == 0 ? 4 : ((KC / 64) % 2 == 0 ? 2 : 1);
+  bool ok = q == 4 ? expert_items<GU, 4>(c, layer, wit, a, b, K, KC, tiles)
+                   : (q == 2 ? expert_items<GU, 2>(c, layer, wit, a, b, K, KC, tiles)
+                             : expert_items<GU, 1>(c, layer, wit, a, b, K, KC, tiles));
+  if (!ok) c.S->abort = 1;
+  named_sync(BAR_CONS, NCT);
+  return !c.S->abort;
+}
+
+/* ---- consumer main loop ---------------------------------------------------------------- */
+template <int HD>
+MSK_DEV void consumer(Ctx& c) {
+  const MskParams* P = c.P;
+  Cons q;
+  q.c = &c;
+  q.it = 0;
+  uint32_t wit = 0; /* this warp's expert chunks so far (its barrier phases) */
+  phase_in(c);
+  if (!grid_sync(c, 0, PH_IN)) return;
+  for (int l = 0; l < P->L; ++l) {
+    const MskLayer& Ly = P->layers[l];
+    /* QKV */
+    {
+      int sQ, sK, nq = qkv_stages(P, &sQ, &sK);
+      const int nqkv = P->qd + 2 * P->kvd;
+      for (int j = c.cta; j < nq; j += c.ncta) {
+        WStage ws = qkv_stage(P, Ly, j, sQ, sK);
+        const int coloff = ws.mat == 0 ? 0 : (ws.mat == 1 ? P->qd : P->qd + P->kvd);
+        bool ok = gemm_stage<MSK_NT_DENSE>(
+            q, ws, c.st.T, [&](int col) { return P->x + (size_t)col * P->d; },
+            [&](int row, int col, float v) {
+              if (row < ws.nrows) P->qkv[(size_t)col * nqkv + coloff + ws.row0 + row] = v;
+            },
+            l, PH_QKV);
+        if (!ok) return;
+      }
+    }
+    if (!grid_sync(c, l, PH_QKV)) return;
+    phase_qknorm(c, l);
+    if (!grid_sync(c, l, PH_QKNORM)) return;
+    if (threadIdx.x == CONS0) c.S->kv_ready = l + 1;
+    bool ok = attention_phase<HD>(q, l);
+    if (!ok) return;
+    if (!grid_sync(c, l, PH_ATT)) return;
+    phase_attc(c, l);
+    if (!grid_sync(c, l, PH_ATTC)) return;
+    {
+      const int nwo = (P->d + rows_per_stage(P->qd) - 1) / rows_per_stage(P->qd);
+      for (int j = c.cta; j < nwo; j += c.ncta) {
+        WStage ws = wo_stage(P, Ly, j);
+        bool ok2 = gemm_stage<MSK_NT_DENSE>(
+            q, ws, c.st.T, [&](int col) { return P->o + (size_t)col * P->qd; },
+            [&](int row, int col, float v) {
+              if (row < ws.nrows) P->h[(size_t)col * P->d + ws.row0 + row] += v;
+            },
+            l, PH_WO);
+        if (!ok2) return;
+      }
+    }
+    if (!grid_sync(c, l, PH_WO)) return;
+    phase_moenorm(c, l);
+    if (!grid_sync(c, l, PH_MOENORM)) return;
+    phase_router(c, l);
+    if (!grid_sync(c, l, PH_ROUTER)) return;
+    phase_topk(c, l);
+    if (!expert_phase<true>(c, l, wit)) return;
+    if (!grid_sync(c, l, PH_GU)) return;
+    if (!expert_phase<false>(c, l, wit)) return;
+    named_sync(BAR_CONS, NCT);
+    if (threadIdx.x == CONS0) c.S->ring_free = l + 1;
+    if (!grid_sync(c, l, PH_DN)) return;
+    phase_comb(c, l);
+    if (l + 1 < P->L && !grid_sync(c, l, PH_COMB)) return;
+  }
+}
+
+}  // namespace
+
+template <int HD>
+__global__ void __launch_bounds__(MSK_NTHREADS, 1)
+    msk_step_kernel(const MskParams* __restrict__ P, const MskStep st, const __grid_constant__ CUtensorMap kvmap) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Ctx c;
+  c.P = P;
+  c.st = st;
+  c.kvmap = &kvmap;
+  c.ring = base;
+  c.scr = reinterpret_cast<float*>(base + (size_t)MSK_NST * MSK_STAGE);
+  c.S = reinterpret_cast<Smem*>(base + (size_t)MSK_NST * MSK_STAGE + MSK_SCR);
+  c.cta = blockIdx.x;
+  c.ncta = gridDim.x;
+  c.nbar = 0;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < MSK_NST; ++i) {
+      mbar_init(&c.S->full[i], 1);
+      mbar_init(&c.S->empty[i], NCW);
+    }
+    c.S->kv_ready = 0;
+    c.S->route_ready = 0;
+    c.S->ring_free = 0;
+    c.S->abort = 0;
+    for (int w = 0; w < MSK_NCW; ++w)
+      for (int i = 0; i < NWS; ++i) mbar_init(&c.S->wfull[w][i], 1);
+    mbar_fence_init();
+  }
+  /* positions: contiguous per sequence, inside the cache */
+  __shared__ int s_bad;
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < st.T; i += blockDim.x) {
+    const int b = i / st.Tq, t = i % st.Tq;
+    const int p = st.positions[i], p0 = st.positions[b * st.Tq];
+    if (p != p0 + t || p0 < 0 || (int64_t)p0 + st.Tq > st.kv_cap) s_bad = 1;
+    if (t == 0) c.S->pos0[b] = p0;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0 && blockIdx.x == 0) atomicCAS(&P->status[ST_CODE], 0u, (uint32_t)MSK_ERR_KV_RANGE);
+    return;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < st.S) {
+    if (threadIdx.x == 0) { P->last_shape[0] = st.S; P->last_shape[1] = st.Tq; }
+    P->last_shape[2 + threadIdx.x] = c.S->pos0[threadIdx.x];
+  }
+  if (threadIdx.x < CONS0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
+    if (threadIdx.x == 0) producer(c);
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_CONSUMER));
+    consumer<HD>(c);
+  }
+}
+
+/* ---- launch ---------------------------------------------------------------------------- */
+extern "C" size_t msk_kernel_smem_bytes() { return SMEM_BYTES; }
+
+static const void* kernel_for(int hd) {
+  return hd == 128 ? (const void*)msk_step_kernel<128> : (const void*)msk_step_kernel<64>;
+}
+
+extern "C" cudaError_t msk_kernel_setup(int hd, int* ctas_per_sm) {
+  const void* k = kernel_for(hd);
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  /* the register split must fit the pool the block is launched with */
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, k);
+  if (e != cudaSuccess) return e;
+  if (128 * REGS_PRODUCER + 2 * 128 * REGS_CONSUMER > MSK_NTHREADS * fa.numRegs) {
+    *ctas_per_sm = 0;
+    return cudaSuccess;
+  }
+  return cudaOccupancyMaxActiveBlocksPerMultiprocessor(ctas_per_sm, k, MSK_NTHREADS, SMEM_BYTES);
+}
+
+extern "C" cudaError_t msk_kernel_launch(int hd, const MskParams* P_dev, const MskStep* st, const CUtensorMap* map,
+                                         int ncta, cudaStream_t stream) {
+  void* args[3] = {(void*)&P_dev, (void*)st, (void*)map};
+  return cudaLaunchCooperativeKernel(kernel_for(hd), dim3(ncta), dim3(MSK_NTHREADS), args, SMEM_BYTES, stream);
+}
