@@ -68,13 +68,13 @@ typedef struct msk_nvfp4 {
 
 typedef struct msk_config {
   int32_t n_layers;       /* 1 .. MSK_MAX_LAYERS */
-  int32_t d_model;        /* multiple of 128, <= 4096 */
+  int32_t d_model;        /* multiple of 128, <= 4096; above 512 a multiple of 512 */
   int32_t n_q_heads;      /* n_q_heads * head_dim <= 4096, multiple of 128 */
   int32_t n_kv_heads;     /* divides n_q_heads */
   int32_t head_dim;       /* 64 or 128 */
   int32_t n_experts;      /* multiple of 32, <= 256 */
   int32_t top_k;          /* 1 .. 8, <= n_experts */
-  int32_t expert_dim;     /* multiple of 128, <= 4096 */
+  int32_t expert_dim;     /* multiple of 128, <= 4096; above 512 a multiple of 512 */
   int32_t window;         /* sliding-window length in keys, >= 1 */
   uint8_t layer_is_sliding[MSK_MAX_LAYERS]; /* 1: sliding-window layer */
   float rms_eps;          /* RMSNorm epsilon (all four norms) */

@@ -74,8 +74,8 @@ static msk_status_t check_config(const msk_config_t* c) {
   if (c->d_model < 128 || c->d_model % 128 || c->d_model > 4096) return MSK_ERR_UNSUPPORTED;
   if (qd % 128 || qd > 4096) return MSK_ERR_UNSUPPORTED;
   if (c->expert_dim < 128 || c->expert_dim % 128 || c->expert_dim > 4096) return MSK_ERR_UNSUPPORTED;
-  /* expert tiles stream K in chunks of 512 or 256: longer rows must split evenly */
-  if ((c->d_model > 512 && c->d_model % 256) || (c->expert_dim > 512 && c->expert_dim % 256))
+  /* expert tiles stream K in chunks of 512: longer rows must split evenly */
+  if ((c->d_model > 512 && c->d_model % 512) || (c->expert_dim > 512 && c->expert_dim % 512))
     return MSK_ERR_UNSUPPORTED;
   if (c->n_experts < 32 || c->n_experts % 32 || c->n_experts > 256) return MSK_ERR_UNSUPPORTED;
   if (c->top_k < 1 || c->top_k > 8 || c->top_k > c->n_experts) return MSK_ERR_INVALID_ARG;
@@ -234,10 +234,10 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       const msk_nvfp4_t* mats[3] = {&w.w_gate, &w.w_up, &w.w_down};
       for (int m = 0; m < 3 && ok; ++m) {
         const int64_t K = m < 2 ? P.d : P.f, rows = (int64_t)P.E * (m < 2 ? P.f : P.d);
-        const int KC = K <= 512 ? (int)K : (K % 512 == 0 ? 512 : 256);
+        const int KC = K <= 512 ? (int)K : 512;
         for (int part = 0; part < 2 && ok; ++part) {
           /* whole-row chunks use plain bulk copies; the map is left zero */
-          if (K <= 512) continue;
+          if (KC == K) continue;
           const int64_t width = part == 0 ? K / 2 : K / 16;
           cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
           cuuint64_t strides[1] = {(cuuint64_t)width};

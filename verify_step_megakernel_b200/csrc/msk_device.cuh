@@ -103,6 +103,19 @@ MSK_DEV uint32_t e2m1x2_to_f16x2(uint32_t byte) {
   asm("{\n .reg .b8 b;\n cvt.u8.u32 b, %1;\n cvt.rn.f16x2.e2m1x2 %0, b;\n}" : "=r"(r) : "r"(byte));
   return r;
 }
+/* four bytes of e2m1 code pairs (byte 0 first) -> four f16x2, exact */
+MSK_DEV void e2m1x8_to_f16x2x4(uint32_t w, uint32_t* o) {
+  asm("{\n .reg .b8 b0, b1, b2, b3;\n mov.b32 {b0, b1, b2, b3}, %4;\n cvt.rn.f16x2.e2m1x2 %0, b0;\n"
+      " cvt.rn.f16x2.e2m1x2 %1, b1;\n cvt.rn.f16x2.e2m1x2 %2, b2;\n cvt.rn.f16x2.e2m1x2 %3, b3;\n}"
+      : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3])
+      : "r"(w));
+}
+/* four e4m3 codes (byte 0 first) -> two f16x2, exact */
+MSK_DEV void e4m3x4_to_f16x2x2(uint32_t w, uint32_t* o) {
+  asm("{\n .reg .b16 h0, h1;\n mov.b32 {h0, h1}, %2;\n cvt.rn.f16x2.e4m3x2 %0, h0;\n cvt.rn.f16x2.e4m3x2 %1, h1;\n}"
+      : "=r"(o[0]), "=r"(o[1])
+      : "r"(w));
+}
 /* two e4m3 codes (low byte first) -> f16x2, exact */
 MSK_DEV uint32_t e4m3x2_to_f16x2(uint32_t two) {
   uint32_t r;
@@ -161,15 +174,16 @@ MSK_DEV float fast_exp2(float x) {
 }
 
 /* ---- tensor-core tile op (m16n8k16, fp32 accumulate) -------------------------------- */
+/* pure register ops: not volatile, so the compiler may interleave them */
 MSK_DEV void mma_f16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 MSK_DEV void mma_bf16(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])

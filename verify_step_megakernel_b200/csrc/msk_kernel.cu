@@ -76,6 +76,7 @@ struct Smem {
   volatile int abort;
   int pos0[MSK_MAX_TOKENS];
   float lbuf[4][32][2];
+  float red8[MSK_NCW];
   Route route;
 };
 
@@ -462,8 +463,14 @@ MSK_DEV void gemm_warp(const uint8_t* stg, int nrows, int K, int ks, int mi, int
     }
 #pragma unroll
     for (int qb = 0; qb < BPT; ++qb) {
-      const uint32_t s0 = (sw0 >> (8 * qb)) & 0xFF, s1 = (sw1 >> (8 * qb)) & 0xFF;
-      const uint32_t sc0 = e4m3x2_to_f16x2(s0 | (s0 << 8)), sc1 = e4m3x2_to_f16x2(s1 | (s1 << 8));
+      uint32_t sc[2];
+      e4m3x4_to_f16x2x2(__byte_perm(sw0, sw1, (uint32_t)(qb | (qb << 4) | ((qb + 4) << 8) | ((qb + 4) << 12))), sc);
+      const uint32_t sc0 = sc[0], sc1 = sc[1];
+      uint32_t r0[8], r1[8];
+      e2m1x8_to_f16x2x4(w0[2 * qb], r0);
+      e2m1x8_to_f16x2x4(w0[2 * qb + 1], r0 + 4);
+      e2m1x8_to_f16x2x4(w1[2 * qb], r1);
+      e2m1x8_to_f16x2x4(w1[2 * qb + 1], r1 + 4);
       const int kb = kw + 16 * (cq * BPT + qb);
       uint4 bl[NT][2];
 #pragma unroll
@@ -477,13 +484,11 @@ MSK_DEV void gemm_warp(const uint8_t* stg, int nrows, int K, int ks, int mi, int
       }
 #pragma unroll
       for (int s = 0; s < 4; ++s) {
-        const uint32_t x0 = w0[2 * qb + (s >> 1)] >> (16 * (s & 1));
-        const uint32_t x1 = w1[2 * qb + (s >> 1)] >> (16 * (s & 1));
         uint32_t a[4];
-        a[0] = hmul2(e2m1x2_to_f16x2(x0 & 0xFF), sc0);
-        a[1] = hmul2(e2m1x2_to_f16x2(x1 & 0xFF), sc1);
-        a[2] = hmul2(e2m1x2_to_f16x2((x0 >> 8) & 0xFF), sc0);
-        a[3] = hmul2(e2m1x2_to_f16x2((x1 >> 8) & 0xFF), sc1);
+        a[0] = hmul2(r0[2 * s], sc0);
+        a[1] = hmul2(r1[2 * s], sc1);
+        a[2] = hmul2(r0[2 * s + 1], sc0);
+        a[3] = hmul2(r1[2 * s + 1], sc1);
 #pragma unroll
         for (int j = 0; j < NT; ++j) {
           if (j < ntl) {
@@ -558,112 +563,141 @@ MSK_DEV uint32_t swz(uint32_t off, int hd) {
   return hd == 128 ? (off ^ (((off >> 7) & 7u) << 4)) : (off ^ (((off >> 7) & 3u) << 4));
 }
 
-template <int HD>
+template <int HD, int MT>
 struct AttState {
-  float o[HD / 8][4];
-  float l0, l1;
-  int lo0, hi0, lo1, hi1; /* key window of rows g and g+8 (empty if lo > hi) */
+  float o[MT][HD / 8][4];
+  float l[MT][2];
+  int lo[MT][2], hi[MT][2]; /* key window of rows g and g+8 of each m-tile (empty if lo > hi) */
+  int lo_max, hi_min;       /* every valid row sees [lo_max, hi_min] */
 };
 
 /* Q of the segment's rows as A fragments in the scratch, fragment order:
- * qf[mi][step][lane] = 16 bytes (a0a1, a2a3, a4a5, a6a7).  Warps with ki == 0
- * fill their m-tile; every consumer warp passes the barrier. */
-template <int HD>
-MSK_DEV void att_begin(const Ctx& c, AttState<HD>& A, int pair, int mi, bool writer) {
+ * qf[m-tile][step][lane] = 16 bytes (a0a1, a2a3, a4a5, a6a7).  Warps with
+ * ki == 0 fill their MT m-tiles; every consumer warp passes the barrier. */
+template <int HD, int MT>
+MSK_DEV void att_begin(const Ctx& c, AttState<HD, MT>& A, int pair, int mg, bool writer, bool sliding) {
   const MskParams* P = c.P;
   const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
   const int b = pair / P->hkv, kvh = pair % P->hkv;
   const int R = c.st.Tq * P->G;
+  A.lo_max = -1;
+  A.hi_min = 0x7FFFFFFF;
 #pragma unroll
-  for (int j = 0; j < HD / 8; ++j) A.o[j][0] = A.o[j][1] = A.o[j][2] = A.o[j][3] = 0.f;
-  A.l0 = A.l1 = 0.f;
-  uint4* qf = reinterpret_cast<uint4*>(c.scr) + (size_t)mi * (HD / 16) * 32;
+  for (int m = 0; m < MT; ++m) {
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int rho = mi * 16 + g + 8 * half;
-    int lo = 1, hi = 0;
-    uint32_t qw[HD / 8];
+    for (int j = 0; j < HD / 8; ++j) A.o[m][j][0] = A.o[m][j][1] = A.o[m][j][2] = A.o[m][j][3] = 0.f;
+    A.l[m][0] = A.l[m][1] = 0.f;
+    const int mi = mg * MT + m;
+    uint32_t* qfw = reinterpret_cast<uint32_t*>(reinterpret_cast<uint4*>(c.scr) + (size_t)mi * (HD / 16) * 32);
 #pragma unroll
-    for (int i = 0; i < HD / 8; ++i) qw[i] = 0;
-    if (rho < R) {
-      const int ti = rho / P->G, h = kvh * P->G + rho % P->G;
-      const int t = b * c.st.Tq + ti;
-      hi = c.S->pos0[b] + ti;
-      lo = 0;
+    for (int half = 0; half < 2; ++half) {
+      const int rho = mi * 16 + g + 8 * half;
+      int lo = 1, hi = 0;
+      uint32_t qw[HD / 8];
+#pragma unroll
+      for (int i = 0; i < HD / 8; ++i) qw[i] = 0;
+      if (rho < R) {
+        const int ti = rho / P->G, h = kvh * P->G + rho % P->G;
+        const int t = b * c.st.Tq + ti;
+        hi = c.S->pos0[b] + ti;
+        lo = sliding ? max(0, hi - P->W + 1) : 0;
+        if (writer) {
+          const uint16_t* qrow = P->qs + (size_t)t * P->qd + h * HD + cq * (HD / 4);
+#pragma unroll
+          for (int i = 0; i < HD / 32; ++i) {
+            uint4 v = ldg128(qrow + 8 * i);
+            qw[4 * i] = v.x; qw[4 * i + 1] = v.y; qw[4 * i + 2] = v.z; qw[4 * i + 3] = v.w;
+          }
+        }
+      }
+      A.lo[m][half] = lo;
+      A.hi[m][half] = hi;
       if (writer) {
-        const uint16_t* qrow = P->qs + (size_t)t * P->qd + h * HD + cq * (HD / 4);
+        /* step s uses q[c*HD/4 + 4s .. +4): words 2s (a0a1 / a2a3) and 2s+1 (a4a5 / a6a7) */
 #pragma unroll
-        for (int i = 0; i < HD / 32; ++i) {
-          uint4 v = ldg128(qrow + 8 * i);
-          qw[4 * i] = v.x; qw[4 * i + 1] = v.y; qw[4 * i + 2] = v.z; qw[4 * i + 3] = v.w;
+        for (int s = 0; s < HD / 16; ++s) {
+          qfw[(s * 32 + lane) * 4 + half] = qw[2 * s];
+          qfw[(s * 32 + lane) * 4 + 2 + half] = qw[2 * s + 1];
         }
       }
     }
-    if (half == 0) { A.lo0 = lo; A.hi0 = hi; } else { A.lo1 = lo; A.hi1 = hi; }
-    if (writer) {
-      /* step s uses q[c*HD/4 + 4s .. +4): words 2s (a0a1 / a2a3) and 2s+1 (a4a5 / a6a7) */
-      uint32_t* qfw = reinterpret_cast<uint32_t*>(qf);
-#pragma unroll
-      for (int s = 0; s < HD / 16; ++s) {
-        qfw[(s * 32 + lane) * 4 + half] = qw[2 * s];
-        qfw[(s * 32 + lane) * 4 + 2 + half] = qw[2 * s + 1];
-      }
-    }
+  }
+  /* the window every valid row of the pair shares (rows differ only in the
+   * draft-block position) */
+  {
+    const int T0 = c.S->pos0[b], T1 = T0 + c.st.Tq - 1;
+    A.hi_min = T0;
+    A.lo_max = sliding ? max(0, T1 - P->W + 1) : 0;
   }
   named_sync(BAR_CONS, NCT);
 }
 
-template <int HD>
-MSK_DEV void att_stage(const Ctx& c, AttState<HD>& A, const uint8_t* stg, int64_t k0, int nkeys, int ks, int mi,
+template <int HD, int MT>
+MSK_DEV void att_stage(const Ctx& c, AttState<HD, MT>& A, const uint8_t* stg, int k0, int nkeys, int ks, int mg,
                        int ki, float scale_log2, float bound_log2) {
   const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
   const uint32_t kbase = smem_u32(stg);
   const int C = (HD == 128) ? 128 : 256;
   const uint32_t vbase = kbase + C * HD;
-  const uint32_t qfb = smem_u32(c.scr) + (uint32_t)(mi * (HD / 16) * 32 + lane) * 16;
+  const uint32_t qfb = smem_u32(c.scr) + (uint32_t)(mg * MT * (HD / 16) * 32 + lane) * 16;
   const float two120 = 1.329227995784916e36f; /* 2^120 */
-  const int k0i = (int)k0;
   for (int kb = ki; kb * 16 < nkeys; kb += ks) {
-    float sacc[2][4];
+    const int kp0 = k0 + kb * 16;
+    const bool full = kb * 16 + 16 <= nkeys && kp0 >= A.lo_max && kp0 + 15 <= A.hi_min;
+    uint32_t kw[2][HD / 16];
 #pragma unroll
     for (int n2 = 0; n2 < 2; ++n2) {
-      sacc[n2][0] = sacc[n2][1] = sacc[n2][2] = sacc[n2][3] = 0.f;
       const uint32_t row = kb * 16 + n2 * 8 + g;
-      uint32_t kw[HD / 16];
 #pragma unroll
       for (int i = 0; i < HD / 64; ++i) {
         uint4 v = lds128(kbase + swz(row * HD + cq * (HD / 4) + 16 * i, HD));
-        kw[4 * i] = v.x; kw[4 * i + 1] = v.y; kw[4 * i + 2] = v.z; kw[4 * i + 3] = v.w;
+        kw[n2][4 * i] = v.x; kw[n2][4 * i + 1] = v.y; kw[n2][4 * i + 2] = v.z; kw[n2][4 * i + 3] = v.w;
       }
+    }
+    float sacc[MT][2][4];
 #pragma unroll
-      for (int s = 0; s < HD / 16; ++s) {
-        const uint4 qv = lds128(qfb + s * 32 * 16);
+    for (int m = 0; m < MT; ++m)
+#pragma unroll
+      for (int n2 = 0; n2 < 2; ++n2) sacc[m][n2][0] = sacc[m][n2][1] = sacc[m][n2][2] = sacc[m][n2][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < HD / 16; ++s) {
+      uint32_t kf0[2], kf1[2];
+      e4m3x4_to_f16x2x2(kw[0][s], kf0);
+      e4m3x4_to_f16x2x2(kw[1][s], kf1);
+      const uint32_t k00 = kf0[0], k01 = kf0[1], k10 = kf1[0], k11 = kf1[1];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) {
+        const uint4 qv = lds128(qfb + (uint32_t)(m * (HD / 16) + s) * 32 * 16);
         const uint32_t qa[4] = {qv.x, qv.y, qv.z, qv.w};
-        mma_f16(sacc[n2], qa, e4m3x2_to_f16x2(kw[s] & 0xFFFF), e4m3x2_to_f16x2(kw[s] >> 16));
+        mma_f16(sacc[m][0], qa, k00, k01);
+        mma_f16(sacc[m][1], qa, k10, k11);
       }
     }
-    /* p = exp(s - M) under the key windows; l in fp32, P as bf16 scaled by 2^120
-     * to match V's 2^-120 */
-    uint32_t pa[4];
+    /* p = exp(s - M) under the key windows; l in fp32, P as bf16 scaled by
+     * 2^120 to match V's 2^-120 */
+    uint32_t pa[MT][4];
 #pragma unroll
-    for (int n2 = 0; n2 < 2; ++n2) {
-      float p[4];
+    for (int m = 0; m < MT; ++m) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kl = kb * 16 + n2 * 8 + 2 * cq + (e & 1);
-        const int kp = k0i + kl;
-        const bool r1 = e >= 2;
-        const bool ok = kl < nkeys && (r1 ? (kp >= A.lo1 && kp <= A.hi1) : (kp >= A.lo0 && kp <= A.hi0));
-        p[e] = ok ? fast_exp2(sacc[n2][e] * scale_log2 - bound_log2) : 0.f;
+      for (int n2 = 0; n2 < 2; ++n2) {
+        float p[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int kl = kb * 16 + n2 * 8 + 2 * cq + (e & 1);
+          const int kp = k0 + kl, hf = e >> 1;
+          const bool ok = full || (kl < nkeys && kp >= A.lo[m][hf] && kp <= A.hi[m][hf]);
+          p[e] = ok ? fast_exp2(sacc[m][n2][e] * scale_log2 - bound_log2) : 0.f;
+        }
+        A.l[m][0] += p[0] + p[1];
+        A.l[m][1] += p[2] + p[3];
+        pa[m][2 * n2] = f32x2_to_bf16x2(p[0] * two120, p[1] * two120);
+        pa[m][2 * n2 + 1] = f32x2_to_bf16x2(p[2] * two120, p[3] * two120);
       }
-      A.l0 += p[0] + p[1];
-      A.l1 += p[2] + p[3];
-      pa[2 * n2] = f32x2_to_bf16x2(p[0] * two120, p[1] * two120);
-      pa[2 * n2 + 1] = f32x2_to_bf16x2(p[2] * two120, p[3] * two120);
     }
-    /* V: lane (g, c) holds columns g*HD/8 .. +HD/8 of keys 2c, 2c+1, 2c+8, 2c+9
-     * (the mma k-slots of this lane: keys 2c, 2c+1 from S tile 0, 8+2c, 9+2c
-     * from S tile 1); read 8 columns at a time */
+    /* V: lane (g, c) holds columns g*HD/8 .. +HD/8 of keys 2c, 2c+1, 2c+8,
+     * 2c+9 (its mma k-slots: keys 2c, 2c+1 from S tile 0, 8+2c, 9+2c from S
+     * tile 1); read 8 columns at a time; each converted fragment feeds MT
+     * m-tiles */
     const uint32_t rA = kb * 16 + 2 * cq;
 #pragma unroll
     for (int hv = 0; hv < HD / 64; ++hv) {
@@ -681,73 +715,85 @@ MSK_DEV void att_stage(const Ctx& c, AttState<HD>& A, const uint8_t* stg, int64_
           const uint32_t sel = (uint32_t)(j | (j << 4) | ((j + 4) << 8) | ((j + 4) << 12));
           const uint32_t b0 = e4m3pair_to_bf16x2_scaled(vw[0][wi], vw[1][wi], sel);
           const uint32_t b1 = e4m3pair_to_bf16x2_scaled(vw[2][wi], vw[3][wi], sel);
-          mma_bf16(A.o[(hv * 2 + wi) * 4 + j], pa, b0, b1);
+#pragma unroll
+          for (int m = 0; m < MT; ++m) mma_bf16(A.o[m][(hv * 2 + wi) * 4 + j], pa[m], b0, b1);
         }
       }
     }
   }
 }
 
-/* Reduce the key-split warps of each m-tile (fixed order) and write the
- * segment's partial (o[rho][0..hd), l at [hd]) to slot `slot`. */
-template <int HD>
-MSK_DEV void att_end(const Ctx& c, AttState<HD>& A, int pair, int slot, int mt, int ks) {
+/* Reduce the key-split warps of each m-tile group (fixed order, one m-tile
+ * at a time through the scratch) and write the segment's partial
+ * (o[rho][0..hd), l at [hd]) to slot `slot`. */
+template <int HD, int MT>
+MSK_DEV void att_end(const Ctx& c, AttState<HD, MT>& A, int slot, int ngroups, int ks) {
   const MskParams* P = c.P;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
-  const bool active = cw < mt * ks;
-  const int mi = active ? cw / ks : 0, ki = active ? cw % ks : 0;
+  const bool active = cw < ngroups * ks;
+  const int mg = active ? cw / ks : 0, ki = active ? cw % ks : 0;
   /* quad-reduce the row sums first (each lane summed its own key columns) */
-  A.l0 += __shfl_xor_sync(0xffffffffu, A.l0, 1);
-  A.l0 += __shfl_xor_sync(0xffffffffu, A.l0, 2);
-  A.l1 += __shfl_xor_sync(0xffffffffu, A.l1, 1);
-  A.l1 += __shfl_xor_sync(0xffffffffu, A.l1, 2);
+#pragma unroll
+  for (int m = 0; m < MT; ++m)
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+      A.l[m][hf] += __shfl_xor_sync(0xffffffffu, A.l[m][hf], 1);
+      A.l[m][hf] += __shfl_xor_sync(0xffffffffu, A.l[m][hf], 2);
+    }
   named_sync(BAR_CONS, NCT); /* every warp is done with the Q fragments */
   float* buf = c.scr;
-  for (int step = ks / 2; step >= 1; step >>= 1) {
-    if (active && ki >= step && ki < 2 * step) {
-      const int bi = mi * step + (ki - step);
-      float* dst = buf + (size_t)bi * (HD / 8) * 128;
 #pragma unroll
-      for (int j = 0; j < HD / 8; ++j)
-        *reinterpret_cast<float4*>(&dst[(j * 32 + lane) * 4]) = make_float4(A.o[j][0], A.o[j][1], A.o[j][2], A.o[j][3]);
-      c.S->lbuf[bi][lane][0] = A.l0;
-      c.S->lbuf[bi][lane][1] = A.l1;
-    }
-    named_sync(BAR_CONS, NCT);
-    if (active && ki < step) {
-      const int bi = mi * step + ki;
-      const float* src = buf + (size_t)bi * (HD / 8) * 128;
+  for (int m = 0; m < MT; ++m) {
+    for (int step = ks / 2; step >= 1; step >>= 1) {
+      if (active && ki >= step && ki < 2 * step) {
+        const int bi = mg * step + (ki - step);
+        float* dst = buf + (size_t)bi * (HD / 8) * 128;
 #pragma unroll
-      for (int j = 0; j < HD / 8; ++j) {
-        float4 v = *reinterpret_cast<const float4*>(&src[(j * 32 + lane) * 4]);
-        A.o[j][0] += v.x; A.o[j][1] += v.y; A.o[j][2] += v.z; A.o[j][3] += v.w;
+        for (int j = 0; j < HD / 8; ++j)
+          *reinterpret_cast<float4*>(&dst[(j * 32 + lane) * 4]) =
+              make_float4(A.o[m][j][0], A.o[m][j][1], A.o[m][j][2], A.o[m][j][3]);
+        c.S->lbuf[bi][lane][0] = A.l[m][0];
+        c.S->lbuf[bi][lane][1] = A.l[m][1];
       }
-      A.l0 += c.S->lbuf[bi][lane][0];
-      A.l1 += c.S->lbuf[bi][lane][1];
+      named_sync(BAR_CONS, NCT);
+      if (active && ki < step) {
+        const int bi = mg * step + ki;
+        const float* src = buf + (size_t)bi * (HD / 8) * 128;
+#pragma unroll
+        for (int j = 0; j < HD / 8; ++j) {
+          float4 v = *reinterpret_cast<const float4*>(&src[(j * 32 + lane) * 4]);
+          A.o[m][j][0] += v.x; A.o[m][j][1] += v.y; A.o[m][j][2] += v.z; A.o[m][j][3] += v.w;
+        }
+        A.l[m][0] += c.S->lbuf[bi][lane][0];
+        A.l[m][1] += c.S->lbuf[bi][lane][1];
+      }
+      named_sync(BAR_CONS, NCT);
     }
-    named_sync(BAR_CONS, NCT);
   }
   if (active && ki == 0) {
     const int R = c.st.Tq * P->G;
     float* base = P->part + (size_t)slot * P->part_stride;
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int rho = mi * 16 + g + 8 * half;
-      if (rho >= R) continue;
-      float* row = base + (size_t)rho * (HD + 4);
+    for (int m = 0; m < MT; ++m) {
 #pragma unroll
-      for (int j = 0; j < HD / 8; ++j) {
-        /* C-fragment column 2c+e of n-tile j is head dim (2c+e)*HD/8 + j */
-        row[(2 * cq) * (HD / 8) + j] = A.o[j][2 * half];
-        row[(2 * cq + 1) * (HD / 8) + j] = A.o[j][2 * half + 1];
+      for (int half = 0; half < 2; ++half) {
+        const int rho = (mg * MT + m) * 16 + g + 8 * half;
+        if (rho >= R) continue;
+        float* row = base + (size_t)rho * (HD + 4);
+#pragma unroll
+        for (int j = 0; j < HD / 8; ++j) {
+          /* C-fragment column 2c+e of n-tile j is head dim (2c+e)*HD/8 + j */
+          row[(2 * cq) * (HD / 8) + j] = A.o[m][j][2 * half];
+          row[(2 * cq + 1) * (HD / 8) + j] = A.o[m][j][2 * half + 1];
+        }
+        if (cq == 0) row[HD] = A.l[m][half];
       }
-      if (cq == 0) row[HD] = half ? A.l1 : A.l0;
     }
   }
 }
 
-template <int HD>
-MSK_DEV bool attention_phase(Cons& q, int layer) {
+template <int HD, int MT>
+MSK_DEV bool attention_phase_mt(Cons& q, int layer) {
   Ctx& c = *q.c;
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
@@ -755,12 +801,11 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
   att_geo(c, layer, g);
   const int R = c.st.Tq * P->G;
   const int mt = (R + 15) / 16;
-  int mp = 1;
-  while (mp < mt) mp <<= 1;
-  const int ks = NCW / mp;
+  const int ngroups = (mt + MT - 1) / MT; /* 1 or 2 */
+  const int ks = NCW / ngroups;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0;
-  const bool active = cw < mt * ks;
-  const int mi = active ? cw / ks : 0, ki = active ? cw % ks : 0;
+  const bool active = cw < ngroups * ks;
+  const int mg = active ? cw / ks : 0, ki = active ? cw % ks : 0;
   const int C = att_keys_per_stage(HD);
   const float scale_log2 = P->scale_log2, bound_log2 = Ly.bound_log2;
   if (c.cta < g.nparts) {
@@ -769,63 +814,89 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
       const int64_t a = max(A0, g.off[p]), b = min(B0, g.off[p + 1]);
       if (a >= b) continue;
       const int k0 = (int)(g.lo[p] + (a - g.off[p])), k1 = (int)(g.lo[p] + (b - g.off[p]));
-      AttState<HD> A;
-      att_begin<HD>(c, A, p, mi, active && ki == 0);
-      if (Ly.sliding) { /* key windows of this layer */
-        if (A.lo0 <= A.hi0) { A.lo0 = A.hi0 - P->W + 1; if (A.lo0 < 0) A.lo0 = 0; }
-        if (A.lo1 <= A.hi1) { A.lo1 = A.hi1 - P->W + 1; if (A.lo1 < 0) A.lo1 = 0; }
-      }
+      AttState<HD, MT> A;
+      att_begin<HD, MT>(c, A, p, mg, active && ki == 0, Ly.sliding != 0);
       for (int x = k0; x < k1; x += C) {
         uint32_t sl;
         const uint8_t* stg = cons_wait(q, layer, PH_ATT, &sl);
         if (stg) {
-          if (active) att_stage<HD>(c, A, stg, x, min(C, k1 - x), ks, mi, ki, scale_log2, bound_log2);
+          if (active) att_stage<HD, MT>(c, A, stg, x, min(C, k1 - x), ks, mg, ki, scale_log2, bound_log2);
           cons_release(q, sl);
         }
       }
-      att_end<HD>(c, A, p, c.cta + p, mt, ks);
+      att_end<HD, MT>(c, A, c.cta + p, ngroups, ks);
     }
   }
   named_sync(BAR_CONS, NCT);
   return !c.S->abort;
 }
 
+/* one warp owns up to two 16-row tiles of a pair (their keys are converted
+ * once); more rows split the warps into two groups */
+template <int HD>
+MSK_DEV bool attention_phase(Cons& q, int layer) {
+  const int R = q.c->st.Tq * q.c->P->G;
+  return R <= 16 ? attention_phase_mt<HD, 1>(q, layer) : attention_phase_mt<HD, 2>(q, layer);
+}
+
 /* ---- consumer: small phases (warp per item over the whole grid) --------------------- */
 MSK_DEV int gwarp(const Ctx& c) { return c.cta * NCW + (threadIdx.x >> 5) - CONS_WARP0; }
 MSK_DEV int nwarps(const Ctx& c) { return c.ncta * NCW; }
 
-/* x = f16(rmsnorm(h) * g) for the row of token t (whole warp) */
-MSK_DEV void norm_row(const float* h, const float* gain, int d, float eps, uint16_t* xh, float* xf) {
-  const int lane = threadIdx.x & 31;
-  float ss = 0.f;
-  for (int i = lane * 4; i < d; i += 128) {
-    float4 v = *reinterpret_cast<const float4*>(h + i);
-    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
-  }
-  ss = warp_sum(ss);
-  const float r = 1.0f / sqrtf(ss / d + eps);
-  for (int i = lane * 4; i < d; i += 128) {
-    float4 v = *reinterpret_cast<const float4*>(h + i);
-    float4 gg = *reinterpret_cast<const float4*>(gain + i);
-    float a = v.x * r * gg.x, b = v.y * r * gg.y, cc = v.z * r * gg.z, dd = v.w * r * gg.w;
-    if (xf) *reinterpret_cast<float4*>(xf + i) = make_float4(a, b, cc, dd);
-    *reinterpret_cast<uint2*>(xh + i) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(cc, dd));
+/* Row work of one token by a whole CTA: the consumer warps split d into
+ * NCW slices (lane-strided float4), the row's sum of squares is reduced in
+ * shared memory in fixed order. */
+constexpr int ROWV = 4; /* float4 per lane per slice: d <= 4096 */
+
+MSK_DEV float cta_sum(const Ctx& c, float part) {
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  part = warp_sum(part);
+  if (lane == 0) c.S->red8[cw] = part;
+  named_sync(BAR_CONS, NCT);
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < NCW; ++i) t += c.S->red8[i];
+  named_sync(BAR_CONS, NCT);
+  return t;
+}
+
+/* xh[i] = f16(v[i] * r * g[i]) (and xf = fp32 copy) over this lane's slice */
+MSK_DEV void row_norm_store(const float4* v, int d, float r, const float* gain, uint16_t* xh, float* xf) {
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  const int sl = d / NCW, base = cw * sl + lane * 4;
+#pragma unroll
+  for (int u = 0; u < ROWV; ++u) {
+    const int i = base + u * 128;
+    if (i < (cw + 1) * sl) {
+      const float4 gg = *reinterpret_cast<const float4*>(gain + i);
+      const float a = v[u].x * r * gg.x, b = v[u].y * r * gg.y, cc = v[u].z * r * gg.z, dd = v[u].w * r * gg.w;
+      if (xf) *reinterpret_cast<float4*>(xf + i) = make_float4(a, b, cc, dd);
+      *reinterpret_cast<uint2*>(xh + i) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(cc, dd));
+    }
   }
 }
 
 MSK_DEV void phase_in(const Ctx& c) {
   const MskParams* P = c.P;
-  const int lane = threadIdx.x & 31;
-  for (int t = gwarp(c); t < c.st.T; t += nwarps(c)) {
-    float* h = P->h + (size_t)t * P->d;
-    const uint16_t* hin = c.st.hidden_in + (size_t)t * P->d;
-    for (int i = lane * 4; i < P->d; i += 128) {
-      uint2 v = *reinterpret_cast<const uint2*>(hin + i);
-      *reinterpret_cast<float4*>(h + i) = make_float4(bf16_to_f32(v.x & 0xFFFF), bf16_to_f32(v.x >> 16),
-                                                      bf16_to_f32(v.y & 0xFFFF), bf16_to_f32(v.y >> 16));
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  const int d = P->d, sl = d / NCW, base = cw * sl + lane * 4;
+  for (int t = c.cta; t < c.st.T; t += c.ncta) {
+    float4 v[ROWV];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < (cw + 1) * sl) {
+        const uint2 hb = *reinterpret_cast<const uint2*>(c.st.hidden_in + (size_t)t * d + i);
+        v[u] = make_float4(bf16_to_f32(hb.x & 0xFFFF), bf16_to_f32(hb.x >> 16), bf16_to_f32(hb.y & 0xFFFF),
+                           bf16_to_f32(hb.y >> 16));
+        *reinterpret_cast<float4*>(P->h + (size_t)t * d + i) = v[u];
+        ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
+      }
     }
-    __syncwarp();
-    norm_row(h, P->layers[0].g_attn, P->d, P->eps, P->x + (size_t)t * P->d, nullptr);
+    const float r = 1.0f / sqrtf(cta_sum(c, ss) / d + P->eps);
+    row_norm_store(v, d, r, P->layers[0].g_attn, P->x + (size_t)t * d, nullptr);
   }
 }
 
@@ -901,38 +972,60 @@ MSK_DEV void phase_attc(const Ctx& c, int layer) {
 
 MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
   const MskParams* P = c.P;
-  for (int t = gwarp(c); t < c.st.T; t += nwarps(c))
-    norm_row(P->h + (size_t)t * P->d, P->layers[layer].g_moe, P->d, P->eps, P->x2h + (size_t)t * P->d,
-             P->x2f + (size_t)t * P->d);
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  const int d = P->d, sl = d / NCW, base = cw * sl + lane * 4;
+  for (int t = c.cta; t < c.st.T; t += c.ncta) {
+    float4 v[ROWV];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < (cw + 1) * sl) {
+        v[u] = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
+        ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
+      }
+    }
+    const float r = 1.0f / sqrtf(cta_sum(c, ss) / d + P->eps);
+    row_norm_store(v, d, r, P->layers[layer].g_moe, P->x2h + (size_t)t * d, P->x2f + (size_t)t * d);
+  }
 }
 
-/* router logits in fp32: items (8 tokens, 8 experts), one expert per warp */
+/* router logits in fp32: warp items (8 tokens, 2 experts); the warps of a
+ * CTA take consecutive expert pairs of the same tokens (shared in L1) */
 MSK_DEV void phase_router(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const float* Wr = P->layers[layer].router;
-  const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - CONS_WARP0;
-  const int ntg = (c.st.T + 7) / 8, neg = P->E / NCW;
-  for (int item = c.cta; item < ntg * neg; item += c.ncta) {
-    const int tg = item / neg, e = (item % neg) * NCW + cw;
+  const int lane = threadIdx.x & 31, d = P->d;
+  const int ntg = (c.st.T + 7) / 8, nep = P->E / 2;
+  for (int item = gwarp(c); item < ntg * nep; item += nwarps(c)) {
+    const int tg = item / nep, e0 = (item % nep) * 2;
     const int nt = min(8, c.st.T - tg * 8);
-    float acc[8];
+    float a0[8], a1[8];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-    const float* wrow = Wr + (size_t)e * P->d;
-    for (int i = lane * 4; i < P->d; i += 128) {
-      float4 w = *reinterpret_cast<const float4*>(wrow + i);
+    for (int j = 0; j < 8; ++j) a0[j] = a1[j] = 0.f;
+    const float* w0p = Wr + (size_t)e0 * d;
+    const float* w1p = w0p + d;
+    const float* xp = P->x2f + (size_t)tg * 8 * d;
+#pragma unroll 2
+    for (int i = lane * 4; i < d; i += 128) {
+      const float4 w0 = *reinterpret_cast<const float4*>(w0p + i), w1 = *reinterpret_cast<const float4*>(w1p + i);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j < nt) {
-          float4 x = *reinterpret_cast<const float4*>(P->x2f + (size_t)(tg * 8 + j) * P->d + i);
-          acc[j] += w.x * x.x + w.y * x.y + w.z * x.z + w.w * x.w;
+          const float4 x = *reinterpret_cast<const float4*>(xp + (size_t)j * d + i);
+          a0[j] += w0.x * x.x + w0.y * x.y + w0.z * x.z + w0.w * x.w;
+          a1[j] += w1.x * x.x + w1.y * x.y + w1.z * x.z + w1.w * x.w;
         }
       }
     }
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float s = warp_sum(acc[j]);
-      if (lane == 0 && j < nt) P->logits[(size_t)(tg * 8 + j) * P->E + e] = s;
+      const float s0 = warp_sum(a0[j]), s1 = warp_sum(a1[j]);
+      if (lane == 0 && j < nt) {
+        P->logits[(size_t)(tg * 8 + j) * P->E + e0] = s0;
+        P->logits[(size_t)(tg * 8 + j) * P->E + e0 + 1] = s1;
+      }
     }
   }
 }
@@ -1052,36 +1145,47 @@ MSK_DEV void phase_topk(Ctx& c, int layer) {
 }
 
 /* h += sum_slot w * y (slot order); then the next layer's attention norm, or
- * the bf16 output after the last layer */
+ * the bf16 output after the last layer.  One CTA per token. */
 MSK_DEV void phase_comb(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const Route& R = c.S->route;
-  const int lane = threadIdx.x & 31, k = P->k;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, k = P->k;
+  const int d = P->d, sl = d / NCW, base = cw * sl + lane * 4;
   const bool last = layer == P->L - 1;
-  for (int t = gwarp(c); t < c.st.T; t += nwarps(c)) {
-    float* h = P->h + (size_t)t * P->d;
-    for (int i = lane * 4; i < P->d; i += 128) {
-      float4 acc = *reinterpret_cast<const float4*>(h + i);
-      for (int s = 0; s < k; ++s) {
-        const float w = R.w[t * k + s];
-        float4 y = *reinterpret_cast<const float4*>(P->y + (size_t)(t * k + s) * P->d + i);
-        acc.x += w * y.x; acc.y += w * y.y; acc.z += w * y.z; acc.w += w * y.w;
-      }
-      *reinterpret_cast<float4*>(h + i) = acc;
-      if (last) {
-        uint16_t* out = c.st.hidden_out + (size_t)t * P->d + i;
-        *reinterpret_cast<uint2*>(out) =
-            make_uint2((uint32_t)f32_to_bf16(acc.x) | ((uint32_t)f32_to_bf16(acc.y) << 16),
-                       (uint32_t)f32_to_bf16(acc.z) | ((uint32_t)f32_to_bf16(acc.w) << 16));
+  for (int t = c.cta; t < c.st.T; t += c.ncta) {
+    float4 v[ROWV];
+    float ss = 0.f;
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < (cw + 1) * sl) {
+        float4 acc = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
+        for (int s = 0; s < k; ++s) {
+          const float w = R.w[t * k + s];
+          const float4 y = *reinterpret_cast<const float4*>(P->y + (size_t)(t * k + s) * d + i);
+          acc.x += w * y.x; acc.y += w * y.y; acc.z += w * y.z; acc.w += w * y.w;
+        }
+        v[u] = acc;
+        *reinterpret_cast<float4*>(P->h + (size_t)t * d + i) = acc;
+        ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
+        if (last) {
+          uint16_t* out = c.st.hidden_out + (size_t)t * d + i;
+          *reinterpret_cast<uint2*>(out) =
+              make_uint2((uint32_t)f32_to_bf16(acc.x) | ((uint32_t)f32_to_bf16(acc.y) << 16),
+                         (uint32_t)f32_to_bf16(acc.z) | ((uint32_t)f32_to_bf16(acc.w) << 16));
+        }
       }
     }
-    __syncwarp();
-    if (!last) norm_row(h, P->layers[layer + 1].g_attn, P->d, P->eps, P->x + (size_t)t * P->d, nullptr);
+    if (!last) {
+      const float r = 1.0f / sqrtf(cta_sum(c, ss) / d + P->eps);
+      row_norm_store(v, d, r, P->layers[layer + 1].g_attn, P->x + (size_t)t * d, nullptr);
+    }
   }
 }
 
 /* ---- consumer: expert tiles, one pipeline per warp ---------------------------------- */
-MSK_DEV int expert_kc(int K) { return K <= WKC_MAX ? K : (K % 512 == 0 ? 512 : 256); }
+MSK_DEV int expert_kc(int K) { return K <= WKC_MAX ? K : WKC_MAX; } /* K <= 512 or a multiple of 512 */
 
 /* Copies rows [grow, grow+16) x K-chunk kc of an NVFP4 matrix into dst laid
  * out codes[16][KC/2] then scales[16][KC/16]: whole rows are one contiguous
@@ -1103,87 +1207,120 @@ MSK_DEV void warp_copy_rows(uint8_t* dst, const uint8_t* codes, const uint8_t* s
 /*
  * NM 16-row NVFP4 tiles (gate and up, or down alone; mstride bytes apart in
  * smem, each codes[16][K/2] + scales[16][K/16]) times one 8-column
- * activation tile whose column rows are bp (this lane's column, or null).
- * Same k permutation as gemm_warp; the activation fragments are loaded once
- * for all NM matrices and one block ahead of their use.
+ * activation tile.  bq holds this lane's activation fragments of the whole
+ * chunk (block b: bq[2b], bq[2b+1]), loaded a chunk ahead by the caller.
+ * Same k permutation as gemm_warp; each fragment feeds all NM matrices.
  */
+constexpr int EBLK = WKC_MAX / 16 / 4; /* blocks per lane per 512-wide chunk: 8 */
+constexpr int EPF = 1;                  /* activation prefetch distance in blocks */
+
 template <int NM, int BPT>
-MSK_DEV void gemm_rows16(const uint8_t* stg, int mstride, int K, const uint16_t* bp, float (*acc)[4]) {
+MSK_DEV void gemm_rows16(const uint8_t* stg, int mstride, int K, uint4* bq, const uint16_t* cur_bp,
+                         const uint16_t* next_bp, float (*acc)[4], float (*acc2)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
   const int nwin = K / (64 * BPT);
-  const int nblk = nwin * BPT;
+  const int nblk = K / 64;
   const uint32_t sb0 = smem_u32(stg);
-  uint4 bn0 = make_uint4(0, 0, 0, 0), bn1 = bn0;
-  if (bp) {
-    const int kb = 16 * (cq * BPT);
-    bn0 = ldg128(bp + kb);
-    bn1 = ldg128(bp + kb + 8);
-  }
-  for (int win = 0; win < nwin; ++win) {
+#pragma unroll
+  for (int win = 0; win < WKC_MAX / (64 * BPT); ++win) {
+    if (win >= nwin) break;
     const int kw = win * 64 * BPT;
     const uint32_t coff = kw / 2 + cq * BPT * 8, soff = 16 * (K / 2) + kw / 16 + cq * BPT;
-    uint32_t w0[NM][2 * BPT], w1[NM][2 * BPT], sw0[NM], sw1[NM];
+    uint32_t sw0[NM], sw1[NM];
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
       const uint32_t mb = sb0 + m * mstride;
-      const uint32_t r0 = mb + g * (K / 2) + coff, r1 = r0 + 8 * (K / 2);
       if (BPT == 4) {
-        uint4 a = lds128(r0), b = lds128(r0 + 16), d = lds128(r1), e = lds128(r1 + 16);
-        w0[m][0] = a.x; w0[m][1] = a.y; w0[m][2] = a.z; w0[m][3] = a.w;
-        w0[m][4 % (2 * BPT)] = b.x; w0[m][5 % (2 * BPT)] = b.y; w0[m][6 % (2 * BPT)] = b.z; w0[m][7 % (2 * BPT)] = b.w;
-        w1[m][0] = d.x; w1[m][1] = d.y; w1[m][2] = d.z; w1[m][3] = d.w;
-        w1[m][4 % (2 * BPT)] = e.x; w1[m][5 % (2 * BPT)] = e.y; w1[m][6 % (2 * BPT)] = e.z; w1[m][7 % (2 * BPT)] = e.w;
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
         asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
       } else if (BPT == 2) {
-        uint4 a = lds128(r0), d = lds128(r1);
-        w0[m][0] = a.x; w0[m][1] = a.y; w0[m][2 % (2 * BPT)] = a.z; w0[m][3 % (2 * BPT)] = a.w;
-        w1[m][0] = d.x; w1[m][1] = d.y; w1[m][2 % (2 * BPT)] = d.z; w1[m][3 % (2 * BPT)] = d.w;
         asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
         asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
       } else {
-        uint2 a = lds64(r0), d = lds64(r1);
-        w0[m][0] = a.x; w0[m][1 % (2 * BPT)] = a.y;
-        w1[m][0] = d.x; w1[m][1 % (2 * BPT)] = d.y;
         asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
         asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
       }
     }
 #pragma unroll
     for (int qb = 0; qb < BPT; ++qb) {
-      const uint4 b0 = bn0, b1 = bn1;
-      const int nxt = win * BPT + qb + 1;
-      if (bp && nxt < nblk) {
-        const int kb = (nxt / BPT) * 64 * BPT + 16 * (cq * BPT + nxt % BPT);
-        bn0 = ldg128(bp + kb);
-        bn1 = ldg128(bp + kb + 8);
+      const int blk = win * BPT + qb;
+      const int rs = blk % EPF; /* ring slot of this block's fragments */
+      const uint4 b0 = bq[2 * rs], b1 = bq[2 * rs + 1];
+      /* refill the slot with the fragments EPF blocks ahead (in this chunk
+       * or the next one): half a chunk of work hides their latency */
+      {
+        const int ab = blk + EPF;
+        const uint16_t* src = ab < nblk ? cur_bp : next_bp;
+        const int bb = ab < nblk ? ab : ab - nblk;
+        if (src) {
+          const int kb = (bb / BPT) * 64 * BPT + 16 * (cq * BPT + bb % BPT);
+          bq[2 * rs] = ldg128(src + kb);
+          bq[2 * rs + 1] = ldg128(src + kb + 8);
+        } else {
+          bq[2 * rs] = bq[2 * rs + 1] = make_uint4(0, 0, 0, 0);
+        }
       }
 #pragma unroll
       for (int m = 0; m < NM; ++m) {
-        const uint32_t s0 = (sw0[m] >> (8 * qb)) & 0xFF, s1 = (sw1[m] >> (8 * qb)) & 0xFF;
-        const uint32_t sc0 = e4m3x2_to_f16x2(s0 | (s0 << 8)), sc1 = e4m3x2_to_f16x2(s1 | (s1 << 8));
+        const uint32_t mb = sb0 + m * mstride;
+        /* this block's 16 codes of rows g and g+8 (8 bytes each) */
+        const uint2 c0 = lds64(mb + g * (K / 2) + coff + qb * 8), c1 = lds64(mb + (g + 8) * (K / 2) + coff + qb * 8);
+        /* the block's scales of rows g and g+8, broadcast to f16x2 */
+        const uint32_t s01 = __byte_perm(sw0[m], sw1[m], (uint32_t)(qb | (qb << 4) | ((qb + 4) << 8) | ((qb + 4) << 12)));
+        uint32_t sc[2];
+        e4m3x4_to_f16x2x2(s01, sc);
+        uint32_t r0[8], r1[8];
+        e2m1x8_to_f16x2x4(c0.x, r0);
+        e2m1x8_to_f16x2x4(c0.y, r0 + 4);
+        e2m1x8_to_f16x2x4(c1.x, r1);
+        e2m1x8_to_f16x2x4(c1.y, r1 + 4);
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
-          const uint32_t x0 = w0[m][2 * qb + (s >> 1)] >> (16 * (s & 1));
-          const uint32_t x1 = w1[m][2 * qb + (s >> 1)] >> (16 * (s & 1));
           uint32_t a[4];
-          a[0] = hmul2(e2m1x2_to_f16x2(x0 & 0xFF), sc0);
-          a[1] = hmul2(e2m1x2_to_f16x2(x1 & 0xFF), sc1);
-          a[2] = hmul2(e2m1x2_to_f16x2((x0 >> 8) & 0xFF), sc0);
-          a[3] = hmul2(e2m1x2_to_f16x2((x1 >> 8) & 0xFF), sc1);
+          a[0] = hmul2(r0[2 * s], sc[0]);
+          a[1] = hmul2(r1[2 * s], sc[1]);
+          a[2] = hmul2(r0[2 * s + 1], sc[0]);
+          a[3] = hmul2(r1[2 * s + 1], sc[1]);
           const uint4& bb = (s >> 1) ? b1 : b0;
-          mma_f16(acc[m], a, (s & 1) ? bb.z : bb.x, (s & 1) ? bb.w : bb.y);
+          /* alternate two accumulators: two independent mma chains */
+          mma_f16((s & 1) ? acc2[m] : acc[m], a, (s & 1) ? bb.z : bb.x, (s & 1) ? bb.w : bb.y);
         }
       }
     }
   }
 }
 
+/* this lane's activation fragments of the first EPF blocks of a chunk (K
+ * chunk KC, BPT blocks per window) from row bp (null: zeros) */
+template <int BPT>
+MSK_DEV void load_bchunk(const uint16_t* bp, int KC, uint4* bq) {
+  const int cq = threadIdx.x & 3;
+  const int nblk = KC / 64;
+#pragma unroll
+  for (int bl = 0; bl < EPF; ++bl) {
+    if (bl < nblk && bp) {
+      const int kb = (bl / BPT) * 64 * BPT + 16 * (cq * BPT + bl % BPT);
+      bq[2 * bl] = ldg128(bp + kb);
+      bq[2 * bl + 1] = ldg128(bp + kb + 8);
+    } else {
+      bq[2 * bl] = bq[2 * bl + 1] = make_uint4(0, 0, 0, 0);
+    }
+  }
+}
+
+/* the expert tensors of one phase, read once from the parameter block */
+struct ExpMats {
+  const uint8_t* codes[2];
+  const uint8_t* scales[2];
+  const CUtensorMap* cmap[2];
+  const CUtensorMap* smap[2];
+  float gs[2];
+};
+
 /* issue chunk j of this warp's expert items into its ring slot */
 template <bool GU>
-MSK_DEV void expert_issue(const Ctx& c, const MskLayer& Ly, const Route& R, uint8_t* wbase, uint64_t* fb,
-                          uint32_t wit0, int j, int a, int cw, int nkc, int tiles, int rows_unit, int K, int KC,
-                          uint32_t bytes) {
+MSK_DEV void expert_issue(const ExpMats& M, const Route& R, uint8_t* wbase, uint64_t* fb, uint32_t wit0, int j, int a,
+                          int cw, int nkc, int tiles, int rows_unit, int K, int KC, uint32_t bytes) {
   const int lane = threadIdx.x & 31;
   const int item = a + cw + (j / nkc) * NCW, kc = j % nkc;
   const int unit = item / tiles, tile = item % tiles;
@@ -1193,12 +1330,9 @@ MSK_DEV void expert_issue(const Ctx& c, const MskLayer& Ly, const Route& R, uint
   uint64_t* bar = &fb[gi % NWS];
   if (lane == 0) mbar_arrive_tx(bar, bytes);
   __syncwarp();
-  const MskNv& m0 = GU ? Ly.wg : Ly.wd;
-  const CUtensorMap* mp = Ly.emap + (GU ? 0 : 4);
-  warp_copy_rows(dst, m0.codes, m0.scales, mp, mp + 1, grow, K, kc, KC, bar);
+  warp_copy_rows(dst, M.codes[0], M.scales[0], M.cmap[0], M.smap[0], grow, K, kc, KC, bar);
   if (GU)
-    warp_copy_rows(dst + 16 * (KC / 2 + KC / 16), Ly.wu.codes, Ly.wu.scales, Ly.emap + 2, Ly.emap + 3, grow, K, kc,
-                   KC, bar);
+    warp_copy_rows(dst + 16 * (KC / 2 + KC / 16), M.codes[1], M.scales[1], M.cmap[1], M.smap[1], grow, K, kc, KC, bar);
 }
 
 /* gate/up (GU) or down projection of the selected experts.  Items are
@@ -1217,14 +1351,41 @@ MSK_DEV bool expert_items(Ctx& c, int layer, uint32_t& wit, int a, int b, int K,
   const int cb = KC / 2, sb = KC / 16;
   const int mine = (b - a > cw) ? (b - a - cw + NCW - 1) / NCW : 0;
   const int total = mine * nkc;
-  const int rows_unit = GU ? P->f : P->d;
+  /* everything the loop needs from the parameter block, read once */
+  const int d = P->d, f = P->f, topk = P->k;
+  const int rows_unit = GU ? f : d;
+  const uint16_t* act = GU ? P->x2h : P->u;
+  const int act_ld = GU ? d : f;
+  uint16_t* uout = P->u;
+  float* yout = P->y;
+  ExpMats M;
+  M.codes[0] = GU ? Ly.wg.codes : Ly.wd.codes;
+  M.scales[0] = GU ? Ly.wg.scales : Ly.wd.scales;
+  M.codes[1] = Ly.wu.codes;
+  M.scales[1] = Ly.wu.scales;
+  M.cmap[0] = Ly.emap + (GU ? 0 : 4);
+  M.smap[0] = Ly.emap + (GU ? 1 : 5);
+  M.cmap[1] = Ly.emap + 2;
+  M.smap[1] = Ly.emap + 3;
+  M.gs[0] = GU ? Ly.wg.gs : Ly.wd.gs;
+  M.gs[1] = Ly.wu.gs;
   uint8_t* wbase = c.ring + (size_t)cw * NWS * WSLOT;
   uint64_t* fb = c.S->wfull[cw];
   const uint32_t wit0 = wit;
   const uint32_t bytes = (GU ? 2u : 1u) * 16u * (uint32_t)(cb + sb);
+  /* row of this lane's activation column for chunk j (null past the unit) */
+  auto act_row = [&](int jj) -> const uint16_t* {
+    const int item = a + cw + (jj / nkc) * NCW, kc = jj % nkc;
+    const int unit = item / tiles;
+    if (g >= R.unit_n[unit]) return nullptr;
+    const int pair = R.pairs[R.unit_start[unit] + g];
+    return act + (size_t)(GU ? pair / topk : pair) * act_ld + (size_t)kc * KC;
+  };
   for (int j = 0; j < total && j < NWS; ++j)
-    expert_issue<GU>(c, Ly, R, wbase, fb, wit0, j, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
-  float acc[2][4];
+    expert_issue<GU>(M, R, wbase, fb, wit0, j, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
+  uint4 bq[2 * EPF];
+  if (total > 0) load_bchunk<BPT>(act_row(0), KC, bq);
+  float acc[2][4], acc2[2][4];
   int j = 0;
   bool ok = true;
   for (; j < total; ++j) {
@@ -1232,33 +1393,27 @@ MSK_DEV bool expert_items(Ctx& c, int layer, uint32_t& wit, int a, int b, int K,
     if (!wait_bar(c, &fb[gi % NWS], (gi / NWS) & 1, layer, phase)) { ok = false; break; }
     const uint8_t* stg = wbase + (size_t)(gi % NWS) * WSLOT;
     const int item = a + cw + (j / nkc) * NCW, kc = j % nkc;
-    const int unit = item / tiles, tile = item % tiles;
-    const int n = R.unit_n[unit], st0 = R.unit_start[unit];
     if (kc == 0) {
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = acc2[0][e] = acc2[1][e] = 0.f;
     }
-    const uint16_t* bp = nullptr;
-    if (g < n) {
-      const int pair = R.pairs[st0 + g];
-      bp = GU ? P->x2h + (size_t)(pair / P->k) * P->d + (size_t)kc * KC : P->u + (size_t)pair * P->f + (size_t)kc * KC;
-    }
-    gemm_rows16<GU ? 2 : 1, BPT>(stg, 16 * (cb + sb), KC, bp, acc);
+    gemm_rows16<GU ? 2 : 1, BPT>(stg, 16 * (cb + sb), KC, bq, act_row(j), j + 1 < total ? act_row(j + 1) : nullptr, acc,
+                                 acc2);
     __syncwarp();
-    if (j + NWS < total)
-      expert_issue<GU>(c, Ly, R, wbase, fb, wit0, j + NWS, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
+    if (j + NWS < total) expert_issue<GU>(M, R, wbase, fb, wit0, j + NWS, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
     if (kc == nkc - 1) {
-      const MskNv& m0 = GU ? Ly.wg : Ly.wd;
+      const int unit = item / tiles, tile = item % tiles;
+      const int n = R.unit_n[unit], st0 = R.unit_start[unit];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = 2 * cq + (e & 1), row = tile * 16 + g + 8 * (e >> 1);
         if (col < n) {
           const int pair = R.pairs[st0 + col];
           if (GU) {
-            const float gv = acc[0][e] * m0.gs, uv = acc[1][e] * Ly.wu.gs;
-            P->u[(size_t)pair * P->f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
+            const float gv = (acc[0][e] + acc2[0][e]) * M.gs[0], uv = (acc[1][e] + acc2[1][e]) * M.gs[1];
+            uout[(size_t)pair * f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
           } else {
-            P->y[(size_t)pair * P->d + row] = acc[0][e] * m0.gs;
+            yout[(size_t)pair * d + row] = (acc[0][e] + acc2[0][e]) * M.gs[0];
           }
         }
       }
