@@ -173,6 +173,43 @@ msk_status_t msk_kv_read(msk_handle_t* h, msk_kv_t* kv, int layer, int seq, int6
 msk_status_t msk_step(msk_handle_t* h, const uint16_t* hidden_in, const int32_t* positions, int n_seqs,
                       int tokens_per_seq, msk_kv_t* kv, uint16_t* hidden_out, void* stream);
 
+/* Size of the working-memory array built into the library for
+ * msk_step_static (8 MiB per device). */
+#define MSK_STATIC_SCRATCH_BYTES (8u << 20)
+
+/* msk_step with no allocation behind it.  The blog post has no counterpart
+ * of this call: it is an integration aid of this library.
+ *
+ * Who needs it: a caller that must not let the library allocate device
+ * memory at step time or tie a step's working memory to one handle -- for
+ * instance a serving engine that hands all free HBM to its own KV-block
+ * pool after start-up (so any later cudaMalloc fails or fragments the pool)
+ * and wants the step's footprint fixed and known when the library loads.
+ *
+ * Same arguments, same results and same kernel as msk_step; the difference
+ * is where the step's working buffers (residual, projections, attention
+ * partials, expert activations, barrier words) and the kernel's copy of the
+ * parameter block live: in one array of MSK_STATIC_SCRATCH_BYTES compiled
+ * into the library, shared by every handle on a device.  The call allocates
+ * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
+ *  - First call on a device: looks the array's device address up
+ *    (cudaGetSymbolAddress) with that device current, once; later calls
+ *    reuse it.  Make that first call before any stream capture begins.
+ *  - Enqueues one small kernel that copies the handle's parameter block into
+ *    the array and zeroes the barrier words (the only bytes that must start
+ *    at zero), then the step kernel; no host synchronisation.
+ *  - Device status and statistics still go to the handle: msk_step_status
+ *    and msk_query work after it as after msk_step.
+ *  - Returns MSK_ERR_UNSUPPORTED, before any device work, when the handle's
+ *    shapes need more working memory than the array holds (about 6.7 MiB for
+ *    16 tokens of d_model 2048; 64 tokens of d_model 4096 do not fit), or the
+ *    device index is 64 or more; MSK_ERR_CUDA if the lookup fails.
+ *  - All calls on a device share the array: two such steps in flight at the
+ *    same time on one device (other streams, handles or threads) race and
+ *    corrupt each other.  Order them on one stream, or use msk_step. */
+msk_status_t msk_step_static(msk_handle_t* h, const uint16_t* hidden_in, const int32_t* positions, int n_seqs,
+                             int tokens_per_seq, msk_kv_t* kv, uint16_t* hidden_out, void* stream);
+
 /* Device status of the steps since the last call (call after synchronising
  * the stream); clears it. */
 msk_status_t msk_step_status(msk_handle_t* h);

@@ -58,7 +58,8 @@ class Stats(C.Structure):
 
 _lib = None
 EXPORTS = ["msk_create", "msk_destroy", "msk_kv_create", "msk_kv_destroy", "msk_kv_append", "msk_kv_read",
-           "msk_step", "msk_step_status", "msk_set_debug", "msk_query", "msk_status_string"]
+           "msk_step", "msk_step_static", "msk_step_status", "msk_set_debug", "msk_query", "msk_status_string"]
+STATIC_SCRATCH_BYTES = 8 << 20
 
 
 def lib():
@@ -77,13 +78,14 @@ def lib():
         L.msk_kv_append.argtypes = [P, P, I, I, I64, I64, P, P, P]
         L.msk_kv_read.argtypes = [P, P, I, I, I64, I64, P, P]
         L.msk_step.argtypes = [P, P, P, I, I, P, P, P]
+        L.msk_step_static.argtypes = [P, P, P, I, I, P, P, P]
         L.msk_step_status.argtypes = [P]
         L.msk_set_debug.argtypes = [P, C.POINTER(Debug)]
         L.msk_query.argtypes = [P, C.POINTER(Stats)]
         L.msk_status_string.argtypes = [I]
         L.msk_status_string.restype = C.c_char_p
         for name in ("msk_create", "msk_kv_create", "msk_kv_append", "msk_kv_read", "msk_step",
-                     "msk_step_status", "msk_set_debug", "msk_query"):
+                     "msk_step_static", "msk_step_status", "msk_set_debug", "msk_query"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -125,6 +127,13 @@ def msk_kv_read(h, kv, layer, seq, pos0, n, k_out, v_out):
 
 def msk_step(h, hidden_in, positions, n_seqs, tokens_per_seq, kv, hidden_out, stream=0):
     _check(lib().msk_step(h, hidden_in, positions, n_seqs, tokens_per_seq, kv, hidden_out, stream), "msk_step")
+
+
+def msk_step_static(h, hidden_in, positions, n_seqs, tokens_per_seq, kv, hidden_out, stream=0):
+    """msk_step with its working memory in the library's fixed array (no
+    allocation); see include/msk.h for who needs it and its limits."""
+    _check(lib().msk_step_static(h, hidden_in, positions, n_seqs, tokens_per_seq, kv, hidden_out, stream),
+           "msk_step_static")
 
 
 def msk_step_status(h) -> int:

@@ -9,6 +9,7 @@
 #include <stdlib.h>
 #include <string.h>
 
+#include <mutex>
 #include <new>
 
 #include "msk_internal.h"
@@ -87,6 +88,94 @@ static msk_status_t check_config(const msk_config_t* c) {
   if (c->max_seqs * c->n_kv_heads > MSK_MAX_PAIRS) return MSK_ERR_UNSUPPORTED;
   if (c->wait_timeout_us < 0) return MSK_ERR_INVALID_ARG;
   return MSK_OK;
+}
+
+/* ---- working memory compiled into the library (msk_step_static) -------------------------
+ * msk_step_static runs the same step kernel as msk_step, but its per-step
+ * working buffers and its copy of the parameter block live in this fixed
+ * array instead of the handle's allocation.  The array is zero when the
+ * module loads; only the control words (barrier counter, abort word) must be
+ * zero when a step starts, and the parameter kernel below clears them before
+ * every step.  Every call on a device uses the same bytes, so two such steps
+ * in flight at once on one device (two streams, two handles, two threads)
+ * overwrite each other's buffers. */
+static __device__ __align__(256) uint8_t g_static_scratch[MSK_STATIC_SCRATCH_BYTES];
+
+#define MSK_STATIC_MAX_DEVICES 64
+struct StaticSlot {
+  std::once_flag once;
+  uint8_t* ptr;
+  cudaError_t err;
+};
+static StaticSlot g_static_slots[MSK_STATIC_MAX_DEVICES];
+
+/* where the step's buffers sit inside g_static_scratch */
+struct StaticLayout {
+  size_t params, h, x, qkv, qs, part, o, x2f, x2h, logits, u, y, ctrl, total;
+};
+
+static StaticLayout static_layout(const msk_handle_t* h) {
+  const MskParams& P = h->host;
+  const msk_config_t& c = h->cfg;
+  const size_t T = (size_t)P.max_T, d = P.d, qd = P.qd, kvd = P.kvd;
+  const size_t slots = (size_t)h->ncta + (size_t)c.max_seqs * P.hkv;
+  StaticLayout L;
+  size_t at = 0;
+  auto take = [&at](size_t bytes) { const size_t o = at; at += (bytes + 255) & ~(size_t)255; return o; };
+  L.params = take(sizeof(MskParams));
+  L.h = take(T * d * 4);
+  L.x = take(T * d * 2);
+  L.qkv = take(T * (qd + 2 * kvd) * 4);
+  L.qs = take(T * qd * 2);
+  L.part = take(slots * (size_t)P.part_stride * 4);
+  L.o = take(T * qd * 2);
+  L.x2f = take(T * d * 4);
+  L.x2h = take(T * d * 2);
+  L.logits = take(T * P.E * 4);
+  L.u = take(T * P.k * P.f * 2);
+  L.y = take(T * P.k * d * 4);
+  L.ctrl = take(CTRL_WORDS * 4);
+  L.total = at;
+  return L;
+}
+
+struct StaticPtrs {
+  float* h;
+  uint16_t* x;
+  float* qkv;
+  uint16_t* qs;
+  float* part;
+  uint16_t* o;
+  float* x2f;
+  uint16_t* x2h;
+  float* logits;
+  uint16_t* u;
+  float* y;
+  uint32_t* ctrl;
+};
+
+/* copy the handle's parameter block into the array, point its working
+ * buffers at the array and zero the control words (one CTA) */
+__global__ void msk_static_params(const MskParams* src, MskParams* dst, StaticPtrs p) {
+  const unsigned long long* s = (const unsigned long long*)src;
+  unsigned long long* t = (unsigned long long*)dst;
+  for (size_t i = threadIdx.x; i < sizeof(MskParams) / 8; i += blockDim.x) t[i] = s[i];
+  for (int i = threadIdx.x; i < CTRL_WORDS; i += blockDim.x) p.ctrl[i] = 0u;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    dst->h = p.h;
+    dst->x = p.x;
+    dst->qkv = p.qkv;
+    dst->qs = p.qs;
+    dst->part = p.part;
+    dst->o = p.o;
+    dst->x2f = p.x2f;
+    dst->x2h = p.x2h;
+    dst->logits = p.logits;
+    dst->u = p.u;
+    dst->y = p.y;
+    dst->ctrl = p.ctrl;
+  }
 }
 
 extern "C" {
@@ -502,6 +591,67 @@ msk_status_t msk_query(msk_handle_t* h, msk_stats_t* out) {
   out->weight_bytes = wbytes;
   out->kv_bytes = kvbytes;
   out->algorithmic_bytes = wbytes + kvbytes + (int64_t)T * d * 2 * 2;
+  return MSK_OK;
+}
+
+msk_status_t msk_step_static(msk_handle_t* h, const uint16_t* hidden_in, const int32_t* positions, int n_seqs,
+                             int tokens_per_seq, msk_kv_t* kv, uint16_t* hidden_out, void* stream) {
+  if (!h || !hidden_in || !positions || !kv || !hidden_out || kv->h != h) return MSK_ERR_INVALID_ARG;
+  if (n_seqs < 1 || tokens_per_seq < 1 || n_seqs > h->cfg.max_seqs || tokens_per_seq > h->cfg.max_tokens_per_seq ||
+      n_seqs > kv->n_seqs)
+    return MSK_ERR_INVALID_ARG;
+  if (!aligned16(hidden_in) || !aligned16(hidden_out) || ((uintptr_t)positions & 3u)) return MSK_ERR_INVALID_ARG;
+  /* the handle's shapes must fit the array: refused before any device work */
+  const StaticLayout Lo = static_layout(h);
+  if (Lo.total > (size_t)MSK_STATIC_SCRATCH_BYTES) return MSK_ERR_UNSUPPORTED;
+  if (h->device < 0 || h->device >= MSK_STATIC_MAX_DEVICES) return MSK_ERR_UNSUPPORTED;
+  int prev = 0;
+  cudaGetDevice(&prev);
+  if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) return MSK_ERR_CUDA;
+  /* first call on this device, with the device current: look up the
+   * array's device address once */
+  StaticSlot& slot = g_static_slots[h->device];
+  std::call_once(slot.once, [&slot]() {
+    slot.ptr = nullptr;
+    slot.err = cudaGetSymbolAddress((void**)&slot.ptr, g_static_scratch);
+  });
+  cudaError_t e = (slot.err == cudaSuccess && slot.ptr) ? cudaSuccess : cudaErrorInvalidSymbol;
+  if (e == cudaSuccess) {
+    uint8_t* b = slot.ptr;
+    StaticPtrs p;
+    p.h = (float*)(b + Lo.h);
+    p.x = (uint16_t*)(b + Lo.x);
+    p.qkv = (float*)(b + Lo.qkv);
+    p.qs = (uint16_t*)(b + Lo.qs);
+    p.part = (float*)(b + Lo.part);
+    p.o = (uint16_t*)(b + Lo.o);
+    p.x2f = (float*)(b + Lo.x2f);
+    p.x2h = (uint16_t*)(b + Lo.x2h);
+    p.logits = (float*)(b + Lo.logits);
+    p.u = (uint16_t*)(b + Lo.u);
+    p.y = (float*)(b + Lo.y);
+    p.ctrl = (uint32_t*)(b + Lo.ctrl);
+    MskParams* Pd = (MskParams*)(b + Lo.params);
+    msk_static_params<<<1, 256, 0, (cudaStream_t)stream>>>(h->dev, Pd, p);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) {
+      MskStep st;
+      st.hidden_in = hidden_in;
+      st.positions = positions;
+      st.hidden_out = hidden_out;
+      st.kv_base = kv->base;
+      st.kv_cap = kv->cap;
+      st.kv_half_rows = kv->half_rows;
+      st.kv_seqs = kv->n_seqs;
+      st.S = n_seqs;
+      st.Tq = tokens_per_seq;
+      st.T = n_seqs * tokens_per_seq;
+      e = msk_kernel_launch(h->host.hd, Pd, &st, &kv->map, h->ncta, (cudaStream_t)stream);
+    }
+  }
+  if (prev != h->device) cudaSetDevice(prev);
+  if (e != cudaSuccess) return MSK_ERR_CUDA;
+  h->have_last = 1;
   return MSK_OK;
 }
 
