@@ -324,18 +324,21 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       for (int m = 0; m < 3 && ok; ++m) {
         const int64_t K = m < 2 ? P.d : P.f, rows = (int64_t)P.E * (m < 2 ? P.f : P.d);
         const int KC = K <= 512 ? (int)K : 512;
+        /* K not a multiple of 256 (128, 384): whole rows go as bulk copies
+         * and the maps stay zero */
+        if (K % 256) continue;
         for (int part = 0; part < 2 && ok; ++part) {
-          /* whole-row chunks use plain bulk copies; the map is left zero */
-          if (KC == K) continue;
-          const int64_t width = part == 0 ? K / 2 : K / 16;
-          cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-          cuuint64_t strides[1] = {(cuuint64_t)width};
-          cuuint32_t box[2] = {(cuuint32_t)(part == 0 ? KC / 2 : KC / 16), 16};
+          /* codes as 16-bit pairs [rows][K/4], a 128-row box 32 bytes wider
+           * than the K chunk; scales [rows][K/16], a 128-row box of the chunk */
+          const bool codes = part == 0;
+          cuuint64_t dims[2] = {(cuuint64_t)(codes ? K / 4 : K / 16), (cuuint64_t)rows};
+          cuuint64_t strides[1] = {(cuuint64_t)(codes ? K / 2 : K / 16)};
+          cuuint32_t box[2] = {(cuuint32_t)(codes ? KC / 4 + 16 : KC / 16), 128};
           cuuint32_t estr[2] = {1, 1};
-          void* base = (void*)(part == 0 ? mats[m]->codes : mats[m]->scales);
-          ok = enc(&hm[l * 6 + m * 2 + part], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+          void* base = (void*)(codes ? mats[m]->codes : mats[m]->scales);
+          ok = enc(&hm[l * 6 + m * 2 + part], codes ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                   base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
         }
       }
       P.layers[l].emap = h->emaps + l * 6;

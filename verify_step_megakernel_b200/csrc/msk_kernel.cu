@@ -61,18 +61,23 @@ struct Route {
   int16_t unit_n[MSK_MAX_UNITS];
 };
 
-constexpr int WKC_MAX = 512;                              /* K chunk of a per-warp expert tile */
-constexpr int NWS = 2;                                    /* per-warp expert ring depth */
-constexpr int WSLOT = 2 * 16 * (WKC_MAX / 2 + WKC_MAX / 16); /* gate+up 16-row chunk: 9216 B */
-static_assert(MSK_NCW * NWS * WSLOT <= MSK_NST * MSK_STAGE, "per-warp expert rings live in the stage ring");
+/* expert phases: a work item is 128 rows (16 per consumer warp) of the
+ * selected expert matrices for one unit of <= 8 tokens; K streams in chunks
+ * of <= 512 through a ring of slots (in the stage ring's memory) that the
+ * producer thread fills */
+constexpr int XROWS = 16 * MSK_NCW;
+constexpr int XKC_MAX = 512;
+constexpr int XNS_MAX = 4;
 
 struct Smem {
   uint64_t full[MSK_NST];
   uint64_t empty[MSK_NST];
-  uint64_t wfull[MSK_NCW][NWS]; /* per consumer warp: expert chunk landed */
+  uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
+  uint64_t xempty[XNS_MAX]; /* expert slot read by all consumer warps */
   volatile int kv_ready;    /* layer+1 whose KV writes all CTAs finished */
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
+  volatile int dn_ready;    /* layer+1 whose gate/up outputs all CTAs finished */
   volatile int abort;
   int pos0[MSK_MAX_TOKENS];
   float lbuf[4][32][2];
@@ -214,6 +219,43 @@ MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
   *b = (int)((int64_t)n * (cta + 1) / ncta);
 }
 
+/* Slot layout of an expert chunk, the same for the producer and consumers.
+ * Per matrix: codes [128][cpitch] then scales [128][spitch]; then the
+ * unit's activation rows [8][bpitch] (f16).  Where K is a multiple of 256
+ * the codes come as one 2-D tensor box 32 bytes wider than the chunk (the
+ * next chunk's first bytes, or zero fill past the row), so that rows sit 32
+ * bytes off the 128-byte bank period; with the lanes' interleaved block
+ * order below, the warp's shared loads are then free of bank conflicts.
+ * Other K (128, 384) take whole rows as single bulk copies. */
+struct XGeo {
+  int K, KC, nkc, rows_unit, ngroups, NM, tma, ns;
+  uint32_t cpitch, spitch, bpitch, mat_bytes, b_off, slot_bytes;
+  int a, b; /* this CTA's items [a, b) */
+};
+
+MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
+  const MskParams* P = c.P;
+  x.K = gu ? P->d : P->f;
+  x.rows_unit = gu ? P->f : P->d;
+  x.KC = x.K <= XKC_MAX ? x.K : XKC_MAX;
+  x.nkc = x.K / x.KC;
+  x.tma = (x.K % 256) == 0;
+  x.cpitch = (uint32_t)(x.tma ? x.KC / 2 + 32 : x.KC / 2);
+  x.spitch = (uint32_t)(x.KC / 16);
+  x.bpitch = (uint32_t)(2 * x.KC + 16);
+  x.NM = gu ? 2 : 1;
+  x.mat_bytes = XROWS * (x.cpitch + x.spitch);
+  x.b_off = x.NM * x.mat_bytes;
+  x.slot_bytes = (x.b_off + MSK_UNIT_TOK * x.bpitch + 127) & ~127u;
+  x.ns = min(XNS_MAX, (int)((uint32_t)(MSK_NST * MSK_STAGE) / x.slot_bytes));
+  x.ngroups = x.rows_unit / XROWS;
+  item_range(c.S->route.n_units * x.ngroups, c.cta, c.ncta, &x.a, &x.b);
+}
+/* gate+up with K = 512 is the largest slot: two must fit the ring */
+static_assert(2 * ((2 * XROWS * (XKC_MAX / 2 + 32 + XKC_MAX / 16) + MSK_UNIT_TOK * (2 * XKC_MAX + 16) + 127) & ~127) <=
+                  MSK_NST * MSK_STAGE,
+              "two expert slots fit the stage ring");
+
 /* attention key space of one layer: pairs (seq, kv head) in order, each
  * with the union of its rows' key ranges; CTA c owns [c N / n, (c+1) N / n) */
 struct AttGeo {
@@ -269,6 +311,8 @@ struct Prod {
   Ctx* c;
   uint32_t it;
   uint32_t last_parity_for_slot[MSK_NST];
+  uint32_t xpar;  /* bit s: parity of the fills of expert slot s so far */
+  uint32_t xused; /* bit s: expert slot s filled at least once */
   bool ok;
 };
 
@@ -310,11 +354,65 @@ MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, in
   return true;
 }
 
+/* Fill the expert ring for one phase: for each of this CTA's items and
+ * each K chunk, the 128-row tiles of the unit's expert (gate and up, or
+ * down) and the unit's activation rows, all on the slot's full barrier. */
+MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
+  Ctx& c = *p.c;
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const Route& R = c.S->route;
+  const int phase = gu ? PH_GU : PH_DN;
+  XGeo x;
+  xgeo(c, gu, x);
+  const MskNv* mat[2] = {gu ? &Ly.wg : &Ly.wd, &Ly.wu};
+  const CUtensorMap* cmap[2] = {Ly.emap + (gu ? 0 : 4), Ly.emap + 2};
+  const CUtensorMap* smap[2] = {Ly.emap + (gu ? 1 : 5), Ly.emap + 3};
+  const uint16_t* act = gu ? P->x2h : P->u;
+  const int act_ld = gu ? P->d : P->f;
+  const uint32_t brow = (uint32_t)(2 * x.KC);
+  int j = 0;
+  for (int item = x.a; item < x.b; ++item) {
+    const int unit = item / x.ngroups, grp = item % x.ngroups;
+    const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+    const int64_t grow = (int64_t)R.unit_e[unit] * x.rows_unit + (int64_t)grp * XROWS;
+    for (int kc = 0; kc < x.nkc; ++kc, ++j) {
+      const int s = j % x.ns;
+      if ((p.xused >> s) & 1u) {
+        if (!wait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, phase)) return false;
+      }
+      p.xpar ^= 1u << s;
+      p.xused |= 1u << s;
+      uint8_t* dst = c.ring + (size_t)s * x.slot_bytes;
+      uint64_t* bar = &c.S->xfull[s];
+      mbar_arrive_tx(bar, x.b_off + (uint32_t)n * brow);
+      for (int m = 0; m < x.NM; ++m) {
+        uint8_t* md = dst + (size_t)m * x.mat_bytes;
+        if (x.tma) {
+          tma_2d_g2s(md, cmap[m], kc * (x.KC / 4), (int32_t)grow, bar);
+          tma_2d_g2s(md + XROWS * x.cpitch, smap[m], kc * (x.KC / 16), (int32_t)grow, bar);
+        } else {
+          bulk_g2s(md, mat[m]->codes + grow * (x.K / 2), XROWS * x.cpitch, bar);
+          bulk_g2s(md + XROWS * x.cpitch, mat[m]->scales + grow * (x.K / 16), XROWS * x.spitch, bar);
+        }
+      }
+      for (int t = 0; t < n; ++t) {
+        const int pair = R.pairs[st0 + t];
+        const int row = gu ? pair / P->k : pair;
+        bulk_g2s(dst + x.b_off + t * x.bpitch, act + (size_t)row * act_ld + (size_t)kc * x.KC, brow, bar);
+      }
+    }
+  }
+  return true;
+}
+
 MSK_DEV void producer(Ctx& c) {
   const MskParams* P = c.P;
   Prod p;
   p.c = &c;
   p.it = 0;
+  p.xpar = 0;
+  p.xused = 0;
   p.ok = true;
   const int hd = P->hd;
   const int C = att_keys_per_stage(hd);
@@ -348,9 +446,9 @@ MSK_DEV void producer(Ctx& c) {
     int nwo = (P->d + rows_per_stage(P->qd) - 1) / rows_per_stage(P->qd);
     for (int j = c.cta; j < nwo && p.ok; j += c.ncta) p.ok = prod_weights(p, wo_stage(P, Ly, j), l, PH_WO);
     if (!p.ok) break;
-    /* the consumer warps stream the selected experts through their own
-     * slices of the ring; meanwhile pull this CTA's next-layer dense tiles
-     * into L2 */
+    /* pull this CTA's next-layer dense tiles into L2, then feed the expert
+     * phases once this layer's routing (and later its gate/up outputs) is
+     * known */
     if (l + 1 < P->L) {
       const MskLayer& Ln = P->layers[l + 1];
       for (int j = c.cta; j < nq; j += c.ncta) {
@@ -364,10 +462,24 @@ MSK_DEV void producer(Ctx& c) {
         prefetch_l2(ws.scales, (uint32_t)ws.nrows * (ws.K / 16));
       }
     }
+    if (!wait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { p.ok = false; break; }
+    fence_proxy_async_global();
+    if (!prod_experts(p, l, true)) { p.ok = false; break; }
+    if (!wait_flag(c, &c.S->dn_ready, l + 1, l, PH_DN)) { p.ok = false; break; }
+    fence_proxy_async_global();
+    if (!prod_experts(p, l, false)) { p.ok = false; break; }
     if (!wait_flag(c, &c.S->ring_free, l + 1, l, PH_DN)) { p.ok = false; break; }
   }
   if (!p.ok) {
     /* let every copy already issued land before the CTA may exit */
+    for (int sl = 0; sl < XNS_MAX; ++sl) {
+      if (!((p.xused >> sl) & 1u)) continue;
+      const uint32_t par = ((p.xpar >> sl) & 1u) ^ 1u; /* the slot's latest fill */
+      uint64_t t0 = gtimer();
+      while (!mbar_try(&c.S->xfull[sl], par)) {
+        if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+      }
+    }
     uint32_t n = p.it < MSK_NST ? p.it : MSK_NST;
     for (uint32_t i = p.it - n; i < p.it; ++i) {
       uint32_t slot = i % MSK_NST;
@@ -1184,266 +1296,107 @@ MSK_DEV void phase_comb(const Ctx& c, int layer) {
   }
 }
 
-/* ---- consumer: expert tiles, one pipeline per warp ---------------------------------- */
-MSK_DEV int expert_kc(int K) { return K <= WKC_MAX ? K : WKC_MAX; } /* K <= 512 or a multiple of 512 */
-
-/* Copies rows [grow, grow+16) x K-chunk kc of an NVFP4 matrix into dst laid
- * out codes[16][KC/2] then scales[16][KC/16]: whole rows are one contiguous
- * bulk copy each; chunks of longer rows are one 2-D tensor box each (maps
- * cmap/smap over codes [rows][K/2] and scales [rows][K/16]). */
-MSK_DEV void warp_copy_rows(uint8_t* dst, const uint8_t* codes, const uint8_t* scales, const CUtensorMap* cmap,
-                            const CUtensorMap* smap, int64_t grow, int K, int kc, int KC, uint64_t* bar) {
-  const int lane = threadIdx.x & 31;
-  const int cb = KC / 2, sb = KC / 16;
-  if (KC == K) {
-    if (lane == 0) bulk_g2s(dst, codes + grow * (K / 2), 16 * cb, bar);
-    else if (lane == 1) bulk_g2s(dst + 16 * cb, scales + grow * (K / 16), 16 * sb, bar);
-  } else {
-    if (lane == 0) tma_2d_g2s(dst, cmap, kc * cb, (int32_t)grow, bar);
-    else if (lane == 1) tma_2d_g2s(dst + 16 * cb, smap, kc * sb, (int32_t)grow, bar);
-  }
-}
-
+/* ---- consumer: expert tiles from the producer's ring --------------------------------- */
 /*
- * NM 16-row NVFP4 tiles (gate and up, or down alone; mstride bytes apart in
- * smem, each codes[16][K/2] + scales[16][K/16]) times one 8-column
- * activation tile.  bq holds this lane's activation fragments of the whole
- * chunk (block b: bq[2b], bq[2b+1]), loaded a chunk ahead by the caller.
- * Same k permutation as gemm_warp; each fragment feeds all NM matrices.
+ * One warp's 16 rows of NM NVFP4 matrices (gate and up, or down) times the
+ * unit's 8 activation columns over one K chunk, all operands in shared
+ * memory.  Lane (g, cq) owns the NVFP4 blocks 4 qb + cq of the chunk (16 k
+ * each, so one scale per block and lane): per block its 16 codes of rows g
+ * and g+8 (8 bytes each), the two scales, and 16 activations of column g.
+ * Each block is 4 m16n8k16 steps whose k slots map onto the block's 16 k in
+ * the same order on both operands.  Decoding is exact: e2m1 and e4m3 are
+ * exact in f16 and so is their product.
  */
-constexpr int EBLK = WKC_MAX / 16 / 4; /* blocks per lane per 512-wide chunk: 8 */
-constexpr int EPF = 1;                  /* activation prefetch distance in blocks */
-
-template <int NM, int BPT>
-MSK_DEV void gemm_rows16(const uint8_t* stg, int mstride, int K, uint4* bq, const uint16_t* cur_bp,
-                         const uint16_t* next_bp, float (*acc)[4], float (*acc2)[4]) {
+template <int NM>
+MSK_DEV void xgemm(uint32_t codes, uint32_t scales, uint32_t mstride, uint32_t cpitch, uint32_t spitch, uint32_t bsm,
+                   uint32_t bpitch, int KC, float (*acc)[4], float (*acc2)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
-  const int nwin = K / (64 * BPT);
-  const int nblk = K / 64;
-  const uint32_t sb0 = smem_u32(stg);
-#pragma unroll
-  for (int win = 0; win < WKC_MAX / (64 * BPT); ++win) {
-    if (win >= nwin) break;
-    const int kw = win * 64 * BPT;
-    const uint32_t coff = kw / 2 + cq * BPT * 8, soff = 16 * (K / 2) + kw / 16 + cq * BPT;
-    uint32_t sw0[NM], sw1[NM];
+  /* bytes [s(g), s(g), s(g+8), s(g+8)] of the two rows' scale words */
+  const uint32_t sel = (uint32_t)(cq | (cq << 4) | ((cq + 4) << 8) | ((cq + 4) << 12));
+  const uint32_t a0 = codes + g * cpitch + 8 * cq, a1 = a0 + 8 * cpitch;
+  const uint32_t s0 = scales + g * spitch, s1 = s0 + 8 * spitch;
+  const uint32_t b = bsm + g * bpitch + 32 * cq;
+  const int nq = KC / 64;
+#pragma unroll 2
+  for (int qb = 0; qb < nq; ++qb) {
+    const uint4 b0 = lds128(b + 128 * qb), b1 = lds128(b + 128 * qb + 16);
 #pragma unroll
     for (int m = 0; m < NM; ++m) {
-      const uint32_t mb = sb0 + m * mstride;
-      if (BPT == 4) {
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
-        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
-      } else if (BPT == 2) {
-        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
-        asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
-      } else {
-        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw0[m]) : "r"(mb + soff + g * (K / 16)));
-        asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw1[m]) : "r"(mb + soff + (g + 8) * (K / 16)));
-      }
-    }
+      const uint32_t mo = m * mstride;
+      const uint2 c0 = lds64(a0 + mo + 32 * qb), c1 = lds64(a1 + mo + 32 * qb);
+      const uint32_t w0 = lds32(s0 + mo + 4 * qb), w1 = lds32(s1 + mo + 4 * qb);
+      uint32_t sc[2];
+      e4m3x4_to_f16x2x2(__byte_perm(w0, w1, sel), sc);
+      uint32_t r0[8], r1[8];
+      e2m1x8_to_f16x2x4(c0.x, r0);
+      e2m1x8_to_f16x2x4(c0.y, r0 + 4);
+      e2m1x8_to_f16x2x4(c1.x, r1);
+      e2m1x8_to_f16x2x4(c1.y, r1 + 4);
 #pragma unroll
-    for (int qb = 0; qb < BPT; ++qb) {
-      const int blk = win * BPT + qb;
-      const int rs = blk % EPF; /* ring slot of this block's fragments */
-      const uint4 b0 = bq[2 * rs], b1 = bq[2 * rs + 1];
-      /* refill the slot with the fragments EPF blocks ahead (in this chunk
-       * or the next one): half a chunk of work hides their latency */
-      {
-        const int ab = blk + EPF;
-        const uint16_t* src = ab < nblk ? cur_bp : next_bp;
-        const int bb = ab < nblk ? ab : ab - nblk;
-        if (src) {
-          const int kb = (bb / BPT) * 64 * BPT + 16 * (cq * BPT + bb % BPT);
-          bq[2 * rs] = ldg128(src + kb);
-          bq[2 * rs + 1] = ldg128(src + kb + 8);
-        } else {
-          bq[2 * rs] = bq[2 * rs + 1] = make_uint4(0, 0, 0, 0);
-        }
-      }
-#pragma unroll
-      for (int m = 0; m < NM; ++m) {
-        const uint32_t mb = sb0 + m * mstride;
-        /* this block's 16 codes of rows g and g+8 (8 bytes each) */
-        const uint2 c0 = lds64(mb + g * (K / 2) + coff + qb * 8), c1 = lds64(mb + (g + 8) * (K / 2) + coff + qb * 8);
-        /* the block's scales of rows g and g+8, broadcast to f16x2 */
-        const uint32_t s01 = __byte_perm(sw0[m], sw1[m], (uint32_t)(qb | (qb << 4) | ((qb + 4) << 8) | ((qb + 4) << 12)));
-        uint32_t sc[2];
-        e4m3x4_to_f16x2x2(s01, sc);
-        uint32_t r0[8], r1[8];
-        e2m1x8_to_f16x2x4(c0.x, r0);
-        e2m1x8_to_f16x2x4(c0.y, r0 + 4);
-        e2m1x8_to_f16x2x4(c1.x, r1);
-        e2m1x8_to_f16x2x4(c1.y, r1 + 4);
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          uint32_t a[4];
-          a[0] = hmul2(r0[2 * s], sc[0]);
-          a[1] = hmul2(r1[2 * s], sc[1]);
-          a[2] = hmul2(r0[2 * s + 1], sc[0]);
-          a[3] = hmul2(r1[2 * s + 1], sc[1]);
-          const uint4& bb = (s >> 1) ? b1 : b0;
-          /* alternate two accumulators: two independent mma chains */
-          mma_f16((s & 1) ? acc2[m] : acc[m], a, (s & 1) ? bb.z : bb.x, (s & 1) ? bb.w : bb.y);
-        }
+      for (int st = 0; st < 4; ++st) {
+        uint32_t a[4];
+        a[0] = hmul2(r0[2 * st], sc[0]);
+        a[1] = hmul2(r1[2 * st], sc[1]);
+        a[2] = hmul2(r0[2 * st + 1], sc[0]);
+        a[3] = hmul2(r1[2 * st + 1], sc[1]);
+        const uint4& bb = (st >> 1) ? b1 : b0;
+        /* alternate two accumulators: two independent mma chains */
+        mma_f16((st & 1) ? acc2[m] : acc[m], a, (st & 1) ? bb.z : bb.x, (st & 1) ? bb.w : bb.y);
       }
     }
   }
 }
 
-/* this lane's activation fragments of the first EPF blocks of a chunk (K
- * chunk KC, BPT blocks per window) from row bp (null: zeros) */
-template <int BPT>
-MSK_DEV void load_bchunk(const uint16_t* bp, int KC, uint4* bq) {
-  const int cq = threadIdx.x & 3;
-  const int nblk = KC / 64;
-#pragma unroll
-  for (int bl = 0; bl < EPF; ++bl) {
-    if (bl < nblk && bp) {
-      const int kb = (bl / BPT) * 64 * BPT + 16 * (cq * BPT + bl % BPT);
-      bq[2 * bl] = ldg128(bp + kb);
-      bq[2 * bl + 1] = ldg128(bp + kb + 8);
-    } else {
-      bq[2 * bl] = bq[2 * bl + 1] = make_uint4(0, 0, 0, 0);
-    }
-  }
-}
-
-/* the expert tensors of one phase, read once from the parameter block */
-struct ExpMats {
-  const uint8_t* codes[2];
-  const uint8_t* scales[2];
-  const CUtensorMap* cmap[2];
-  const CUtensorMap* smap[2];
-  float gs[2];
-};
-
-/* issue chunk j of this warp's expert items into its ring slot */
+/* gate/up (GU) or down projection of the selected experts: this CTA's
+ * items, 16 rows per warp, chunks from the producer's ring.  xpar bit s is
+ * this warp's parity of the uses of slot s so far. */
 template <bool GU>
-MSK_DEV void expert_issue(const ExpMats& M, const Route& R, uint8_t* wbase, uint64_t* fb, uint32_t wit0, int j, int a,
-                          int cw, int nkc, int tiles, int rows_unit, int K, int KC, uint32_t bytes) {
-  const int lane = threadIdx.x & 31;
-  const int item = a + cw + (j / nkc) * NCW, kc = j % nkc;
-  const int unit = item / tiles, tile = item % tiles;
-  const int64_t grow = (int64_t)R.unit_e[unit] * rows_unit + tile * 16;
-  const uint32_t gi = wit0 + (uint32_t)j;
-  uint8_t* dst = wbase + (size_t)(gi % NWS) * WSLOT;
-  uint64_t* bar = &fb[gi % NWS];
-  if (lane == 0) mbar_arrive_tx(bar, bytes);
-  __syncwarp();
-  warp_copy_rows(dst, M.codes[0], M.scales[0], M.cmap[0], M.smap[0], grow, K, kc, KC, bar);
-  if (GU)
-    warp_copy_rows(dst + 16 * (KC / 2 + KC / 16), M.codes[1], M.scales[1], M.cmap[1], M.smap[1], grow, K, kc, KC, bar);
-}
-
-/* gate/up (GU) or down projection of the selected experts.  Items are
- * (expert unit, 16-row tile); a CTA owns a contiguous item range and its
- * warps take every 8th item, so the warps of a CTA share the unit's
- * activation rows in L1.  Each warp streams its items' K chunks through a
- * 2-slot ring of its own and keeps the whole reduction in registers. */
-template <bool GU, int BPT>
-MSK_DEV bool expert_items(Ctx& c, int layer, uint32_t& wit, int a, int b, int K, int KC, int tiles) {
+MSK_DEV bool expert_phase(Ctx& c, int layer, uint32_t& xpar) {
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
   const Route& R = c.S->route;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
   const int phase = GU ? PH_GU : PH_DN;
-  const int nkc = K / KC;
-  const int cb = KC / 2, sb = KC / 16;
-  const int mine = (b - a > cw) ? (b - a - cw + NCW - 1) / NCW : 0;
-  const int total = mine * nkc;
-  /* everything the loop needs from the parameter block, read once */
-  const int d = P->d, f = P->f, topk = P->k;
-  const int rows_unit = GU ? f : d;
-  const uint16_t* act = GU ? P->x2h : P->u;
-  const int act_ld = GU ? d : f;
+  XGeo x;
+  xgeo(c, GU, x);
+  const int d = P->d, f = P->f;
+  const float gs0 = GU ? Ly.wg.gs : Ly.wd.gs, gs1 = Ly.wu.gs;
   uint16_t* uout = P->u;
   float* yout = P->y;
-  ExpMats M;
-  M.codes[0] = GU ? Ly.wg.codes : Ly.wd.codes;
-  M.scales[0] = GU ? Ly.wg.scales : Ly.wd.scales;
-  M.codes[1] = Ly.wu.codes;
-  M.scales[1] = Ly.wu.scales;
-  M.cmap[0] = Ly.emap + (GU ? 0 : 4);
-  M.smap[0] = Ly.emap + (GU ? 1 : 5);
-  M.cmap[1] = Ly.emap + 2;
-  M.smap[1] = Ly.emap + 3;
-  M.gs[0] = GU ? Ly.wg.gs : Ly.wd.gs;
-  M.gs[1] = Ly.wu.gs;
-  uint8_t* wbase = c.ring + (size_t)cw * NWS * WSLOT;
-  uint64_t* fb = c.S->wfull[cw];
-  const uint32_t wit0 = wit;
-  const uint32_t bytes = (GU ? 2u : 1u) * 16u * (uint32_t)(cb + sb);
-  /* row of this lane's activation column for chunk j (null past the unit) */
-  auto act_row = [&](int jj) -> const uint16_t* {
-    const int item = a + cw + (jj / nkc) * NCW, kc = jj % nkc;
-    const int unit = item / tiles;
-    if (g >= R.unit_n[unit]) return nullptr;
-    const int pair = R.pairs[R.unit_start[unit] + g];
-    return act + (size_t)(GU ? pair / topk : pair) * act_ld + (size_t)kc * KC;
-  };
-  for (int j = 0; j < total && j < NWS; ++j)
-    expert_issue<GU>(M, R, wbase, fb, wit0, j, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
-  uint4 bq[2 * EPF];
-  if (total > 0) load_bchunk<BPT>(act_row(0), KC, bq);
+  const uint32_t ring = smem_u32(c.ring);
   float acc[2][4], acc2[2][4];
   int j = 0;
   bool ok = true;
-  for (; j < total; ++j) {
-    const uint32_t gi = wit0 + (uint32_t)j;
-    if (!wait_bar(c, &fb[gi % NWS], (gi / NWS) & 1, layer, phase)) { ok = false; break; }
-    const uint8_t* stg = wbase + (size_t)(gi % NWS) * WSLOT;
-    const int item = a + cw + (j / nkc) * NCW, kc = j % nkc;
-    if (kc == 0) {
+  for (int item = x.a; item < x.b && ok; ++item) {
+    const int unit = item / x.ngroups, grp = item % x.ngroups;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = acc2[0][e] = acc2[1][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = acc2[0][e] = acc2[1][e] = 0.f;
+    for (int kc = 0; kc < x.nkc; ++kc, ++j) {
+      const int s = j % x.ns;
+      if (!wait_bar(c, &c.S->xfull[s], (xpar >> s) & 1u, layer, phase)) { ok = false; break; }
+      xpar ^= 1u << s;
+      const uint32_t slot = ring + (uint32_t)s * x.slot_bytes;
+      xgemm<GU ? 2 : 1>(slot + cw * 16 * x.cpitch, slot + XROWS * x.cpitch + cw * 16 * x.spitch, x.mat_bytes,
+                        x.cpitch, x.spitch, slot + x.b_off, x.bpitch, x.KC, acc, acc2);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.S->xempty[s]);
     }
-    gemm_rows16<GU ? 2 : 1, BPT>(stg, 16 * (cb + sb), KC, bq, act_row(j), j + 1 < total ? act_row(j + 1) : nullptr, acc,
-                                 acc2);
-    __syncwarp();
-    if (j + NWS < total) expert_issue<GU>(M, R, wbase, fb, wit0, j + NWS, a, cw, nkc, tiles, rows_unit, K, KC, bytes);
-    if (kc == nkc - 1) {
-      const int unit = item / tiles, tile = item % tiles;
-      const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+    if (!ok) break;
+    const int n = R.unit_n[unit], st0 = R.unit_start[unit];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int col = 2 * cq + (e & 1), row = tile * 16 + g + 8 * (e >> 1);
-        if (col < n) {
-          const int pair = R.pairs[st0 + col];
-          if (GU) {
-            const float gv = (acc[0][e] + acc2[0][e]) * M.gs[0], uv = (acc[1][e] + acc2[1][e]) * M.gs[1];
-            uout[(size_t)pair * f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
-          } else {
-            yout[(size_t)pair * d + row] = (acc[0][e] + acc2[0][e]) * M.gs[0];
-          }
+    for (int e = 0; e < 4; ++e) {
+      const int col = 2 * cq + (e & 1), row = grp * XROWS + cw * 16 + g + 8 * (e >> 1);
+      if (col < n) {
+        const int pair = R.pairs[st0 + col];
+        if (GU) {
+          const float gv = (acc[0][e] + acc2[0][e]) * gs0, uv = (acc[1][e] + acc2[1][e]) * gs1;
+          uout[(size_t)pair * f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
+        } else {
+          yout[(size_t)pair * d + row] = (acc[0][e] + acc2[0][e]) * gs0;
         }
       }
     }
   }
-  if (!ok) { /* let the copies in flight land before anything reuses the slots */
-    for (int jj = j; jj < total && jj < j + NWS; ++jj) {
-      const uint32_t gi = wit0 + (uint32_t)jj;
-      uint64_t t0 = gtimer();
-      while (!mbar_try(&fb[gi % NWS], (gi / NWS) & 1))
-        if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
-    }
-  }
-  wit = wit0 + (uint32_t)total;
-  return ok;
-}
-
-template <bool GU>
-MSK_DEV bool expert_phase(Ctx& c, int layer, uint32_t& wit) {
-  const MskParams* P = c.P;
-  const Route& R = c.S->route;
-  const int K = GU ? P->d : P->f;
-  const int tiles = (GU ? P->f : P->d) / 16;
-  const int KC = expert_kc(K);
-  int a, b;
-  item_range(R.n_units * tiles, c.cta, c.ncta, &a, &b);
-  const int q = (KC / 64) % 4 == 0 ? 4 : ((KC / 64) % 2 == 0 ? 2 : 1);
-  bool ok = q == 4 ? expert_items<GU, 4>(c, layer, wit, a, b, K, KC, tiles)
-                   : (q == 2 ? expert_items<GU, 2>(c, layer, wit, a, b, K, KC, tiles)
-                             : expert_items<GU, 1>(c, layer, wit, a, b, K, KC, tiles));
   if (!ok) c.S->abort = 1;
   named_sync(BAR_CONS, NCT);
   return !c.S->abort;
@@ -1456,7 +1409,7 @@ MSK_DEV void consumer(Ctx& c) {
   Cons q;
   q.c = &c;
   q.it = 0;
-  uint32_t wit = 0; /* this warp's expert chunks so far (its barrier phases) */
+  uint32_t xpar = 0; /* this warp's expert-slot parities */
   phase_in(c);
   if (!grid_sync(c, 0, PH_IN)) return;
   for (int l = 0; l < P->L; ++l) {
@@ -1505,9 +1458,10 @@ MSK_DEV void consumer(Ctx& c) {
     phase_router(c, l);
     if (!grid_sync(c, l, PH_ROUTER)) return;
     phase_topk(c, l);
-    if (!expert_phase<true>(c, l, wit)) return;
+    if (!expert_phase<true>(c, l, xpar)) return;
     if (!grid_sync(c, l, PH_GU)) return;
-    if (!expert_phase<false>(c, l, wit)) return;
+    if (threadIdx.x == CONS0) c.S->dn_ready = l + 1;
+    if (!expert_phase<false>(c, l, xpar)) return;
     named_sync(BAR_CONS, NCT);
     if (threadIdx.x == CONS0) c.S->ring_free = l + 1;
     if (!grid_sync(c, l, PH_DN)) return;
@@ -1542,8 +1496,11 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     c.S->route_ready = 0;
     c.S->ring_free = 0;
     c.S->abort = 0;
-    for (int w = 0; w < MSK_NCW; ++w)
-      for (int i = 0; i < NWS; ++i) mbar_init(&c.S->wfull[w][i], 1);
+    c.S->dn_ready = 0;
+    for (int i = 0; i < XNS_MAX; ++i) {
+      mbar_init(&c.S->xfull[i], 1);
+      mbar_init(&c.S->xempty[i], NCW);
+    }
     mbar_fence_init();
   }
   /* positions: contiguous per sequence, inside the cache */
