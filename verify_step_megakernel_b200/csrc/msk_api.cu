@@ -27,7 +27,7 @@ struct msk_handle {
   MskParams host;   /* mirror of the device copy */
   MskParams* dev;   /* device copy */
   void* scratch;    /* one allocation for every scratch buffer */
-  CUtensorMap* emaps; /* [L][6] expert tensor maps (device) */
+  CUtensorMap* emaps; /* [L][MSK_NMAPS] weight tensor maps (device) */
   size_t scratch_bytes;
   uint32_t* words;  /* ctrl + status */
   msk_debug_t dbg;
@@ -61,6 +61,14 @@ static EncodeTiledFn encode_fn() {
 
 static bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+/* floats per token of the projections' split-K partials: K slices of 512
+ * (one slice for K <= 512) times the output rows, QKV or W_o */
+static size_t proj_floats(const MskParams& P) {
+  const size_t sq = P.d <= 512 ? 1 : P.d / 512, so = P.qd <= 512 ? 1 : P.qd / 512;
+  const size_t a = sq * (size_t)(P.qd + 2 * P.kvd), b = so * (size_t)P.d;
+  return a > b ? a : b;
+}
+
 static msk_status_t check_nv(const msk_nvfp4_t& w) {
   if (!w.codes || !w.scales || !aligned16(w.codes) || !aligned16(w.scales)) return MSK_ERR_INVALID_ARG;
   if (!(w.global_scale > 0.0f) || !isfinite(w.global_scale)) return MSK_ERR_INVALID_ARG;
@@ -72,8 +80,10 @@ static msk_status_t check_config(const msk_config_t* c) {
   if (c->head_dim != 64 && c->head_dim != 128) return MSK_ERR_UNSUPPORTED;
   if (c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads) return MSK_ERR_INVALID_ARG;
   const int qd = c->n_q_heads * c->head_dim;
-  if (c->d_model < 128 || c->d_model % 128 || c->d_model > 4096) return MSK_ERR_UNSUPPORTED;
-  if (qd % 128 || qd > 4096) return MSK_ERR_UNSUPPORTED;
+  /* the projections' K dimensions (d_model, qd) split into slices of 512
+   * (or one slice of 256 or 512) read as 2-D tensor boxes */
+  if (c->d_model < 256 || c->d_model % 256 || c->d_model > 4096) return MSK_ERR_UNSUPPORTED;
+  if (qd < 256 || qd % 256 || qd > 4096 || (qd > 512 && qd % 512)) return MSK_ERR_UNSUPPORTED;
   if (c->expert_dim < 128 || c->expert_dim % 128 || c->expert_dim > 4096) return MSK_ERR_UNSUPPORTED;
   /* expert tiles stream K in chunks of 512: longer rows must split evenly */
   if ((c->d_model > 512 && c->d_model % 512) || (c->expert_dim > 512 && c->expert_dim % 512))
@@ -117,7 +127,7 @@ struct StaticLayout {
 static StaticLayout static_layout(const msk_handle_t* h) {
   const MskParams& P = h->host;
   const msk_config_t& c = h->cfg;
-  const size_t T = (size_t)P.max_T, d = P.d, qd = P.qd, kvd = P.kvd;
+  const size_t T = (size_t)P.max_T, d = P.d, qd = P.qd;
   const size_t slots = (size_t)h->ncta + (size_t)c.max_seqs * P.hkv;
   StaticLayout L;
   size_t at = 0;
@@ -125,7 +135,7 @@ static StaticLayout static_layout(const msk_handle_t* h) {
   L.params = take(sizeof(MskParams));
   L.h = take(T * d * 4);
   L.x = take(T * d * 2);
-  L.qkv = take(T * (qd + 2 * kvd) * 4);
+  L.qkv = take(T * proj_floats(P) * 4);
   L.qs = take(T * qd * 2);
   L.part = take(slots * (size_t)P.part_stride * 4);
   L.o = take(T * qd * 2);
@@ -270,14 +280,14 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   if (st) { delete h; cudaSetDevice(prev); return st; }
 
   /* scratch */
-  const size_t T = (size_t)P.max_T, d = P.d, qd = P.qd, kvd = P.kvd;
+  const size_t T = (size_t)P.max_T, d = P.d, qd = P.qd;
   const size_t R_max = (size_t)c.max_tokens_per_seq * P.G;
   P.part_stride = (int32_t)(R_max * (P.hd + 4));
   const size_t slots = (size_t)h->ncta + (size_t)c.max_seqs * P.hkv;
   size_t sizes[] = {
       T * d * 4,                 /* h */
       T * d * 2,                 /* x */
-      T * (qd + 2 * kvd) * 4,    /* qkv */
+      T * proj_floats(P) * 4,    /* split-K partials of the projections */
       T * qd * 2,                /* qs */
       slots * P.part_stride * 4, /* part */
       T * qd * 2,                /* o */
@@ -316,8 +326,8 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   /* tensor maps of the expert tensors, for the K-chunked expert tiles */
   {
     EncodeTiledFn enc = encode_fn();
-    CUtensorMap* hm = (CUtensorMap*)calloc((size_t)P.L * 6, sizeof(CUtensorMap));
-    bool ok = enc != nullptr && hm != nullptr && cudaMalloc(&h->emaps, sizeof(CUtensorMap) * 6 * P.L) == cudaSuccess;
+    CUtensorMap* hm = (CUtensorMap*)calloc((size_t)P.L * MSK_NMAPS, sizeof(CUtensorMap));
+    bool ok = enc != nullptr && hm != nullptr && cudaMalloc(&h->emaps, sizeof(CUtensorMap) * MSK_NMAPS * P.L) == cudaSuccess;
     for (int l = 0; l < P.L && ok; ++l) {
       const msk_layer_weights_t& w = layers[l];
       const msk_nvfp4_t* mats[3] = {&w.w_gate, &w.w_up, &w.w_down};
@@ -336,14 +346,33 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
           cuuint32_t box[2] = {(cuuint32_t)(codes ? KC / 4 + 16 : KC / 16), 128};
           cuuint32_t estr[2] = {1, 1};
           void* base = (void*)(codes ? mats[m]->codes : mats[m]->scales);
-          ok = enc(&hm[l * 6 + m * 2 + part], codes ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+          ok = enc(&hm[l * MSK_NMAPS + m * 2 + part], codes ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                    base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
         }
       }
-      P.layers[l].emap = h->emaps + l * 6;
+      /* the dense projections: 16-row boxes of a K slice (512, or all of
+       * K <= 512), codes 32 bytes wider than the slice as for the experts */
+      const msk_nvfp4_t* dm[4] = {&w.wq, &w.wk, &w.wv, &w.wo};
+      for (int m = 0; m < 4 && ok; ++m) {
+        const int64_t K = m < 3 ? P.d : P.qd, rows = m == 0 ? P.qd : (m < 3 ? P.kvd : P.d);
+        const int KS = K <= 512 ? (int)K : 512;
+        for (int part = 0; part < 2 && ok; ++part) {
+          const bool codes = part == 0;
+          cuuint64_t dims[2] = {(cuuint64_t)(codes ? K / 4 : K / 16), (cuuint64_t)rows};
+          cuuint64_t strides[1] = {(cuuint64_t)(codes ? K / 2 : K / 16)};
+          cuuint32_t box[2] = {(cuuint32_t)(codes ? KS / 4 + 16 : KS / 16), 16};
+          cuuint32_t estr[2] = {1, 1};
+          void* base = (void*)(codes ? dm[m]->codes : dm[m]->scales);
+          ok = enc(&hm[l * MSK_NMAPS + MSK_MAP_DENSE + m * 2 + part],
+                   codes ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        }
+      }
+      P.layers[l].emap = h->emaps + l * MSK_NMAPS;
     }
-    if (ok) ok = cudaMemcpy(h->emaps, hm, sizeof(CUtensorMap) * 6 * P.L, cudaMemcpyHostToDevice) == cudaSuccess;
+    if (ok) ok = cudaMemcpy(h->emaps, hm, sizeof(CUtensorMap) * MSK_NMAPS * P.L, cudaMemcpyHostToDevice) == cudaSuccess;
     free(hm);
     if (!ok) {
       if (h->emaps) cudaFree(h->emaps);

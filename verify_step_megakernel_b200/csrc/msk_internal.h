@@ -22,6 +22,9 @@
 #define MSK_MAX_UNITS 512    /* expert units per layer (T*k <= 512) */
 #define MSK_MAX_PAIRS 64     /* (sequence, kv-head) attention pairs */
 
+#define MSK_MAP_DENSE 6
+#define MSK_NMAPS 14
+
 /* per-step control words (zeroed before every launch) */
 enum { CTRL_BARRIER = 0, CTRL_ABORT = 1, CTRL_WORDS = 32 };
 /* persistent status words (cleared by msk_step_status) */
@@ -41,8 +44,9 @@ typedef struct MskLayer {
   const float* g_moe;
   const float* router;
   MskNv wq, wk, wv, wo, wg, wu, wd;
-  /* 2-D tensor maps of the expert tensors for K-chunked tiles (device):
-   * gate codes, gate scales, up codes, up scales, down codes, down scales */
+  /* 2-D tensor maps of the weights (device), MSK_NMAPS of them: gate
+   * codes, gate scales, up codes, up scales, down codes, down scales, then
+   * (from MSK_MAP_DENSE) codes and scales of wq, wk, wv, wo */
   const CUtensorMap* emap;
   float bound_log2; /* M * log2(e), M = sqrt(hd) max|g_q| max|g_k| */
   int32_t sliding;
@@ -57,7 +61,7 @@ typedef struct MskParams {
   /* scratch (device) */
   float* h;         /* [T][d] residual */
   uint16_t* x;      /* [T][d] f16 attention-norm input of the projections */
-  float* qkv;       /* [T][qd + 2 kvd] raw projections */
+  float* qkv;       /* split-K partials of the projections: QKV [S][T][qd + 2 kvd], W_o [S][T][d] */
   uint16_t* qs;     /* [T][qd] f16 normalised queries */
   float* part;      /* [slots][R_max][hd + 4] attention partials */
   uint16_t* o;      /* [T][qd] f16 attention output */

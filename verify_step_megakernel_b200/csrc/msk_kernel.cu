@@ -72,12 +72,16 @@ constexpr int XNS_MAX = 4;
 struct Smem {
   uint64_t full[MSK_NST];
   uint64_t empty[MSK_NST];
+  uint64_t dfull[MSK_NCW][2];  /* dense weight slot of a warp landed */
+  uint64_t dempty[MSK_NCW][2]; /* dense weight slot read by its warp */
+  uint64_t bfull;              /* dense activation slice landed */
   uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
   uint64_t xempty[XNS_MAX]; /* expert slot read by all consumer warps */
   volatile int kv_ready;    /* layer+1 whose KV writes all CTAs finished */
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
   volatile int dn_ready;    /* layer+1 whose gate/up outputs all CTAs finished */
+  volatile int dense_done;  /* dense phases this CTA finished (2 per layer) */
   volatile int abort;
   int pos0[MSK_MAX_TOKENS];
   float lbuf[4][32][2];
@@ -158,62 +162,7 @@ MSK_DEV bool grid_sync(Ctx& c, int layer, int phase) {
   return s_ok != 0;
 }
 
-/* ---- schedule: which stages this CTA streams, in order ---------------------------- */
-MSK_DEV int rows_per_stage(int K) {
-  int m = MSK_STAGE / (16 * (K / 2 + K / 16));
-  return 16 * (m < 1 ? 1 : (m > 8 ? 8 : m));
-}
-
-struct WStage { /* a weight stage: nrows x K NVFP4 rows starting at row0 */
-  const uint8_t* codes;
-  const uint8_t* scales;
-  int nrows, K;
-  int mat;  /* QKV: 0 q, 1 k, 2 v; GU: 0 gate, 1 up */
-  int row0; /* row within the (expert's) matrix */
-  int unit; /* expert unit (GU / DN) */
-  float gs;
-};
-
-MSK_DEV int qkv_stages(const MskParams* P, int* sQ, int* sK) {
-  int r = rows_per_stage(P->d);
-  *sQ = (P->qd + r - 1) / r;
-  *sK = (P->kvd + r - 1) / r;
-  return *sQ + 2 * *sK;
-}
-
-MSK_DEV WStage qkv_stage(const MskParams* P, const MskLayer& Ly, int j, int sQ, int sK) {
-  int r = rows_per_stage(P->d);
-  WStage s;
-  const MskNv* nv;
-  int rows;
-  if (j < sQ) { s.mat = 0; nv = &Ly.wq; rows = P->qd; }
-  else if (j < sQ + sK) { s.mat = 1; nv = &Ly.wk; j -= sQ; rows = P->kvd; }
-  else { s.mat = 2; nv = &Ly.wv; j -= sQ + sK; rows = P->kvd; }
-  s.row0 = j * r;
-  s.nrows = min(r, rows - s.row0);
-  s.K = P->d;
-  s.codes = nv->codes + (int64_t)s.row0 * (P->d / 2);
-  s.scales = nv->scales + (int64_t)s.row0 * (P->d / 16);
-  s.gs = nv->gs;
-  s.unit = 0;
-  return s;
-}
-
-MSK_DEV WStage wo_stage(const MskParams* P, const MskLayer& Ly, int j) {
-  int r = rows_per_stage(P->qd);
-  WStage s;
-  s.mat = 0;
-  s.row0 = j * r;
-  s.nrows = min(r, P->d - s.row0);
-  s.K = P->qd;
-  s.codes = Ly.wo.codes + (int64_t)s.row0 * (P->qd / 2);
-  s.scales = Ly.wo.scales + (int64_t)s.row0 * (P->qd / 16);
-  s.gs = Ly.wo.gs;
-  s.unit = 0;
-  return s;
-}
-
-/* expert stages: items = unit x row block, contiguous ranges per CTA */
+/* ---- work split ------------------------------------------------------------------- */
 MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
   *a = (int)((int64_t)n * cta / ncta);
   *b = (int)((int64_t)n * (cta + 1) / ncta);
@@ -255,6 +204,46 @@ MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
 static_assert(2 * ((2 * XROWS * (XKC_MAX / 2 + 32 + XKC_MAX / 16) + MSK_UNIT_TOK * (2 * XKC_MAX + 16) + 127) & ~127) <=
                   MSK_NST * MSK_STAGE,
               "two expert slots fit the stage ring");
+
+/* Dense projections (QKV, W_o) with T <= 64 tokens: split-K over CTAs.  A
+ * unit is one 16-row m-tile of the output rows times one K slice of 512 (or
+ * all of K <= 512); units run slice-major and each CTA takes a contiguous
+ * range, so it holds one activation slice [T][slice] in shared memory while
+ * its warps stream weight m-tiles against it (unit i of the range goes to
+ * warp i mod 8, through that warp's 2-slot ring).  Each unit writes its
+ * fp32 partial; the next phase adds the slices in order. */
+constexpr int DKS_MAX = 512;
+constexpr int DNS = 2;
+constexpr uint32_t DB_BYTES = MSK_MAX_TOKENS * (2 * DKS_MAX + 16);   /* activation slice */
+constexpr uint32_t DSLOT = 16 * (DKS_MAX / 2 + 32 + DKS_MAX / 16); /* one weight m-tile */
+static_assert(DB_BYTES + MSK_NCW * DNS * DSLOT <= MSK_NST * MSK_STAGE, "dense buffers fit the stage ring");
+
+struct DGeo {
+  int K, rows, KS, S, MT, a, b;
+  uint32_t cpitch, spitch, bpitch;
+};
+
+MSK_DEV void dgeo(const Ctx& c, bool qkv, DGeo& g) {
+  const MskParams* P = c.P;
+  g.K = qkv ? P->d : P->qd;
+  g.rows = qkv ? P->qd + 2 * P->kvd : P->d;
+  g.KS = g.K <= DKS_MAX ? g.K : DKS_MAX;
+  g.S = g.K / g.KS;
+  g.MT = g.rows / 16;
+  g.cpitch = (uint32_t)(g.KS / 2 + 32);
+  g.spitch = (uint32_t)(g.KS / 16);
+  g.bpitch = (uint32_t)(2 * g.KS + 16);
+  item_range(g.S * g.MT, c.cta, c.ncta, &g.a, &g.b);
+}
+
+/* matrix of output row `row` (QKV rows are q, then k, then v): its map
+ * index, local row and global scale */
+MSK_DEV void dense_mat(const MskParams* P, const MskLayer& Ly, bool qkv, int row, int* map, int* lrow, float* gs) {
+  if (!qkv) { *map = MSK_MAP_DENSE + 6; *lrow = row; *gs = Ly.wo.gs; }
+  else if (row < P->qd) { *map = MSK_MAP_DENSE; *lrow = row; *gs = Ly.wq.gs; }
+  else if (row < P->qd + P->kvd) { *map = MSK_MAP_DENSE + 2; *lrow = row - P->qd; *gs = Ly.wk.gs; }
+  else { *map = MSK_MAP_DENSE + 4; *lrow = row - P->qd - P->kvd; *gs = Ly.wv.gs; }
+}
 
 /* attention key space of one layer: pairs (seq, kv head) in order, each
  * with the union of its rows' key ranges; CTA c owns [c N / n, (c+1) N / n) */
@@ -313,6 +302,8 @@ struct Prod {
   uint32_t last_parity_for_slot[MSK_NST];
   uint32_t xpar;  /* bit s: parity of the fills of expert slot s so far */
   uint32_t xused; /* bit s: expert slot s filled at least once */
+  uint32_t dpar;  /* bit 2w+s: parity of the fills of warp w's dense slot s */
+  uint32_t dused; /* bit 2w+s: that slot filled at least once */
   bool ok;
 };
 
@@ -327,14 +318,12 @@ MSK_DEV bool prod_acquire(Prod& p, int layer, int phase, uint8_t** stg, uint64_t
   return true;
 }
 
-MSK_DEV bool prod_weights(Prod& p, const WStage& s, int layer, int phase) {
-  uint8_t* stg;
-  uint64_t* bar;
-  if (!prod_acquire(p, layer, phase, &stg, &bar)) return false;
-  uint32_t cb = (uint32_t)s.nrows * (s.K / 2), sb = (uint32_t)s.nrows * (s.K / 16);
-  mbar_arrive_tx(bar, cb + sb);
-  bulk_g2s(stg, s.codes, cb, bar);
-  bulk_g2s(stg + cb, s.scales, sb, bar);
+/* wait until every stage issued so far has been released by the consumers */
+MSK_DEV bool prod_drain(Prod& p, int layer, int phase) {
+  Ctx& c = *p.c;
+  const uint32_t n = p.it < MSK_NST ? p.it : MSK_NST;
+  for (uint32_t i = p.it - n; i < p.it; ++i)
+    if (!wait_bar(c, &c.S->empty[i % MSK_NST], (i / MSK_NST) & 1, layer, phase)) return false;
   return true;
 }
 
@@ -352,6 +341,52 @@ MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, in
   }
   __threadfence_block();
   return true;
+}
+
+/* Feed the warps' dense weight rings for one projection: this CTA's units
+ * in order, unit i of the range into warp i mod 8's next slot. */
+MSK_DEV bool prod_dense(Prod& p, int layer, bool qkv) {
+  Ctx& c = *p.c;
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const int phase = qkv ? PH_QKV : PH_WO;
+  DGeo g;
+  dgeo(c, qkv, g);
+  const uint32_t bytes = 16 * (g.cpitch + g.spitch);
+  for (int i = g.a; i < g.b; ++i) {
+    const int w = (i - g.a) % NCW, sl = ((i - g.a) / NCW) % DNS, bit = w * DNS + sl;
+    if ((p.dused >> bit) & 1u) {
+      if (!wait_bar(c, &c.S->dempty[w][sl], ((p.dpar >> bit) & 1u) ^ 1u, layer, phase)) return false;
+    }
+    p.dpar ^= 1u << bit;
+    p.dused |= 1u << bit;
+    const int s = i / g.MT;
+    int map, lrow;
+    float gs;
+    dense_mat(P, Ly, qkv, (i % g.MT) * 16, &map, &lrow, &gs);
+    uint8_t* dst = c.ring + DB_BYTES + (size_t)bit * DSLOT;
+    uint64_t* bar = &c.S->dfull[w][sl];
+    mbar_arrive_tx(bar, bytes);
+    tma_2d_g2s(dst, Ly.emap + map, s * (g.KS / 4), lrow, bar);
+    tma_2d_g2s(dst + 16 * g.cpitch, Ly.emap + map + 1, s * (g.KS / 16), lrow, bar);
+  }
+  return true;
+}
+
+/* pull this CTA's weight tiles of a projection of `layer` into L2 */
+MSK_DEV void prefetch_dense(const Ctx& c, int layer, bool qkv) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  DGeo g;
+  dgeo(c, qkv, g);
+  for (int i = g.a; i < g.b; ++i) {
+    int map, lrow;
+    float gs;
+    dense_mat(P, Ly, qkv, (i % g.MT) * 16, &map, &lrow, &gs);
+    const int s = i / g.MT;
+    tma_prefetch_2d(Ly.emap + map, s * (g.KS / 4), lrow);
+    tma_prefetch_2d(Ly.emap + map + 1, s * (g.KS / 16), lrow);
+  }
 }
 
 /* Fill the expert ring for one phase: for each of this CTA's items and
@@ -413,16 +448,19 @@ MSK_DEV void producer(Ctx& c) {
   p.it = 0;
   p.xpar = 0;
   p.xused = 0;
+  p.dpar = 0;
+  p.dused = 0;
   p.ok = true;
   const int hd = P->hd;
   const int C = att_keys_per_stage(hd);
   for (int l = 0; l < P->L && p.ok; ++l) {
-    const MskLayer& Ly = P->layers[l];
-    /* QKV weights: round-robin stages */
-    int sQ, sK, nq = qkv_stages(P, &sQ, &sK);
-    for (int j = c.cta; j < nq && p.ok; j += c.ncta) p.ok = prod_weights(p, qkv_stage(P, Ly, j, sQ, sK), l, PH_QKV);
-    /* attention: past keys stream at once, chunks holding this step's keys
-     * wait until every CTA has written them */
+    /* QKV weight tiles; the ring memory is free once the previous layer's
+     * expert phases released it */
+    if (!prod_dense(p, l, true)) { p.ok = false; break; }
+    /* attention stages reuse the memory once this CTA's QKV units are done:
+     * past keys stream at once, chunks holding this step's keys wait until
+     * every CTA has written them */
+    if (!wait_flag(c, &c.S->dense_done, 2 * l + 1, l, PH_ATT)) { p.ok = false; break; }
     AttGeo g;
     att_geo(c, l, g);
     for_each_att_stage(c, g, [&](int pr, int slot, int64_t k0, int n, bool, bool) {
@@ -443,24 +481,14 @@ MSK_DEV void producer(Ctx& c) {
       return true;
     });
     if (!p.ok) break;
-    int nwo = (P->d + rows_per_stage(P->qd) - 1) / rows_per_stage(P->qd);
-    for (int j = c.cta; j < nwo && p.ok; j += c.ncta) p.ok = prod_weights(p, wo_stage(P, Ly, j), l, PH_WO);
-    if (!p.ok) break;
+    /* W_o tiles once every attention stage has been read */
+    if (!prod_drain(p, l, PH_WO) || !prod_dense(p, l, false)) { p.ok = false; break; }
     /* pull this CTA's next-layer dense tiles into L2, then feed the expert
      * phases once this layer's routing (and later its gate/up outputs) is
      * known */
     if (l + 1 < P->L) {
-      const MskLayer& Ln = P->layers[l + 1];
-      for (int j = c.cta; j < nq; j += c.ncta) {
-        WStage ws = qkv_stage(P, Ln, j, sQ, sK);
-        prefetch_l2(ws.codes, (uint32_t)ws.nrows * (ws.K / 2));
-        prefetch_l2(ws.scales, (uint32_t)ws.nrows * (ws.K / 16));
-      }
-      for (int j = c.cta; j < nwo; j += c.ncta) {
-        WStage ws = wo_stage(P, Ln, j);
-        prefetch_l2(ws.codes, (uint32_t)ws.nrows * (ws.K / 2));
-        prefetch_l2(ws.scales, (uint32_t)ws.nrows * (ws.K / 16));
-      }
+      prefetch_dense(c, l + 1, true);
+      prefetch_dense(c, l + 1, false);
     }
     if (!wait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { p.ok = false; break; }
     fence_proxy_async_global();
@@ -472,6 +500,14 @@ MSK_DEV void producer(Ctx& c) {
   }
   if (!p.ok) {
     /* let every copy already issued land before the CTA may exit */
+    for (int bit = 0; bit < NCW * DNS; ++bit) {
+      if (!((p.dused >> bit) & 1u)) continue;
+      const uint32_t par = ((p.dpar >> bit) & 1u) ^ 1u;
+      uint64_t t0 = gtimer();
+      while (!mbar_try(&c.S->dfull[bit / DNS][bit % DNS], par)) {
+        if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+      }
+    }
     for (int sl = 0; sl < XNS_MAX; ++sl) {
       if (!((p.xused >> sl) & 1u)) continue;
       const uint32_t par = ((p.xpar >> sl) & 1u) ^ 1u; /* the slot's latest fill */
@@ -511,163 +547,128 @@ MSK_DEV void cons_release(Cons& q, uint32_t slot) {
 }
 
 /* split of a weight stage over the consumer warps: mt m-tiles x ks K-slices */
-MSK_DEV void stage_split(int nrows, int K, int* mt, int* ks) {
-  int m = nrows / 16;
-  int mp = 1;
-  while (mp < m) mp <<= 1;
-  int k = NCW / mp;
-  if (k < 1) k = 1;
-  while (k > 1 && ((K / 64) % k) != 0) k >>= 1;
-  *mt = m;
-  *ks = k;
-}
-
+/* ---- consumer: dense projections ------------------------------------------------------ */
 /*
- * One weight stage (nrows x K NVFP4 in smem) times ncols activation columns.
- * Columns are rows of an f16 matrix: bcol(j) gives the row pointer of column j
- * (j < ncols).  K is split into windows of 64*BPT; inside a window lane
- * (g, c) owns NVFP4 blocks c*BPT .. c*BPT+BPT-1 of rows g and g+8, so its
- * A-fragment bytes are contiguous; the same k permutation is applied to the
- * B fragments, which leaves the dot products unchanged.
+ * One warp's 16-row m-tile (codes and scales in its ring slot) times up to
+ * NT 8-column tiles of the activation slice in shared memory, over one K
+ * slice.  Same lane layout as the expert tiles: lane (g, cq) owns the NVFP4
+ * blocks 4 qb + cq, decodes them once and feeds every column tile.
  */
-template <int NT, int BPT>
-MSK_DEV void gemm_warp(const uint8_t* stg, int nrows, int K, int ks, int mi, int ki, int ntl,
-                       const uint16_t* const* bp, float (*acc)[4]) {
+template <int NT>
+MSK_DEV void dgemm(uint32_t codes, uint32_t scales, uint32_t cpitch, uint32_t spitch, uint32_t bsm, uint32_t bpitch,
+                   int KS, int ntl, float (*acc)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
-  const int Kr = K / ks;
-  const int nwin = Kr / (64 * BPT);
-  const int r0 = mi * 16 + g;
-  const uint32_t sbase = smem_u32(stg);
-  const uint32_t cbase0 = sbase + r0 * (K / 2), cbase1 = cbase0 + 8 * (K / 2);
-  const uint32_t scb = sbase + nrows * (K / 2);
-  const uint32_t sbase0 = scb + r0 * (K / 16), sbase1 = sbase0 + 8 * (K / 16);
-  for (int win = 0; win < nwin; ++win) {
-    const int kw = ki * Kr + win * 64 * BPT;
-    const uint32_t coff = kw / 2 + cq * BPT * 8;
-    const uint32_t soff = kw / 16 + cq * BPT;
-    uint32_t w0[2 * BPT], w1[2 * BPT];
-    if (BPT == 4) {
-      uint4 a = lds128(cbase0 + coff), b = lds128(cbase0 + coff + 16);
-      uint4 d = lds128(cbase1 + coff), e = lds128(cbase1 + coff + 16);
-      w0[0] = a.x; w0[1] = a.y; w0[2] = a.z; w0[3] = a.w; w0[4 % (2 * BPT)] = b.x; w0[5 % (2 * BPT)] = b.y;
-      w0[6 % (2 * BPT)] = b.z; w0[7 % (2 * BPT)] = b.w;
-      w1[0] = d.x; w1[1] = d.y; w1[2] = d.z; w1[3] = d.w; w1[4 % (2 * BPT)] = e.x; w1[5 % (2 * BPT)] = e.y;
-      w1[6 % (2 * BPT)] = e.z; w1[7 % (2 * BPT)] = e.w;
-    } else if (BPT == 2) {
-      uint4 a = lds128(cbase0 + coff), d = lds128(cbase1 + coff);
-      w0[0] = a.x; w0[1] = a.y; w0[2 % (2 * BPT)] = a.z; w0[3 % (2 * BPT)] = a.w;
-      w1[0] = d.x; w1[1] = d.y; w1[2 % (2 * BPT)] = d.z; w1[3 % (2 * BPT)] = d.w;
-    } else {
-      uint2 a = lds64(cbase0 + coff), d = lds64(cbase1 + coff);
-      w0[0] = a.x; w0[1 % (2 * BPT)] = a.y;
-      w1[0] = d.x; w1[1 % (2 * BPT)] = d.y;
-    }
-    uint32_t sw0, sw1; /* BPT scale bytes of rows g and g+8 */
-    if (BPT == 4) {
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw0) : "r"(sbase0 + soff));
-      asm volatile("ld.shared.u32 %0, [%1];" : "=r"(sw1) : "r"(sbase1 + soff));
-    } else if (BPT == 2) {
-      asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw0) : "r"(sbase0 + soff));
-      asm volatile("ld.shared.u16 %0, [%1];" : "=r"(sw1) : "r"(sbase1 + soff));
-    } else {
-      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw0) : "r"(sbase0 + soff));
-      asm volatile("ld.shared.u8 %0, [%1];" : "=r"(sw1) : "r"(sbase1 + soff));
+  const uint32_t sel = (uint32_t)(cq | (cq << 4) | ((cq + 4) << 8) | ((cq + 4) << 12));
+  const uint32_t a0 = codes + g * cpitch + 8 * cq, a1 = a0 + 8 * cpitch;
+  const uint32_t s0 = scales + g * spitch, s1 = s0 + 8 * spitch;
+  const uint32_t b = bsm + g * bpitch + 32 * cq;
+  const int nq = KS / 64;
+  for (int qb = 0; qb < nq; ++qb) {
+    const uint2 c0 = lds64(a0 + 32 * qb), c1 = lds64(a1 + 32 * qb);
+    const uint32_t w0 = lds32(s0 + 4 * qb), w1 = lds32(s1 + 4 * qb);
+    uint32_t sc[2];
+    e4m3x4_to_f16x2x2(__byte_perm(w0, w1, sel), sc);
+    uint32_t r0[8], r1[8];
+    e2m1x8_to_f16x2x4(c0.x, r0);
+    e2m1x8_to_f16x2x4(c0.y, r0 + 4);
+    e2m1x8_to_f16x2x4(c1.x, r1);
+    e2m1x8_to_f16x2x4(c1.y, r1 + 4);
+    uint32_t a[4][4];
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+      a[st][0] = hmul2(r0[2 * st], sc[0]);
+      a[st][1] = hmul2(r1[2 * st], sc[1]);
+      a[st][2] = hmul2(r0[2 * st + 1], sc[0]);
+      a[st][3] = hmul2(r1[2 * st + 1], sc[1]);
     }
 #pragma unroll
-    for (int qb = 0; qb < BPT; ++qb) {
-      uint32_t sc[2];
-      e4m3x4_to_f16x2x2(__byte_perm(sw0, sw1, (uint32_t)(qb | (qb << 4) | ((qb + 4) << 8) | ((qb + 4) << 12))), sc);
-      const uint32_t sc0 = sc[0], sc1 = sc[1];
-      uint32_t r0[8], r1[8];
-      e2m1x8_to_f16x2x4(w0[2 * qb], r0);
-      e2m1x8_to_f16x2x4(w0[2 * qb + 1], r0 + 4);
-      e2m1x8_to_f16x2x4(w1[2 * qb], r1);
-      e2m1x8_to_f16x2x4(w1[2 * qb + 1], r1 + 4);
-      const int kb = kw + 16 * (cq * BPT + qb);
-      uint4 bl[NT][2];
-#pragma unroll
-      for (int j = 0; j < NT; ++j) {
-        if (j < ntl && bp[j]) {
-          bl[j][0] = ldg128(bp[j] + kb);
-          bl[j][1] = ldg128(bp[j] + kb + 8);
-        } else {
-          bl[j][0] = bl[j][1] = make_uint4(0, 0, 0, 0);
-        }
-      }
-#pragma unroll
-      for (int s = 0; s < 4; ++s) {
-        uint32_t a[4];
-        a[0] = hmul2(r0[2 * s], sc0);
-        a[1] = hmul2(r1[2 * s], sc1);
-        a[2] = hmul2(r0[2 * s + 1], sc0);
-        a[3] = hmul2(r1[2 * s + 1], sc1);
-#pragma unroll
-        for (int j = 0; j < NT; ++j) {
-          if (j < ntl) {
-            const uint4& lo = bl[j][s >> 1];
-            const uint32_t b0 = (s & 1) ? lo.z : lo.x, b1 = (s & 1) ? lo.w : lo.y;
-            mma_f16(acc[j], a, b0, b1);
-          }
-        }
+    for (int nt = 0; nt < NT; ++nt) {
+      if (nt < ntl) {
+        const uint32_t bt = b + nt * 8 * bpitch + 128 * qb;
+        const uint4 b0 = lds128(bt), b1 = lds128(bt + 16);
+        mma_f16(acc[nt], a[0], b0.x, b0.y);
+        mma_f16(acc[nt], a[1], b0.z, b0.w);
+        mma_f16(acc[nt], a[2], b1.x, b1.y);
+        mma_f16(acc[nt], a[3], b1.z, b1.w);
       }
     }
   }
 }
 
-template <int NT, class BCol, class Epi>
-MSK_DEV bool gemm_stage(Cons& q, const WStage& ws, int ncols, BCol bcol, Epi epi, int layer, int phase) {
-  Ctx& c = *q.c;
-  uint32_t slot;
-  /* on a failed wait the warp skips the math but keeps the barrier sequence,
-   * so no sibling is left waiting in a named barrier */
-  const uint8_t* stg = cons_wait(q, layer, phase, &slot);
-  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2;
-  const int K = ws.K, nrows = ws.nrows;
-  int mt, ks;
-  stage_split(nrows, K, &mt, &ks);
-  const int ntl = (ncols + 7) >> 3;
-  float acc[NT][4];
-#pragma unroll
-  for (int j = 0; j < NT; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-  const bool active = cw < mt * ks && stg != nullptr;
-  if (active) {
-    const int mi = cw / ks, ki = cw % ks;
-    const int Kr = K / ks;
-    const uint16_t* bp[NT];
-#pragma unroll
-    for (int j = 0; j < NT; ++j) {
-      const int col = j * 8 + g;
-      bp[j] = (j < ntl && col < ncols) ? bcol(col) : nullptr;
-    }
-    if ((Kr / 64) % 4 == 0) gemm_warp<NT, 4>(stg, nrows, K, ks, mi, ki, ntl, bp, acc);
-    else if ((Kr / 64) % 2 == 0) gemm_warp<NT, 2>(stg, nrows, K, ks, mi, ki, ntl, bp, acc);
-    else gemm_warp<NT, 1>(stg, nrows, K, ks, mi, ki, ntl, bp, acc);
-  }
-  if (stg) cons_release(q, slot);
-  /* split-K reduction in fixed order, then the epilogue */
-  float* red = c.scr;
-  if (active) {
-#pragma unroll
-    for (int j = 0; j < NT; ++j)
-      if (j < ntl)
-        *reinterpret_cast<float4*>(&red[((cw * NT + j) * 32 + lane) * 4]) =
-            make_float4(acc[j][0], acc[j][1], acc[j][2], acc[j][3]);
-  }
-  named_sync(BAR_CONS, NCT);
+/* QKV or W_o for this step's T tokens: this CTA's units, slice by slice.
+ * dpar bits 0-1: this warp's parities of its two weight slots; bit 8: the
+ * activation slice barrier's parity.  Every warp takes part in every slice
+ * (the CTA-wide barriers keep one sequence even after a failed wait). */
+template <bool QKV>
+MSK_DEV bool dense_phase(Ctx& c, int layer, uint32_t& dpar) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
   const int ctid = threadIdx.x - CONS0;
-  for (int idx = ctid; idx < mt * ntl * 32; idx += NCT) {
-    int mi = idx / (ntl * 32), j = (idx / 32) % ntl, ln = idx & 31;
-    float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int ki = 0; ki < ks; ++ki) {
-      float4 v = *reinterpret_cast<const float4*>(&red[(((mi * ks + ki) * NT + j) * 32 + ln) * 4]);
-      s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+  const int phase = QKV ? PH_QKV : PH_WO;
+  DGeo G;
+  dgeo(c, QKV, G);
+  const int T = c.st.T, ntl = (T + 7) >> 3;
+  const uint16_t* act = QKV ? P->x : P->o;
+  float* out = P->qkv;
+  const uint32_t ring = smem_u32(c.ring);
+  bool ok = true;
+  for (int i0 = G.a; i0 < G.b;) {
+    const int s = i0 / G.MT;
+    const int i1 = min(G.b, (s + 1) * G.MT);
+    /* the activation slice: the byte count is posted first, the copies go
+     * out once every warp is done with the region */
+    const uint32_t bpar = (dpar >> 8) & 1u;
+    dpar ^= 1u << 8;
+    if (ok && ctid == 0) mbar_arrive_tx(&c.S->bfull, (uint32_t)(T * 2 * G.KS));
+    named_sync(BAR_CONS, NCT);
+    const bool issued = ok && ctid < T;
+    if (issued) {
+      fence_proxy_async_global();
+      bulk_g2s(c.ring + (size_t)ctid * G.bpitch, act + (size_t)ctid * G.K + (size_t)s * G.KS, (uint32_t)(2 * G.KS),
+               &c.S->bfull);
     }
-    int row = mi * 16 + (ln >> 2), col = j * 8 + 2 * (ln & 3);
-    if (col < ncols) { epi(row, col, s.x * ws.gs); epi(row + 8, col, s.z * ws.gs); }
-    if (col + 1 < ncols) { epi(row, col + 1, s.y * ws.gs); epi(row + 8, col + 1, s.w * ws.gs); }
+    if (ok && !wait_bar(c, &c.S->bfull, bpar, layer, phase)) ok = false;
+    if (!ok && issued) { /* this thread's copy must land before the CTA may exit */
+      const uint64_t t0 = gtimer();
+      while (!mbar_try(&c.S->bfull, bpar) && gtimer() - t0 < 2 * (uint64_t)P->timeout_ns) {
+      }
+    }
+    const int first = i0 + ((cw - (i0 - G.a)) % NCW + NCW) % NCW;
+    for (int i = first; ok && i < i1; i += NCW) {
+      const int sl = ((i - G.a) / NCW) % DNS;
+      if (!wait_bar(c, &c.S->dfull[cw][sl], (dpar >> sl) & 1u, layer, phase)) { ok = false; break; }
+      dpar ^= 1u << sl;
+      float acc[MSK_NT_DENSE][4];
+#pragma unroll
+      for (int nt = 0; nt < MSK_NT_DENSE; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
+      const uint32_t slot = ring + DB_BYTES + (uint32_t)(cw * DNS + sl) * DSLOT;
+      dgemm<MSK_NT_DENSE>(slot, slot + 16 * G.cpitch, G.cpitch, G.spitch, ring, G.bpitch, G.KS, ntl, acc);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.S->dempty[cw][sl]);
+      int map, lrow;
+      float gs;
+      const int row0 = (i % G.MT) * 16;
+      dense_mat(P, Ly, QKV, row0, &map, &lrow, &gs);
+      float* dst = out + (size_t)s * T * G.rows;
+#pragma unroll
+      for (int nt = 0; nt < MSK_NT_DENSE; ++nt) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = nt * 8 + 2 * cq + (e & 1), row = row0 + g + 8 * (e >> 1);
+          if (nt < ntl && col < T) dst[(size_t)col * G.rows + row] = acc[nt][e] * gs;
+        }
+      }
+    }
+    i0 = i1;
   }
+  if (!ok) c.S->abort = 1;
   named_sync(BAR_CONS, NCT);
-  return !c.S->abort; /* read after the barrier: the same answer in every warp */
+  if (ctid == 0) {
+    __threadfence_block();
+    c.S->dense_done = 2 * layer + (QKV ? 1 : 2);
+  }
+  return !c.S->abort;
 }
 
 /* ---- consumer: attention stages ------------------------------------------------------ */
@@ -1021,9 +1022,13 @@ MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
   const int per = hd / 32; /* 4 or 2 values per lane */
   for (int item = gwarp(c); item < c.st.T * nh; item += nwarps(c)) {
     const int t = item / nh, hh = item % nh;
-    const float* raw = P->qkv + (size_t)t * nqkv + hh * hd + lane * per;
-    float v[4];
-    for (int i = 0; i < per; ++i) v[i] = raw[i];
+    /* the projection: its K slices' partials added in slice order */
+    const int S = P->d <= DKS_MAX ? 1 : P->d / DKS_MAX;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sl = 0; sl < S; ++sl) {
+      const float* raw = P->qkv + ((size_t)sl * c.st.T + t) * nqkv + hh * hd + lane * per;
+      for (int i = 0; i < per; ++i) v[i] += raw[i];
+    }
     const int b = t / c.st.Tq, ti = t % c.st.Tq;
     if (hh < P->hq + P->hkv) {
       float ss = 0.f;
@@ -1086,6 +1091,7 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
   const int d = P->d, sl = d / NCW, base = cw * sl + lane * 4;
+  const int So = P->qd <= DKS_MAX ? 1 : P->qd / DKS_MAX;
   for (int t = c.cta; t < c.st.T; t += c.ncta) {
     float4 v[ROWV];
     float ss = 0.f;
@@ -1094,7 +1100,14 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
       const int i = base + u * 128;
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (i < (cw + 1) * sl) {
-        v[u] = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
+        /* residual + W_o o, the projection's K slices added in order */
+        float4* hp = reinterpret_cast<float4*>(P->h + (size_t)t * d + i);
+        v[u] = *hp;
+        for (int s = 0; s < So; ++s) {
+          const float4 q = *reinterpret_cast<const float4*>(P->qkv + ((size_t)s * c.st.T + t) * d + i);
+          v[u].x += q.x; v[u].y += q.y; v[u].z += q.z; v[u].w += q.w;
+        }
+        *hp = v[u];
         ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
       }
     }
@@ -1152,7 +1165,10 @@ MSK_DEV void phase_topk(Ctx& c, int layer) {
   for (int t = cw; t < c.st.T; t += NCW) {
     float v[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) v[i] = i < per ? P->logits[(size_t)t * E + lane * per + i] : -INFINITY;
+    for (int i = 0; i < 8; ++i) {
+      const float x = i < per ? P->logits[(size_t)t * E + lane * per + i] : -INFINITY;
+      v[i] = x == x ? x : -INFINITY; /* a NaN logit ranks last */
+    }
     uint32_t taken = 0;
     float sel[8];
     float vmax = 0.f;
@@ -1161,7 +1177,12 @@ MSK_DEV void phase_topk(Ctx& c, int layer) {
       int bi = 0x7FFFFFFF;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        if (i < per && !(taken >> i & 1) && (v[i] > bv)) { bv = v[i]; bi = lane * per + i; }
+        /* ties (-inf included) go to the lower index, so every pick is a
+         * valid expert even when all remaining logits are -inf */
+        if (i < per && !(taken >> i & 1) && (v[i] > bv || (v[i] == bv && lane * per + i < bi))) {
+          bv = v[i];
+          bi = lane * per + i;
+        }
 #pragma unroll
       for (int o = 16; o; o >>= 1) {
         float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -1410,26 +1431,11 @@ MSK_DEV void consumer(Ctx& c) {
   q.c = &c;
   q.it = 0;
   uint32_t xpar = 0; /* this warp's expert-slot parities */
+  uint32_t dpar = 0; /* this warp's dense-slot and activation-slice parities */
   phase_in(c);
   if (!grid_sync(c, 0, PH_IN)) return;
   for (int l = 0; l < P->L; ++l) {
-    const MskLayer& Ly = P->layers[l];
-    /* QKV */
-    {
-      int sQ, sK, nq = qkv_stages(P, &sQ, &sK);
-      const int nqkv = P->qd + 2 * P->kvd;
-      for (int j = c.cta; j < nq; j += c.ncta) {
-        WStage ws = qkv_stage(P, Ly, j, sQ, sK);
-        const int coloff = ws.mat == 0 ? 0 : (ws.mat == 1 ? P->qd : P->qd + P->kvd);
-        bool ok = gemm_stage<MSK_NT_DENSE>(
-            q, ws, c.st.T, [&](int col) { return P->x + (size_t)col * P->d; },
-            [&](int row, int col, float v) {
-              if (row < ws.nrows) P->qkv[(size_t)col * nqkv + coloff + ws.row0 + row] = v;
-            },
-            l, PH_QKV);
-        if (!ok) return;
-      }
-    }
+    if (!dense_phase<true>(c, l, dpar)) return;
     if (!grid_sync(c, l, PH_QKV)) return;
     phase_qknorm(c, l);
     if (!grid_sync(c, l, PH_QKNORM)) return;
@@ -1439,19 +1445,7 @@ MSK_DEV void consumer(Ctx& c) {
     if (!grid_sync(c, l, PH_ATT)) return;
     phase_attc(c, l);
     if (!grid_sync(c, l, PH_ATTC)) return;
-    {
-      const int nwo = (P->d + rows_per_stage(P->qd) - 1) / rows_per_stage(P->qd);
-      for (int j = c.cta; j < nwo; j += c.ncta) {
-        WStage ws = wo_stage(P, Ly, j);
-        bool ok2 = gemm_stage<MSK_NT_DENSE>(
-            q, ws, c.st.T, [&](int col) { return P->o + (size_t)col * P->qd; },
-            [&](int row, int col, float v) {
-              if (row < ws.nrows) P->h[(size_t)col * P->d + ws.row0 + row] += v;
-            },
-            l, PH_WO);
-        if (!ok2) return;
-      }
-    }
+    if (!dense_phase<false>(c, l, dpar)) return;
     if (!grid_sync(c, l, PH_WO)) return;
     phase_moenorm(c, l);
     if (!grid_sync(c, l, PH_MOENORM)) return;
@@ -1497,6 +1491,13 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     c.S->ring_free = 0;
     c.S->abort = 0;
     c.S->dn_ready = 0;
+    c.S->dense_done = 0;
+    for (int w = 0; w < MSK_NCW; ++w)
+      for (int i = 0; i < DNS; ++i) {
+        mbar_init(&c.S->dfull[w][i], 1);
+        mbar_init(&c.S->dempty[w][i], 1);
+      }
+    mbar_init(&c.S->bfull, 1);
     for (int i = 0; i < XNS_MAX; ++i) {
       mbar_init(&c.S->xfull[i], 1);
       mbar_init(&c.S->xempty[i], NCW);
