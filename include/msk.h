@@ -68,8 +68,9 @@ typedef struct msk_nvfp4 {
 
 typedef struct msk_config {
   int32_t n_layers;       /* 1 .. MSK_MAX_LAYERS */
-  int32_t d_model;        /* multiple of 128, <= 4096; above 512 a multiple of 512 */
-  int32_t n_q_heads;      /* n_q_heads * head_dim <= 4096, multiple of 128 */
+  int32_t d_model;        /* multiple of 256, <= 4096; above 512 a multiple of 512 */
+  int32_t n_q_heads;      /* n_q_heads * head_dim: multiple of 256, <= 4096;
+                             above 512 a multiple of 512 */
   int32_t n_kv_heads;     /* divides n_q_heads */
   int32_t head_dim;       /* 64 or 128 */
   int32_t n_experts;      /* multiple of 32, <= 256 */

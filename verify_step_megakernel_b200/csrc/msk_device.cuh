@@ -64,9 +64,6 @@ MSK_DEV void tma_2d_g2s(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
 MSK_DEV void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y) : "memory");
 }
-MSK_DEV void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 MSK_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 /* ---- misc memory ops ------------------------------------------------------------- */

@@ -40,10 +40,10 @@ constexpr int NCT = MSK_NCW * 32;  /* consumer threads */
 constexpr int BAR_CONS = 1;        /* named barrier of the consumer warps */
 constexpr int CONS_WARP0 = 4;      /* warpgroup 0 produces, warpgroups 1-2 consume */
 constexpr int CONS0 = CONS_WARP0 * 32;
-/* registers per thread after the split; 128*40 + 256*224 must not exceed
+/* registers per thread after the split; 128*64 + 256*208 must not exceed
  * the launch pool 384 * (launch registers), checked by the host */
-constexpr int REGS_PRODUCER = 40;
-constexpr int REGS_CONSUMER = 224;
+constexpr int REGS_PRODUCER = 64;
+constexpr int REGS_CONSUMER = 208;
 
 enum Phase {
   PH_IN = 0, PH_QKV, PH_QKNORM, PH_ATT, PH_ATTC, PH_WO, PH_MOENORM, PH_ROUTER, PH_TOPK, PH_GU, PH_DN, PH_COMB
@@ -1027,7 +1027,13 @@ MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
     float v[4] = {0.f, 0.f, 0.f, 0.f};
     for (int sl = 0; sl < S; ++sl) {
       const float* raw = P->qkv + ((size_t)sl * c.st.T + t) * nqkv + hh * hd + lane * per;
-      for (int i = 0; i < per; ++i) v[i] += raw[i];
+      if (per == 4) {
+        const float4 q = *reinterpret_cast<const float4*>(raw);
+        v[0] += q.x; v[1] += q.y; v[2] += q.z; v[3] += q.w;
+      } else {
+        const float2 q = *reinterpret_cast<const float2*>(raw);
+        v[0] += q.x; v[1] += q.y;
+      }
     }
     const int b = t / c.st.Tq, ti = t % c.st.Tq;
     if (hh < P->hq + P->hkv) {
