@@ -307,10 +307,18 @@ struct Prod {
   bool ok;
 };
 
+/* The producer is one warp: every lane keeps the same schedule state and
+ * waits itself; a failed wait anywhere fails the whole warp, so its control
+ * flow stays uniform.  Lane 0 posts each barrier's byte count, then the
+ * lanes issue the copies in parallel. */
+MSK_DEV bool pwait_bar(const Ctx& c, uint64_t* bar, uint32_t parity, int layer, int phase) {
+  return __all_sync(0xffffffffu, wait_bar(c, bar, parity, layer, phase)) != 0;
+}
+
 MSK_DEV bool prod_acquire(Prod& p, int layer, int phase, uint8_t** stg, uint64_t** bar) {
   Ctx& c = *p.c;
   uint32_t slot = p.it % MSK_NST, round = p.it / MSK_NST;
-  if (round > 0 && !wait_bar(c, &c.S->empty[slot], (round - 1) & 1, layer, phase)) return false;
+  if (round > 0 && !pwait_bar(c, &c.S->empty[slot], (round - 1) & 1, layer, phase)) return false;
   *stg = c.ring + (size_t)slot * MSK_STAGE;
   *bar = &c.S->full[slot];
   p.last_parity_for_slot[slot] = round & 1;
@@ -323,7 +331,7 @@ MSK_DEV bool prod_drain(Prod& p, int layer, int phase) {
   Ctx& c = *p.c;
   const uint32_t n = p.it < MSK_NST ? p.it : MSK_NST;
   for (uint32_t i = p.it - n; i < p.it; ++i)
-    if (!wait_bar(c, &c.S->empty[i % MSK_NST], (i / MSK_NST) & 1, layer, phase)) return false;
+    if (!pwait_bar(c, &c.S->empty[i % MSK_NST], (i / MSK_NST) & 1, layer, phase)) return false;
   return true;
 }
 
@@ -342,6 +350,9 @@ MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, in
   __threadfence_block();
   return true;
 }
+MSK_DEV bool pwait_flag(const Ctx& c, volatile int* flag, int want, int layer, int phase) {
+  return __all_sync(0xffffffffu, wait_flag(c, flag, want, layer, phase)) != 0;
+}
 
 /* Feed the warps' dense weight rings for one projection: this CTA's units
  * in order, unit i of the range into warp i mod 8's next slot. */
@@ -356,7 +367,7 @@ MSK_DEV bool prod_dense(Prod& p, int layer, bool qkv) {
   for (int i = g.a; i < g.b; ++i) {
     const int w = (i - g.a) % NCW, sl = ((i - g.a) / NCW) % DNS, bit = w * DNS + sl;
     if ((p.dused >> bit) & 1u) {
-      if (!wait_bar(c, &c.S->dempty[w][sl], ((p.dpar >> bit) & 1u) ^ 1u, layer, phase)) return false;
+      if (!pwait_bar(c, &c.S->dempty[w][sl], ((p.dpar >> bit) & 1u) ^ 1u, layer, phase)) return false;
     }
     p.dpar ^= 1u << bit;
     p.dused |= 1u << bit;
@@ -366,9 +377,11 @@ MSK_DEV bool prod_dense(Prod& p, int layer, bool qkv) {
     dense_mat(P, Ly, qkv, (i % g.MT) * 16, &map, &lrow, &gs);
     uint8_t* dst = c.ring + DB_BYTES + (size_t)bit * DSLOT;
     uint64_t* bar = &c.S->dfull[w][sl];
-    mbar_arrive_tx(bar, bytes);
-    tma_2d_g2s(dst, Ly.emap + map, s * (g.KS / 4), lrow, bar);
-    tma_2d_g2s(dst + 16 * g.cpitch, Ly.emap + map + 1, s * (g.KS / 16), lrow, bar);
+    const int lane = threadIdx.x & 31;
+    if (lane == 0) mbar_arrive_tx(bar, bytes);
+    __syncwarp();
+    if (lane == 0) tma_2d_g2s(dst, Ly.emap + map, s * (g.KS / 4), lrow, bar);
+    else if (lane == 1) tma_2d_g2s(dst + 16 * g.cpitch, Ly.emap + map + 1, s * (g.KS / 16), lrow, bar);
   }
   return true;
 }
@@ -379,7 +392,7 @@ MSK_DEV void prefetch_dense(const Ctx& c, int layer, bool qkv) {
   const MskLayer& Ly = P->layers[layer];
   DGeo g;
   dgeo(c, qkv, g);
-  for (int i = g.a; i < g.b; ++i) {
+  for (int i = g.a + (int)(threadIdx.x & 31); i < g.b; i += 32) {
     int map, lrow;
     float gs;
     dense_mat(P, Ly, qkv, (i % g.MT) * 16, &map, &lrow, &gs);
@@ -406,35 +419,40 @@ MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
   const uint16_t* act = gu ? P->x2h : P->u;
   const int act_ld = gu ? P->d : P->f;
   const uint32_t brow = (uint32_t)(2 * x.KC);
+  const int lane = threadIdx.x & 31;
   int j = 0;
   for (int item = x.a; item < x.b; ++item) {
     const int unit = item / x.ngroups, grp = item % x.ngroups;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
     const int64_t grow = (int64_t)R.unit_e[unit] * x.rows_unit + (int64_t)grp * XROWS;
+    int my_row = 0; /* lanes 8.. : the activation row of the unit's token lane-8 */
+    if (lane >= 8 && lane < 8 + n) {
+      const int pair = R.pairs[st0 + lane - 8];
+      my_row = gu ? pair / P->k : pair;
+    }
     for (int kc = 0; kc < x.nkc; ++kc, ++j) {
       const int s = j % x.ns;
       if ((p.xused >> s) & 1u) {
-        if (!wait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, phase)) return false;
+        if (!pwait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, phase)) return false;
       }
       p.xpar ^= 1u << s;
       p.xused |= 1u << s;
       uint8_t* dst = c.ring + (size_t)s * x.slot_bytes;
       uint64_t* bar = &c.S->xfull[s];
-      mbar_arrive_tx(bar, x.b_off + (uint32_t)n * brow);
-      for (int m = 0; m < x.NM; ++m) {
+      if (lane == 0) mbar_arrive_tx(bar, x.b_off + (uint32_t)n * brow);
+      __syncwarp();
+      if (lane < 2 * x.NM) { /* lane 2m: codes of matrix m, lane 2m+1: its scales */
+        const int m = lane >> 1;
         uint8_t* md = dst + (size_t)m * x.mat_bytes;
         if (x.tma) {
-          tma_2d_g2s(md, cmap[m], kc * (x.KC / 4), (int32_t)grow, bar);
-          tma_2d_g2s(md + XROWS * x.cpitch, smap[m], kc * (x.KC / 16), (int32_t)grow, bar);
+          if (lane & 1) tma_2d_g2s(md + XROWS * x.cpitch, smap[m], kc * (x.KC / 16), (int32_t)grow, bar);
+          else tma_2d_g2s(md, cmap[m], kc * (x.KC / 4), (int32_t)grow, bar);
         } else {
-          bulk_g2s(md, mat[m]->codes + grow * (x.K / 2), XROWS * x.cpitch, bar);
-          bulk_g2s(md + XROWS * x.cpitch, mat[m]->scales + grow * (x.K / 16), XROWS * x.spitch, bar);
+          if (lane & 1) bulk_g2s(md + XROWS * x.cpitch, mat[m]->scales + grow * (x.K / 16), XROWS * x.spitch, bar);
+          else bulk_g2s(md, mat[m]->codes + grow * (x.K / 2), XROWS * x.cpitch, bar);
         }
-      }
-      for (int t = 0; t < n; ++t) {
-        const int pair = R.pairs[st0 + t];
-        const int row = gu ? pair / P->k : pair;
-        bulk_g2s(dst + x.b_off + t * x.bpitch, act + (size_t)row * act_ld + (size_t)kc * x.KC, brow, bar);
+      } else if (lane >= 8 && lane < 8 + n) { /* one activation row per lane */
+        bulk_g2s(dst + x.b_off + (lane - 8) * x.bpitch, act + (size_t)my_row * act_ld + (size_t)kc * x.KC, brow, bar);
       }
     }
   }
@@ -460,22 +478,24 @@ MSK_DEV void producer(Ctx& c) {
     /* attention stages reuse the memory once this CTA's QKV units are done:
      * past keys stream at once, chunks holding this step's keys wait until
      * every CTA has written them */
-    if (!wait_flag(c, &c.S->dense_done, 2 * l + 1, l, PH_ATT)) { p.ok = false; break; }
+    if (!pwait_flag(c, &c.S->dense_done, 2 * l + 1, l, PH_ATT)) { p.ok = false; break; }
     AttGeo g;
     att_geo(c, l, g);
     for_each_att_stage(c, g, [&](int pr, int slot, int64_t k0, int n, bool, bool) {
       int b = pr / P->hkv, h = pr % P->hkv;
       if (k0 + C > c.S->pos0[b]) {
-        if (!wait_flag(c, &c.S->kv_ready, l + 1, l, PH_ATT)) { p.ok = false; return false; }
+        if (!pwait_flag(c, &c.S->kv_ready, l + 1, l, PH_ATT)) { p.ok = false; return false; }
         fence_proxy_async_global();
       }
       uint8_t* stg;
       uint64_t* bar;
       if (!prod_acquire(p, l, PH_ATT, &stg, &bar)) { p.ok = false; return false; }
       int64_t row = (((int64_t)l * c.st.kv_seqs + b) * P->hkv + h) * c.st.kv_cap + k0;
-      mbar_arrive_tx(bar, (uint32_t)(2 * C * hd));
-      tma_2d_g2s(stg, c.kvmap, 0, (int32_t)row, bar);
-      tma_2d_g2s(stg + C * hd, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), bar);
+      const int lane = threadIdx.x & 31;
+      if (lane == 0) mbar_arrive_tx(bar, (uint32_t)(2 * C * hd));
+      __syncwarp();
+      if (lane == 0) tma_2d_g2s(stg, c.kvmap, 0, (int32_t)row, bar);
+      else if (lane == 1) tma_2d_g2s(stg + C * hd, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), bar);
       (void)slot;
       (void)n;
       return true;
@@ -490,15 +510,15 @@ MSK_DEV void producer(Ctx& c) {
       prefetch_dense(c, l + 1, true);
       prefetch_dense(c, l + 1, false);
     }
-    if (!wait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { p.ok = false; break; }
+    if (!pwait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { p.ok = false; break; }
     fence_proxy_async_global();
     if (!prod_experts(p, l, true)) { p.ok = false; break; }
-    if (!wait_flag(c, &c.S->dn_ready, l + 1, l, PH_DN)) { p.ok = false; break; }
+    if (!pwait_flag(c, &c.S->dn_ready, l + 1, l, PH_DN)) { p.ok = false; break; }
     fence_proxy_async_global();
     if (!prod_experts(p, l, false)) { p.ok = false; break; }
-    if (!wait_flag(c, &c.S->ring_free, l + 1, l, PH_DN)) { p.ok = false; break; }
+    if (!pwait_flag(c, &c.S->ring_free, l + 1, l, PH_DN)) { p.ok = false; break; }
   }
-  if (!p.ok) {
+  if (!p.ok && (threadIdx.x & 31) == 0) {
     /* let every copy already issued land before the CTA may exit */
     for (int bit = 0; bit < NCW * DNS; ++bit) {
       if (!((p.dused >> bit) & 1u)) continue;
@@ -1531,7 +1551,7 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
   }
   if (threadIdx.x < CONS0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
-    if (threadIdx.x == 0) producer(c);
+    if (threadIdx.x < 32) producer(c);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_CONSUMER));
     consumer<HD>(c);
