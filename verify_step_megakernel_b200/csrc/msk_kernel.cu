@@ -137,20 +137,23 @@ MSK_DEV bool grid_sync(Ctx& c, int layer, int phase) {
   if (threadIdx.x == CONS0) {
     int ok = !c.S->abort;
     if (ok) {
-      __threadfence();
-      atomicAdd(&c.P->ctrl[CTRL_BARRIER], 1u);
-      uint32_t target = (c.nbar + 1) * (uint32_t)c.ncta;
-      uint64_t t0 = gtimer();
-      while (ld_acquire_u32(&c.P->ctrl[CTRL_BARRIER]) < target) {
-        if (ld_volatile_u32(&c.P->ctrl[CTRL_ABORT])) { ok = 0; break; }
-        if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
-          raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
-          ok = 0;
-          break;
+      /* release: the CTA's writes (ordered before this thread by the CTA
+       * barrier above) become visible before the count moves; acquire on
+       * the poll orders the other CTAs' writes before ours */
+      red_release_add_u32(&c.P->ctrl[CTRL_BARRIER], 1u);
+      const uint32_t target = (c.nbar + 1) * (uint32_t)c.ncta;
+      uint64_t t0 = 0;
+      for (uint32_t it = 0; ld_acquire_u32(&c.P->ctrl[CTRL_BARRIER]) < target; ++it) {
+        if ((it & 15) == 15) { /* the abort word and the clock, now and then */
+          if (ld_volatile_u32(&c.P->ctrl[CTRL_ABORT])) { ok = 0; break; }
+          if (t0 == 0) t0 = gtimer();
+          else if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+            raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
+            ok = 0;
+            break;
+          }
         }
-        __nanosleep(64);
       }
-      __threadfence();
     }
     if (!ok) c.S->abort = 1;
     s_ok = ok;
