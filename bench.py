@@ -195,7 +195,7 @@ def run_msk(args, w):
             dist.barrier()
 
     t_setup = time.perf_counter()
-    eng = Engine(w, device=local)
+    eng = Engine(w, device=local, flags=msk.F_TC_EXPERTS if args.tc_experts else 0)
     eng.fill_past()
     hid = sg.hidden(w, local)
     pos = torch.tensor(w.positions(), dtype=torch.int32, device=dev)
@@ -369,6 +369,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-threads", type=int, default=0)
     ap.add_argument("--trace", action="store_true", help="print a per-phase device-time breakdown instead")
+    ap.add_argument("--tc-experts", action="store_true",
+                    help="gate/up on the block-scaled tensor cores (MSK_F_TC_EXPERTS) instead of the default path")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

@@ -89,6 +89,13 @@ typedef struct msk_config {
 } msk_config_t;
 
 #define MSK_F_TRACE 1u /* record per-phase %globaltimer stamps (msk_query) */
+/* Gate/up projections on the block-scaled tensor cores (tcgen05.mma
+ * kind::mxf4nvf4): the NVFP4 weights are consumed as stored, the moe-norm
+ * activations as eight e2m1 terms (relative error ~1e-5 of the row's
+ * largest value).  Default off: with units of 2-3 tokens per expert the
+ * per-instruction cost of the tensor-core path exceeds the CUDA-core
+ * decode it saves (see the design notes for the measurements). */
+#define MSK_F_TC_EXPERTS 2u
 
 /* Per-layer weights, all device pointers, borrowed.
  *  attn_norm_g [d], moe_norm_g [d]      RMSNorm gains (fp32)

@@ -50,6 +50,20 @@ def _kv_written_match(w, eng, ref, positions, seqs):
 
 
 @pytest.mark.parametrize("name", ["tiny", "dec8", "ver8"])
+def test_parity_tensor_core_experts(name):
+    """The same parity bar with gate/up on the block-scaled tensor cores
+    (MSK_F_TC_EXPERTS): NVFP4 weights as stored, activations as e2m1 terms."""
+    w = synth.WORKLOADS[name]
+    eng = Engine(w, flags=msk.F_TC_EXPERTS)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions())
+    _report(name + " tc", rep)
+    assert_parity(rep)
+    eng.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "dec8", "ver8"])
 def test_parity_workload(name):
     w = synth.WORKLOADS[name]
     eng = Engine(w)
@@ -67,10 +81,11 @@ RAGGED = Workload("ragged", 3, 256, 4, 2, 64, 128, [1, 0, 1], 3, 3, 0, 0x5EED + 
                   window=100)
 
 
-def test_parity_ragged_sequences():
+@pytest.mark.parametrize("flags", [0, msk.F_TC_EXPERTS], ids=["cuda_core", "tensor_core"])
+def test_parity_ragged_sequences(flags):
     w = RAGGED
     past = [0, 130, 517]  # empty past, a chunk boundary crossed, window < context
-    eng = Engine(w, past_per_seq=past)
+    eng = Engine(w, past_per_seq=past, flags=flags)
     eng.fill_past()
     hid = sg.hidden(w)
     pos = [[p + i for i in range(w.tokens_per_seq)] for p in past]

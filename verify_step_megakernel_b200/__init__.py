@@ -17,6 +17,7 @@ MAX_TOKENS = 64
 STATUS = {0: "MSK_OK", 1: "MSK_ERR_INVALID_ARG", 2: "MSK_ERR_UNSUPPORTED", 3: "MSK_ERR_OOM", 4: "MSK_ERR_CUDA",
           5: "MSK_ERR_BOUND", 6: "MSK_ERR_KV_RANGE", 7: "MSK_ERR_TIMEOUT", 8: "MSK_ERR_DEVICE"}
 F_TRACE = 1
+F_TC_EXPERTS = 2  # gate/up on the block-scaled tensor cores
 
 
 class MskError(RuntimeError):

@@ -121,7 +121,7 @@ static StaticSlot g_static_slots[MSK_STATIC_MAX_DEVICES];
 
 /* where the step's buffers sit inside g_static_scratch */
 struct StaticLayout {
-  size_t params, h, x, qkv, qs, part, o, x2f, x2h, logits, u, y, ctrl, total;
+  size_t params, h, x, qkv, qs, part, o, x2f, x2h, xq, logits, u, y, ctrl, total;
 };
 
 static StaticLayout static_layout(const msk_handle_t* h) {
@@ -141,6 +141,7 @@ static StaticLayout static_layout(const msk_handle_t* h) {
   L.o = take(T * qd * 2);
   L.x2f = take(T * d * 4);
   L.x2h = take(T * d * 2);
+  L.xq = take(T * MSK_XQ_BYTES(d));
   L.logits = take(T * P.E * 4);
   L.u = take(T * P.k * P.f * 2);
   L.y = take(T * P.k * d * 4);
@@ -158,6 +159,7 @@ struct StaticPtrs {
   uint16_t* o;
   float* x2f;
   uint16_t* x2h;
+  uint8_t* xq;
   float* logits;
   uint16_t* u;
   float* y;
@@ -181,6 +183,7 @@ __global__ void msk_static_params(const MskParams* src, MskParams* dst, StaticPt
     dst->o = p.o;
     dst->x2f = p.x2f;
     dst->x2h = p.x2h;
+    dst->xq = p.xq;
     dst->logits = p.logits;
     dst->u = p.u;
     dst->y = p.y;
@@ -293,6 +296,7 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       T * qd * 2,                /* o */
       T * d * 4,                 /* x2f */
       T * d * 2,                 /* x2h */
+      T * MSK_XQ_BYTES(d),       /* xq */
       T * P.E * 4,               /* logits */
       T * P.k * P.f * 2,         /* u */
       T * P.k * d * 4,           /* y */
@@ -315,13 +319,14 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   P.o = (uint16_t*)(b + off[5]);
   P.x2f = (float*)(b + off[6]);
   P.x2h = (uint16_t*)(b + off[7]);
-  P.logits = (float*)(b + off[8]);
-  P.u = (uint16_t*)(b + off[9]);
-  P.y = (float*)(b + off[10]);
-  P.ctrl = (uint32_t*)(b + off[11]);
+  P.xq = b + off[8];
+  P.logits = (float*)(b + off[9]);
+  P.u = (uint16_t*)(b + off[10]);
+  P.y = (float*)(b + off[11]);
+  P.ctrl = (uint32_t*)(b + off[12]);
   P.status = P.ctrl + CTRL_WORDS;
-  P.n_distinct = (int32_t*)(b + off[12]);
-  P.last_shape = (int32_t*)(b + off[13]);
+  P.n_distinct = (int32_t*)(b + off[13]);
+  P.last_shape = (int32_t*)(b + off[14]);
   h->words = P.ctrl;
   /* tensor maps of the expert tensors, for the K-chunked expert tiles */
   {
@@ -333,7 +338,8 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       const msk_nvfp4_t* mats[3] = {&w.w_gate, &w.w_up, &w.w_down};
       for (int m = 0; m < 3 && ok; ++m) {
         const int64_t K = m < 2 ? P.d : P.f, rows = (int64_t)P.E * (m < 2 ? P.f : P.d);
-        const int KC = K <= 512 ? (int)K : 512;
+        /* K chunks: 256 for gate/up on the tensor cores, else 512 (or all of K) */
+        const int KC = (m < 2 && (c.flags & MSK_F_TC_EXPERTS)) ? 256 : (K <= 512 ? (int)K : 512);
         /* K not a multiple of 256 (128, 384): whole rows go as bulk copies
          * and the maps stay zero */
         if (K % 256) continue;
@@ -369,6 +375,18 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
         }
+      }
+      /* gate and up codes for the block-scaled tensor cores: 128 rows x 128
+       * bytes (256 codes) per box, 128-byte swizzle */
+      for (int m = 0; m < 2 && ok; ++m) {
+        const int64_t K = P.d, rows = (int64_t)P.E * P.f;
+        cuuint64_t dims[2] = {(cuuint64_t)(K / 2), (cuuint64_t)rows};
+        cuuint64_t strides[1] = {(cuuint64_t)(K / 2)};
+        cuuint32_t box[2] = {128, 128};
+        cuuint32_t estr[2] = {1, 1};
+        ok = enc(&hm[l * MSK_NMAPS + MSK_MAP_GUSW + m], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, (void*)mats[m]->codes, dims,
+                 strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
       }
       P.layers[l].emap = h->emaps + l * MSK_NMAPS;
     }
@@ -659,6 +677,7 @@ msk_status_t msk_step_static(msk_handle_t* h, const uint16_t* hidden_in, const i
     p.o = (uint16_t*)(b + Lo.o);
     p.x2f = (float*)(b + Lo.x2f);
     p.x2h = (uint16_t*)(b + Lo.x2h);
+    p.xq = b + Lo.xq;
     p.logits = (float*)(b + Lo.logits);
     p.u = (uint16_t*)(b + Lo.u);
     p.y = (float*)(b + Lo.y);

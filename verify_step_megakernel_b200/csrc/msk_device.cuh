@@ -66,6 +66,57 @@ MSK_DEV void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
 }
 MSK_DEV void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
+/* ---- 5th-generation tensor cores (tcgen05) ----------------------------------------- */
+/* shared-memory matrix descriptor: start address, leading / stride byte
+ * offsets (16-byte units), version 1, layout (0 none, 2 = 128-byte swizzle) */
+MSK_DEV uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+         ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46) | ((uint64_t)(layout & 7u) << 61);
+}
+MSK_DEV void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+               "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+MSK_DEV void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+MSK_DEV void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+MSK_DEV void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+MSK_DEV void fence_proxy_async_shared() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+/* 32 rows x 16 bytes of shared memory -> TMEM, replicated into the four
+ * 32-lane quadrants (the layout block-scale factors use) */
+MSK_DEV void tc_cp_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+/* D (+)= A B^T, A and B NVFP4 (e2m1 codes, ue4m3 scale per 16 along K) */
+MSK_DEV void tc_mma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate,
+                         uint32_t tmem_sfa, uint32_t tmem_sfb) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
+      : "memory");
+}
+/* arrive on an mbarrier once every tcgen05 operation this thread issued has completed */
+MSK_DEV void tc_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+/* 32 consecutive TMEM columns of this warp's 32 lanes */
+MSK_DEV void tc_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,"
+      "%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+MSK_DEV void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
 /* ---- misc memory ops ------------------------------------------------------------- */
 MSK_DEV uint32_t ld_acquire_u32(const uint32_t* p) {
   uint32_t v;
@@ -84,6 +135,15 @@ MSK_DEV uint32_t ld_volatile_u32(const uint32_t* p) {
 }
 MSK_DEV void named_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+/* named barrier that also ORs a predicate over the participating threads */
+MSK_DEV bool named_sync_or(int id, int nthreads, bool pred) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n barrier.cta.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}"
+               : "=r"(r)
+               : "r"((uint32_t)pred), "r"(id), "r"(nthreads)
+               : "memory");
+  return r != 0;
 }
 MSK_DEV uint4 lds128(uint32_t addr) {
   uint4 v;
@@ -139,6 +199,24 @@ MSK_DEV uint32_t e4m3x2_to_f16x2(uint32_t two) {
 MSK_DEV uint32_t e4m3pair_to_bf16x2_scaled(uint32_t w0, uint32_t w1, uint32_t sel) {
   uint32_t t = __byte_perm(w0, w1, sel); /* [b, b, b', b'] */
   return (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
+}
+/* the low / high f16 of an f16x2 word as fp32 (exact) */
+MSK_DEV float f16lo_f32(uint32_t w) {
+  float f;
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n cvt.f32.f16 %0, l;\n}" : "=f"(f) : "r"(w));
+  return f;
+}
+MSK_DEV float f16hi_f32(uint32_t w) {
+  float f;
+  asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n cvt.f32.f16 %0, h;\n}" : "=f"(f) : "r"(w));
+  return f;
+}
+/* two floats -> e2m1x2 byte (low nibble = a, high = b), round to nearest
+ * even on the e2m1 grid, saturating at 6 */
+MSK_DEV uint32_t f32x2_to_e2m1x2(float a, float b) {
+  uint32_t r;
+  asm("{\n .reg .b8 q;\n cvt.rn.satfinite.e2m1x2.f32 q, %1, %2;\n cvt.u32.u8 %0, q;\n}" : "=r"(r) : "f"(b), "f"(a));
+  return r;
 }
 /* two floats -> e4m3x2 (lo = a, hi = b), round to nearest even, satfinite */
 MSK_DEV uint32_t f32x2_to_e4m3x2(float a, float b) {

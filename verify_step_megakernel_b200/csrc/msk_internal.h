@@ -23,7 +23,9 @@
 #define MSK_MAX_PAIRS 64     /* (sequence, kv-head) attention pairs */
 
 #define MSK_MAP_DENSE 6
-#define MSK_NMAPS 14
+#define MSK_MAP_GUSW 14 /* gate and up codes as 128-byte-swizzled 128 x 128-byte boxes */
+#define MSK_NMAPS 16
+#define MSK_XQ_BYTES(d) ((size_t)(d) * 4 + 16)
 
 /* per-step control words (zeroed before every launch) */
 enum { CTRL_BARRIER = 0, CTRL_ABORT = 1, CTRL_WORDS = 32 };
@@ -66,7 +68,9 @@ typedef struct MskParams {
   float* part;      /* [slots][R_max][hd + 4] attention partials */
   uint16_t* o;      /* [T][qd] f16 attention output */
   float* x2f;       /* [T][d] moe-norm output, fp32 (router) */
-  uint16_t* x2h;    /* [T][d] same, f16 (experts) */
+  uint16_t* x2h;    /* [T][d] same, f16 (gate/up on the CUDA-core path) */
+  uint8_t* xq;      /* [T] the same row as eight e2m1 terms for the gate/up tensor cores, MSK_XQ_BYTES(d) each:
+                       codes [d/32][8 term rows][16 B], then the fp32 factor */
   float* logits;    /* [T][E] */
   uint16_t* u;      /* [T*k][f] f16 SwiGLU activations */
   float* y;         /* [T*k][d] expert outputs */

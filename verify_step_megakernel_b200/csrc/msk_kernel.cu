@@ -75,8 +75,16 @@ struct Smem {
   uint64_t dfull[MSK_NCW][2];  /* dense weight slot of a warp landed */
   uint64_t dempty[MSK_NCW][2]; /* dense weight slot read by its warp */
   uint64_t bfull;              /* dense activation slice landed */
+  uint64_t sfdone[4];       /* tensor-core ops up to the last chunk using scale staging b done */
+  uint64_t sfready[4];      /* scale staging b written by every consumer warp */
+  uint64_t dfull2[2];       /* accumulator buffer 0/1 holds a finished item */
+  uint64_t dempty2[2];      /* accumulator buffer 0/1 read by every consumer warp */
+  uint64_t tfin;            /* every tensor-core op issued complete */
+  uint32_t tmem_base;
+  uint4 sfb_one[32];        /* 128 rows x 4 ue4m3 scales of 1.0, the activation terms' scales */
+  volatile int issuer_done; /* the MMA-issuing warp has committed its last work */
   uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
-  uint64_t xempty[XNS_MAX]; /* expert slot read by all consumer warps */
+  uint64_t xempty[XNS_MAX]; /* expert slot consumed (one arrival: a tensor-core commit or the consumers' last warp) */
   volatile int kv_ready;    /* layer+1 whose KV writes all CTAs finished */
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
@@ -179,17 +187,43 @@ MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
  * bytes off the 128-byte bank period; with the lanes' interleaved block
  * order below, the warp's shared loads are then free of bank conflicts.
  * Other K (128, 384) take whole rows as single bulk copies. */
+/* gate/up on the block-scaled tensor cores: K chunks of 256, slot layout
+ * (1024-byte aligned, four slots in the ring):
+ * [GU_A]  codes of gate, up: one 128-row x 128-byte box each (256 codes per
+ *         row), 128-byte swizzled — the K-major SW128 layout
+ * [GU_AS] scales of gate, up: [128 rows][16] each
+ * [GU_B]  the unit's tokens' activation terms: token t at t*1024, its chunk's
+ *         [8 core-matrix columns][8 term rows][16 B] (all term scales are 1) */
+constexpr int GU_KC = 256;
+constexpr uint32_t GU_A = 0, GU_AS = 32768, GU_B = 36864, GU_SLOT = 45056;
+/* TMEM columns: two buffers of gate and up accumulators (128 lanes x 64
+ * each), then the scale factors of two chunks in flight */
+constexpr uint32_t TM_D = 0, TM_DU = 64, TM_SFA = 256, TM_SFB = 384, TM_COLS = 512;
+/* scale-factor buffers: four chunks in flight, so that waiting for the
+ * copies of chunk j-4 (a commit covers every earlier op) does not
+ * serialise the consumers' staging with the tensor pipe */
+constexpr int NSF = 4;
+constexpr uint32_t TM_SFA_BUF = 32; /* columns per buffer: 2 matrices x 4 steps x 4; SFB: 4 columns of ones */
+/* per-chunk staging of the scale factors in the interleaved block layout
+ * (scratch region): SFA [matrix][k step][512 B], SFB [k step][512 B] */
+constexpr uint32_t SF_STAGE = 4096; /* SFA [matrix][4 k steps][512 B] */
+static_assert(NSF * SF_STAGE <= MSK_SCR, "scale staging fits the scratch region");
+static_assert(TM_SFA + NSF * TM_SFA_BUF <= TM_SFB && TM_SFB + 4 <= TM_COLS, "TMEM columns");
+
 struct XGeo {
   int K, KC, nkc, rows_unit, ngroups, NM, tma, ns;
   uint32_t cpitch, spitch, bpitch, mat_bytes, b_off, slot_bytes;
   int a, b; /* this CTA's items [a, b) */
 };
 
+MSK_DEV bool tc_experts(const MskParams* P) { return (P->flags & MSK_F_TC_EXPERTS) != 0; }
+
 MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
   const MskParams* P = c.P;
+  const bool tc = gu && tc_experts(P);
   x.K = gu ? P->d : P->f;
   x.rows_unit = gu ? P->f : P->d;
-  x.KC = x.K <= XKC_MAX ? x.K : XKC_MAX;
+  x.KC = tc ? GU_KC : (x.K <= XKC_MAX ? x.K : XKC_MAX);
   x.nkc = x.K / x.KC;
   x.tma = (x.K % 256) == 0;
   x.cpitch = (uint32_t)(x.tma ? x.KC / 2 + 32 : x.KC / 2);
@@ -198,7 +232,7 @@ MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
   x.NM = gu ? 2 : 1;
   x.mat_bytes = XROWS * (x.cpitch + x.spitch);
   x.b_off = x.NM * x.mat_bytes;
-  x.slot_bytes = (x.b_off + MSK_UNIT_TOK * x.bpitch + 127) & ~127u;
+  x.slot_bytes = tc ? GU_SLOT : (x.b_off + MSK_UNIT_TOK * x.bpitch + 127) & ~127u;
   x.ns = min(XNS_MAX, (int)((uint32_t)(MSK_NST * MSK_STAGE) / x.slot_bytes));
   x.ngroups = x.rows_unit / XROWS;
   item_range(c.S->route.n_units * x.ngroups, c.cta, c.ncta, &x.a, &x.b);
@@ -206,7 +240,8 @@ MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
 /* gate+up with K = 512 is the largest slot: two must fit the ring */
 static_assert(2 * ((2 * XROWS * (XKC_MAX / 2 + 32 + XKC_MAX / 16) + MSK_UNIT_TOK * (2 * XKC_MAX + 16) + 127) & ~127) <=
                   MSK_NST * MSK_STAGE,
-              "two expert slots fit the stage ring");
+              "two gate+up slots of the CUDA-core path fit the stage ring");
+static_assert(XNS_MAX * GU_SLOT <= MSK_NST * MSK_STAGE, "four gate/up slots fit the stage ring");
 
 /* Dense projections (QKV, W_o) with T <= 64 tokens: split-K over CTAs.  A
  * unit is one 16-row m-tile of the output rows times one K slice of 512 (or
@@ -419,16 +454,49 @@ MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
   const MskNv* mat[2] = {gu ? &Ly.wg : &Ly.wd, &Ly.wu};
   const CUtensorMap* cmap[2] = {Ly.emap + (gu ? 0 : 4), Ly.emap + 2};
   const CUtensorMap* smap[2] = {Ly.emap + (gu ? 1 : 5), Ly.emap + 3};
+  const int lane = threadIdx.x & 31;
+  int j = 0;
+  if (gu && tc_experts(P)) { /* block-scaled tensor cores: swizzled code boxes, raw scales, the tokens' terms */
+    const size_t xqb = MSK_XQ_BYTES(P->d);
+    for (int item = x.a; item < x.b; ++item) {
+      const int unit = item / x.ngroups, grp = item % x.ngroups;
+      const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+      const int64_t grow = (int64_t)R.unit_e[unit] * x.rows_unit + (int64_t)grp * XROWS;
+      const int tl = lane - 8; /* lanes 8-15 copy token tl's terms */
+      const uint8_t* tq = nullptr;
+      if (lane >= 8 && tl < n) tq = P->xq + (size_t)(R.pairs[st0 + tl] / P->k) * xqb;
+      const uint32_t bytes = (uint32_t)(2 * 16384 + 2 * XROWS * (GU_KC / 16) + n * 8 * (GU_KC / 2));
+      for (int kc = 0; kc < x.nkc; ++kc, ++j) {
+        const int s = j % x.ns;
+        if ((p.xused >> s) & 1u) {
+          if (!pwait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, phase)) return false;
+        }
+        p.xpar ^= 1u << s;
+        p.xused |= 1u << s;
+        uint8_t* dst = c.ring + (size_t)s * x.slot_bytes;
+        uint64_t* bar = &c.S->xfull[s];
+        if (lane == 0) mbar_arrive_tx(bar, bytes);
+        __syncwarp();
+        if (lane < 2) {
+          tma_2d_g2s(dst + GU_A + lane * 16384, Ly.emap + MSK_MAP_GUSW + lane, kc * (GU_KC / 2), (int32_t)grow, bar);
+        } else if (lane == 4 || lane == 5) {
+          const int m = lane - 4;
+          tma_2d_g2s(dst + GU_AS + m * (XROWS * GU_KC / 16), smap[m], kc * (GU_KC / 16), (int32_t)grow, bar);
+        } else if (tq) {
+          bulk_g2s(dst + GU_B + tl * (8 * GU_KC / 2), tq + (size_t)kc * (8 * GU_KC / 2), 8 * GU_KC / 2, bar);
+        }
+      }
+    }
+    return true;
+  }
   const uint16_t* act = gu ? P->x2h : P->u;
   const int act_ld = gu ? P->d : P->f;
   const uint32_t brow = (uint32_t)(2 * x.KC);
-  const int lane = threadIdx.x & 31;
-  int j = 0;
   for (int item = x.a; item < x.b; ++item) {
     const int unit = item / x.ngroups, grp = item % x.ngroups;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
     const int64_t grow = (int64_t)R.unit_e[unit] * x.rows_unit + (int64_t)grp * XROWS;
-    int my_row = 0; /* lanes 8.. : the activation row of the unit's token lane-8 */
+    int my_row = 0; /* lanes 8.. : the activation row of the unit's entry lane-8 (token, or pair) */
     if (lane >= 8 && lane < 8 + n) {
       const int pair = R.pairs[st0 + lane - 8];
       my_row = gu ? pair / P->k : pair;
@@ -460,6 +528,78 @@ MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
     }
   }
   return true;
+}
+
+/* The MMA-issuing warp (one elected lane does the issuing): walks the same
+ * gate/up chunk sequence as the consumers; per chunk it waits for the
+ * consumers' scale staging, copies the scales into TMEM, issues the
+ * block-scaled MMAs into the item's accumulator buffer (after the
+ * consumers released that buffer) and commits (see expert_gu_tc). */
+MSK_DEV void issuer(Ctx& c) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31;
+  const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(64 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+  uint32_t bits = 0; /* 0-3 sfready parities, 4-5 dempty parities, 6-7 accumulator buffer used */
+  bool ok = true;
+  uint32_t tb = 0;
+  for (int l = 0; l < P->L && ok && tc_experts(P); ++l) {
+    if (!pwait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { ok = false; break; }
+    tb = c.S->tmem_base;
+    if (l == 0) { /* the activation terms' block scales, all 1.0 (ue4m3 0x38), once */
+      c.S->sfb_one[lane] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) {
+        tc_fence_after();
+        tc_cp_sf(tb + TM_SFB, umma_desc(smem_u32(c.S->sfb_one), 16, 128, 0));
+      }
+      __syncwarp();
+    }
+    XGeo x;
+    xgeo(c, true, x);
+    const int nsteps = x.KC / 64;
+    const uint32_t ring = smem_u32(c.ring), sfs = smem_u32(c.scr);
+    int j = 0;
+    for (int item = x.a; item < x.b && ok; ++item) {
+      const int db = (item - x.a) & 1;
+      for (int kc = 0; kc < x.nkc; ++kc, ++j) {
+        const int s = j % x.ns, buf = j & (NSF - 1);
+        if (!pwait_bar(c, &c.S->sfready[buf], (bits >> buf) & 1u, l, PH_GU)) { ok = false; break; }
+        bits ^= 1u << buf;
+        if (kc == 0 && ((bits >> (6 + db)) & 1u)) {
+          if (!pwait_bar(c, &c.S->dempty2[db], (bits >> (4 + db)) & 1u, l, PH_GU)) { ok = false; break; }
+          bits ^= 1u << (4 + db);
+        }
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t slot = ring + (uint32_t)s * x.slot_bytes, stg = sfs + (uint32_t)buf * SF_STAGE;
+          const uint64_t sd = umma_desc(stg, 16, 128, 0), ad = umma_desc(slot + GU_A, 16, 1024, 2),
+                         bd = umma_desc(slot + GU_B, 128, 8 * GU_KC / 2, 0);
+          const uint32_t sfa = tb + TM_SFA + buf * TM_SFA_BUF, sfb = tb + TM_SFB, dg = tb + TM_D + db * 128;
+#pragma unroll 1
+          for (int st = 0; st < 2 * nsteps; ++st) tc_cp_sf(sfa + 4 * st, sd + (uint64_t)((st * 512) >> 4));
+#pragma unroll 1
+          for (int st = 0; st < nsteps; ++st) {
+            const uint32_t acc = (kc > 0 || st > 0) ? 1u : 0u;
+            const uint64_t b = bd + (uint64_t)((256 * st) >> 4);
+            const uint64_t a = ad + (uint64_t)((32 * st) >> 4);
+            tc_mma_nvf4(dg, a, b, idesc, acc, sfa + 4 * st, sfb);
+            tc_mma_nvf4(dg + TM_DU, a + (uint64_t)(16384 >> 4), b, idesc, acc, sfa + 16 + 4 * st, sfb);
+          }
+          tc_commit(&c.S->xempty[s]);
+          tc_commit(&c.S->sfdone[buf]);
+          if (kc == x.nkc - 1) tc_commit(&c.S->dfull2[db]);
+        }
+        __syncwarp();
+        if (kc == x.nkc - 1) bits |= 1u << (6 + db);
+      }
+    }
+  }
+  if (lane == 0) {
+    tc_commit(&c.S->tfin);
+    __threadfence_block();
+    c.S->issuer_done = 1;
+  }
 }
 
 MSK_DEV void producer(Ctx& c) {
@@ -686,12 +826,12 @@ MSK_DEV bool dense_phase(Ctx& c, int layer, uint32_t& dpar) {
     i0 = i1;
   }
   if (!ok) c.S->abort = 1;
-  named_sync(BAR_CONS, NCT);
+  const bool aborting = named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
   if (ctid == 0) {
     __threadfence_block();
     c.S->dense_done = 2 * layer + (QKV ? 1 : 2);
   }
-  return !c.S->abort;
+  return !aborting;
 }
 
 /* ---- consumer: attention stages ------------------------------------------------------ */
@@ -963,8 +1103,8 @@ MSK_DEV bool attention_phase_mt(Cons& q, int layer) {
       att_end<HD, MT>(c, A, c.cta + p, ngroups, ks);
     }
   }
-  named_sync(BAR_CONS, NCT);
-  return !c.S->abort;
+  /* one answer for every warp, even if the abort word changes meanwhile */
+  return !named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
 }
 
 /* one warp owns up to two 16-row tiles of a pair (their keys are converted
@@ -1007,9 +1147,75 @@ MSK_DEV void row_norm_store(const float4* v, int d, float r, const float* gain, 
       const float4 gg = *reinterpret_cast<const float4*>(gain + i);
       const float a = v[u].x * r * gg.x, b = v[u].y * r * gg.y, cc = v[u].z * r * gg.z, dd = v[u].w * r * gg.w;
       if (xf) *reinterpret_cast<float4*>(xf + i) = make_float4(a, b, cc, dd);
-      *reinterpret_cast<uint2*>(xh + i) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(cc, dd));
+      if (xh) *reinterpret_cast<uint2*>(xh + i) = make_uint2(f32x2_to_f16x2(a, b), f32x2_to_f16x2(cc, dd));
     }
   }
+}
+
+MSK_DEV float cta_max(const Ctx& c, float part) {
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) part = fmaxf(part, __shfl_xor_sync(0xffffffffu, part, o));
+  if (lane == 0) c.S->red8[cw] = part;
+  named_sync(BAR_CONS, NCT);
+  float t = 0.f;
+#pragma unroll
+  for (int i = 0; i < NCW; ++i) t = fmaxf(t, c.S->red8[i]);
+  named_sync(BAR_CONS, NCT);
+  return t;
+}
+
+/* The moe-norm row of a token as eight e2m1 terms for the block-scaled
+ * tensor cores, all with block scale 1: with f0 the power of two that
+ * brings the row's largest magnitude into (3, 6], term j codes the
+ * residual the previous terms left, scaled by f0 4^j, rounded to nearest
+ * on the e2m1 grid.  Each term leaves at most one grid unit of its scale,
+ * which the next (4x finer) term still represents without clipping, so
+ * eight terms reach about 6^-1 4^-7 (~1e-5) of the row's largest value.
+ * Layout per token (xq): codes [d/32][8 term rows][16 B] (one 8-row
+ * core-matrix group per token, any 256-wide K chunk one contiguous
+ * kilobyte), then the fp32 factor 1/f0. */
+MSK_DEV void row_quant8(const Ctx& c, const float4* v, int d, float r, const float* gain, uint8_t* xq) {
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  const int sl = d / NCW, base = cw * sl + lane * 4;
+  float x[ROWV][4];
+  float mx = 0.f;
+#pragma unroll
+  for (int u = 0; u < ROWV; ++u) {
+    const int i = base + u * 128;
+    x[u][0] = x[u][1] = x[u][2] = x[u][3] = 0.f;
+    if (i < (cw + 1) * sl) {
+      const float4 gg = *reinterpret_cast<const float4*>(gain + i);
+      x[u][0] = v[u].x * r * gg.x;
+      x[u][1] = v[u].y * r * gg.y;
+      x[u][2] = v[u].z * r * gg.z;
+      x[u][3] = v[u].w * r * gg.w;
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(x[u][0]), fabsf(x[u][1])), fmaxf(fabsf(x[u][2]), fabsf(x[u][3]))));
+    }
+  }
+  mx = cta_max(c, mx);
+  int pe = 0;
+  if (mx > 0.f) pe = max(-100, min(100, (int)floorf(log2f(6.0f / mx))));
+  float fj = __int_as_float((127 + pe) << 23); /* f0 */
+  const float finv = __int_as_float((127 - pe) << 23);
+#pragma unroll
+  for (int t = 0; t < 8; ++t) {
+    const float inv = 1.0f / fj; /* powers of two: exact */
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      const uint32_t c01 = f32x2_to_e2m1x2(x[u][0] * fj, x[u][1] * fj), c23 = f32x2_to_e2m1x2(x[u][2] * fj, x[u][3] * fj);
+      const uint32_t h01 = e2m1x2_to_f16x2(c01), h23 = e2m1x2_to_f16x2(c23);
+      x[u][0] -= f16lo_f32(h01) * inv;
+      x[u][1] -= f16hi_f32(h01) * inv;
+      x[u][2] -= f16lo_f32(h23) * inv;
+      x[u][3] -= f16hi_f32(h23) * inv;
+      if (i < (cw + 1) * sl)
+        *reinterpret_cast<uint16_t*>(xq + (size_t)(i / 32) * 128 + t * 16 + (i % 32) / 2) = (uint16_t)(c01 | (c23 << 8));
+    }
+    fj *= 4.0f;
+  }
+  if (cw == 0 && lane == 0) *reinterpret_cast<float*>(xq + (size_t)4 * d) = finv;
 }
 
 MSK_DEV void phase_in(const Ctx& c) {
@@ -1141,7 +1347,12 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
       }
     }
     const float r = 1.0f / sqrtf(cta_sum(c, ss) / d + P->eps);
-    row_norm_store(v, d, r, P->layers[layer].g_moe, P->x2h + (size_t)t * d, P->x2f + (size_t)t * d);
+    if (tc_experts(P)) {
+      row_norm_store(v, d, r, P->layers[layer].g_moe, nullptr, P->x2f + (size_t)t * d);
+      row_quant8(c, v, d, r, P->layers[layer].g_moe, P->xq + (size_t)t * MSK_XQ_BYTES(d));
+    } else {
+      row_norm_store(v, d, r, P->layers[layer].g_moe, P->x2h + (size_t)t * d, P->x2f + (size_t)t * d);
+    }
   }
 }
 
@@ -1397,41 +1608,142 @@ MSK_DEV void xgemm(uint32_t codes, uint32_t scales, uint32_t mstride, uint32_t c
   }
 }
 
-/* gate/up (GU) or down projection of the selected experts: this CTA's
- * items, 16 rows per warp, chunks from the producer's ring.  xpar bit s is
- * this warp's parity of the uses of slot s so far. */
+/* Gate/up of the selected experts on the block-scaled tensor cores
+ * (tcgen05.mma kind::mxf4nvf4, M = 128 weight rows, N = 8 tokens x 8 term
+ * rows, K = 64 per instruction, fp32 accumulators in TMEM).  Three parties
+ * per chunk: the producer warp lands the slot; each consumer warp lays its
+ * share of the chunk's scales out in the interleaved block layout the
+ * scale-factor copies read (staging buffer j mod 4) and arrives on
+ * sfready; the issuing warp then copies the scales into TMEM, issues the
+ * MMAs and commits to the slot's empty barrier, the staging barrier and,
+ * after an item's last chunk, to that item's accumulator buffer (two
+ * buffers, so an item's epilogue overlaps the next item's MMAs).  The
+ * epilogue reads the accumulators (TMEM lane = weight row), sums each
+ * token's four term columns, undoes the token's power-of-two factor and
+ * applies the global scales and SwiGLU.
+ * xpar: bits 0-3 weight-slot parities; 4-7 parity of the chunks handed
+ * to each staging buffer, 8-11 whether any was; 12-13 accumulator-buffer
+ * parities. */
+MSK_DEV bool expert_gu_tc(Ctx& c, int layer, uint32_t& xpar) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const Route& R = c.S->route;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  XGeo x;
+  xgeo(c, true, x);
+  const int f = P->f, nsteps = x.KC / 64;
+  const float gs0 = Ly.wg.gs, gs1 = Ly.wu.gs;
+  const size_t xqb = MSK_XQ_BYTES(P->d);
+  const uint32_t ring = smem_u32(c.ring), sfs = smem_u32(c.scr);
+  const uint32_t tb = c.S->tmem_base;
+  const int q = (threadIdx.x >> 5) & 3, th = cw >> 2; /* TMEM lane quadrant, token half of the epilogue */
+  bool ok = true;
+  int j = 0;
+  for (int item = x.a; item < x.b; ++item) {
+    const int unit = item / x.ngroups, grp = item % x.ngroups, db = (item - x.a) & 1;
+    const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+    for (int kc = 0; kc < x.nkc; ++kc, ++j) {
+      const int s = j % x.ns, buf = j & (NSF - 1);
+      const uint32_t slot = ring + (uint32_t)s * x.slot_bytes, stg = sfs + (uint32_t)buf * SF_STAGE;
+      if (ok && !wait_bar(c, &c.S->xfull[s], (xpar >> s) & 1u, layer, PH_GU)) ok = false;
+      xpar ^= 1u << s;
+      /* the scale copies last issued from this staging buffer must be done */
+      if (ok && ((xpar >> (8 + buf)) & 1u) &&
+          !wait_bar(c, &c.S->sfdone[buf], ((xpar >> (4 + buf)) & 1u) ^ 1u, layer, PH_GU))
+        ok = false;
+      if (!ok) continue;
+      /* this warp's share: SFA block (m, k step st), 16-byte row r0 = rows
+       * r0 + 32 m1 (m1 = 0..3), 4 scales each */
+      for (int u = cw * 32 + lane; u < 2 * nsteps * 32; u += NCT) {
+        const int blk = u / 32, r0 = u % 32;
+        const int m = blk / nsteps, st = blk % nsteps;
+        const uint32_t src = slot + GU_AS + m * (XROWS * GU_KC / 16) + 4 * st;
+        uint32_t wv[4];
+#pragma unroll
+        for (int m1 = 0; m1 < 4; ++m1) wv[m1] = lds32(src + (r0 + 32 * m1) * (GU_KC / 16));
+        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + (m * 4 + st) * 512 + r0 * 16), "r"(wv[0]),
+                     "r"(wv[1]), "r"(wv[2]), "r"(wv[3]));
+      }
+      fence_proxy_async_shared();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.S->sfready[buf]);
+      xpar ^= 1u << (4 + buf);
+      xpar |= 1u << (8 + buf);
+    }
+    const uint32_t dp = (xpar >> (12 + db)) & 1u;
+    xpar ^= 1u << (12 + db);
+    if (ok && !wait_bar(c, &c.S->dfull2[db], dp, layer, PH_GU)) ok = false;
+    if (!ok) continue;
+    tc_fence_after();
+    uint32_t gr[32], ur[32];
+    const uint32_t dcol = tb + TM_D + db * 128 + ((uint32_t)(q * 32) << 16) + th * 32;
+    tc_ld32(dcol, gr);
+    tc_ld32(dcol + TM_DU, ur);
+    tc_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c.S->dempty2[db]); /* the buffer may take the item after next */
+    const int row = grp * XROWS + q * 32 + lane;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int tt = th * 4 + t;
+      if (tt < n) {
+        const int pair = R.pairs[st0 + tt];
+        const float fi = *reinterpret_cast<const float*>(P->xq + (size_t)(pair / P->k) * xqb + xqb - 16);
+        float gsum = 0.f, usum = 0.f;
+#pragma unroll
+        for (int jt = 7; jt >= 0; --jt) { /* term jt weighs 4^-jt; smallest first */
+          gsum = gsum * 0.25f + __uint_as_float(gr[8 * t + jt]);
+          usum = usum * 0.25f + __uint_as_float(ur[8 * t + jt]);
+        }
+        const float gv = gsum * fi * gs0, uv = usum * fi * gs1;
+        P->u[(size_t)pair * f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
+      }
+    }
+  }
+  if (!ok) c.S->abort = 1;
+  /* one answer for every warp, even if the abort word changes meanwhile */
+  return !named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
+}
+
+/* Gate/up (GU) or down projection of the selected experts on the CUDA-core
+ * tensor path (mma.sync, weights decoded in registers): this CTA's items,
+ * 16 rows per warp, weight chunks and the unit's activation rows from the
+ * producer's ring.  After a chunk every warp meets at a CTA barrier and
+ * one thread releases the slot.  xpar bit s is the parity of weight slot
+ * s's uses. */
 template <bool GU>
-MSK_DEV bool expert_phase(Ctx& c, int layer, uint32_t& xpar) {
+MSK_DEV bool expert_mma(Ctx& c, int layer, uint32_t& xpar) {
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
   const Route& R = c.S->route;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
+  const int ctid = threadIdx.x - CONS0;
   const int phase = GU ? PH_GU : PH_DN;
   XGeo x;
   xgeo(c, GU, x);
   const int d = P->d, f = P->f;
   const float gs0 = GU ? Ly.wg.gs : Ly.wd.gs, gs1 = Ly.wu.gs;
-  uint16_t* uout = P->u;
-  float* yout = P->y;
   const uint32_t ring = smem_u32(c.ring);
   float acc[2][4], acc2[2][4];
   int j = 0;
   bool ok = true;
-  for (int item = x.a; item < x.b && ok; ++item) {
+  for (int item = x.a; item < x.b; ++item) {
     const int unit = item / x.ngroups, grp = item % x.ngroups;
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = acc2[0][e] = acc2[1][e] = 0.f;
     for (int kc = 0; kc < x.nkc; ++kc, ++j) {
       const int s = j % x.ns;
-      if (!wait_bar(c, &c.S->xfull[s], (xpar >> s) & 1u, layer, phase)) { ok = false; break; }
+      if (ok && !wait_bar(c, &c.S->xfull[s], (xpar >> s) & 1u, layer, phase)) ok = false;
       xpar ^= 1u << s;
       const uint32_t slot = ring + (uint32_t)s * x.slot_bytes;
-      xgemm<GU ? 2 : 1>(slot + cw * 16 * x.cpitch, slot + XROWS * x.cpitch + cw * 16 * x.spitch, x.mat_bytes,
-                        x.cpitch, x.spitch, slot + x.b_off, x.bpitch, x.KC, acc, acc2);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&c.S->xempty[s]);
+      if (ok)
+        xgemm<GU ? 2 : 1>(slot + cw * 16 * x.cpitch, slot + XROWS * x.cpitch + cw * 16 * x.spitch, x.mat_bytes,
+                          x.cpitch, x.spitch, slot + x.b_off, x.bpitch, x.KC, acc, acc2);
+      named_sync(BAR_CONS, NCT);
+      if (ok && ctid == 0) mbar_arrive(&c.S->xempty[s]);
     }
-    if (!ok) break;
+    if (!ok) continue;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -1440,16 +1752,16 @@ MSK_DEV bool expert_phase(Ctx& c, int layer, uint32_t& xpar) {
         const int pair = R.pairs[st0 + col];
         if (GU) {
           const float gv = (acc[0][e] + acc2[0][e]) * gs0, uv = (acc[1][e] + acc2[1][e]) * gs1;
-          uout[(size_t)pair * f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
+          P->u[(size_t)pair * f + row] = f32_to_f16(gv / (1.0f + expf(-gv)) * uv);
         } else {
-          yout[(size_t)pair * d + row] = (acc[0][e] + acc2[0][e]) * gs0;
+          P->y[(size_t)pair * d + row] = (acc[0][e] + acc2[0][e]) * gs0;
         }
       }
     }
   }
   if (!ok) c.S->abort = 1;
-  named_sync(BAR_CONS, NCT);
-  return !c.S->abort;
+  /* one answer for every warp, even if the abort word changes meanwhile */
+  return !named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
 }
 
 /* ---- consumer main loop ---------------------------------------------------------------- */
@@ -1481,10 +1793,10 @@ MSK_DEV void consumer(Ctx& c) {
     phase_router(c, l);
     if (!grid_sync(c, l, PH_ROUTER)) return;
     phase_topk(c, l);
-    if (!expert_phase<true>(c, l, xpar)) return;
+    if (!(tc_experts(P) ? expert_gu_tc(c, l, xpar) : expert_mma<true>(c, l, xpar))) return;
     if (!grid_sync(c, l, PH_GU)) return;
     if (threadIdx.x == CONS0) c.S->dn_ready = l + 1;
-    if (!expert_phase<false>(c, l, xpar)) return;
+    if (!expert_mma<false>(c, l, xpar)) return;
     named_sync(BAR_CONS, NCT);
     if (threadIdx.x == CONS0) c.S->ring_free = l + 1;
     if (!grid_sync(c, l, PH_DN)) return;
@@ -1529,8 +1841,18 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     mbar_init(&c.S->bfull, 1);
     for (int i = 0; i < XNS_MAX; ++i) {
       mbar_init(&c.S->xfull[i], 1);
-      mbar_init(&c.S->xempty[i], NCW);
+      mbar_init(&c.S->xempty[i], 1);
     }
+    for (int i = 0; i < NSF; ++i) {
+      mbar_init(&c.S->sfdone[i], 1);
+      mbar_init(&c.S->sfready[i], NCW);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c.S->dfull2[i], 1);
+      mbar_init(&c.S->dempty2[i], NCW);
+    }
+    mbar_init(&c.S->tfin, 1);
+    c.S->issuer_done = 0;
     mbar_fence_init();
   }
   /* positions: contiguous per sequence, inside the cache */
@@ -1555,9 +1877,30 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
   if (threadIdx.x < CONS0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
     if (threadIdx.x < 32) producer(c);
+    else if (threadIdx.x < 64) issuer(c);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_CONSUMER));
+    const bool w0 = (threadIdx.x >> 5) == CONS_WARP0;
+    /* the whole TMEM of the SM (one CTA per SM): gate/up accumulators and
+     * scale factors of the block-scaled expert MMAs */
+    if (w0) tmem_alloc(&c.S->tmem_base, TM_COLS);
+    tc_fence_before();
+    named_sync(BAR_CONS, NCT);
+    tc_fence_after();
     consumer<HD>(c);
+    /* every consumer warp leaves the step at the same barrier; wait for the
+     * tensor-core work issued so far (bounded), then free the TMEM */
+    named_sync(BAR_CONS, NCT);
+    if (threadIdx.x == CONS0) {
+      const uint64_t t0 = gtimer();
+      while (!c.S->issuer_done && gtimer() - t0 < 2 * (uint64_t)P->timeout_ns) __nanosleep(64);
+      while (!mbar_try(&c.S->tfin, 0) && gtimer() - t0 < 4 * (uint64_t)P->timeout_ns) {
+      }
+    }
+    tc_fence_before();
+    named_sync(BAR_CONS, NCT);
+    tc_fence_after();
+    if (w0) tmem_dealloc(c.S->tmem_base, TM_COLS);
   }
 }
 
