@@ -69,6 +69,13 @@ constexpr int XROWS = 16 * MSK_NCW;
 constexpr int XKC_MAX = 512;
 constexpr int XNS_MAX = 4;
 
+struct AttGeo {
+  int npairs;
+  int nparts; /* CTAs that take part: each gets >= 2 stages of keys when possible */
+  int64_t N;
+  int64_t lo[MSK_MAX_PAIRS];  /* first key position of the pair */
+  int64_t off[MSK_MAX_PAIRS + 1]; /* prefix sums of key counts */
+};
 struct Smem {
   uint64_t full[MSK_NST];
   uint64_t empty[MSK_NST];
@@ -81,6 +88,7 @@ struct Smem {
   uint64_t dempty2[2];      /* accumulator buffer 0/1 read by every consumer warp */
   uint64_t tfin;            /* every tensor-core op issued complete */
   uint32_t tmem_base;
+  AttGeo ag;                /* this layer's attention key split (consumers) */
   uint4 sfb_one[32];        /* 128 rows x 4 ue4m3 scales of 1.0, the activation terms' scales */
   volatile int issuer_done; /* the MMA-issuing warp has committed its last work */
   uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
@@ -285,13 +293,6 @@ MSK_DEV void dense_mat(const MskParams* P, const MskLayer& Ly, bool qkv, int row
 
 /* attention key space of one layer: pairs (seq, kv head) in order, each
  * with the union of its rows' key ranges; CTA c owns [c N / n, (c+1) N / n) */
-struct AttGeo {
-  int npairs;
-  int nparts; /* CTAs that take part: each gets >= 2 stages of keys when possible */
-  int64_t N;
-  int64_t lo[MSK_MAX_PAIRS];  /* first key position of the pair */
-  int64_t off[MSK_MAX_PAIRS + 1]; /* prefix sums of key counts */
-};
 MSK_DEV void att_geo(const Ctx& c, int layer, AttGeo& g) {
   const MskParams* P = c.P;
   g.npairs = c.st.S * P->hkv;
@@ -309,6 +310,49 @@ MSK_DEV void att_geo(const Ctx& c, int layer, AttGeo& g) {
   const int64_t C = P->hd == 128 ? 128 : 256;
   int64_t parts = (g.N + 2 * C - 1) / (2 * C);
   g.nparts = (int)(parts < 1 ? 1 : (parts > c.ncta ? c.ncta : parts));
+}
+/* the same geometry, computed once per layer by consumer warp 0 into
+ * shared memory (per-thread copies of the arrays would live in local
+ * memory); every consumer warp passes the barrier */
+MSK_DEV void att_geo_shared(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  if (cw == 0) {
+    AttGeo& g = c.S->ag;
+    const int npairs = c.st.S * P->hkv;
+    const bool sliding = P->layers[layer].sliding != 0;
+    int64_t run = 0;
+    for (int base = 0; base < npairs; base += 32) {
+      const int p = base + lane;
+      int64_t lo = 0, cnt = 0;
+      if (p < npairs) {
+        const int b = p / P->hkv;
+        const int64_t first = c.S->pos0[b], last = first + c.st.Tq - 1;
+        if (sliding) { lo = first - P->W + 1; if (lo < 0) lo = 0; }
+        cnt = last - lo + 1;
+      }
+      int64_t x = cnt; /* inclusive scan over the lanes */
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (p < npairs) {
+        g.lo[p] = lo;
+        g.off[p + 1] = run + x;
+      }
+      run += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) {
+      g.npairs = npairs;
+      g.off[0] = 0;
+      g.N = run;
+      const int64_t C = P->hd == 128 ? 128 : 256;
+      const int64_t parts = (run + 2 * C - 1) / (2 * C);
+      g.nparts = (int)(parts < 1 ? 1 : (parts > c.ncta ? c.ncta : parts));
+    }
+  }
+  named_sync(BAR_CONS, NCT);
 }
 MSK_DEV int att_owner(const AttGeo& g, int64_t x) {
   return (int)(((x + 1) * (int64_t)g.nparts - 1) / g.N);
@@ -1073,8 +1117,8 @@ MSK_DEV bool attention_phase_mt(Cons& q, int layer) {
   Ctx& c = *q.c;
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
-  AttGeo g;
-  att_geo(c, layer, g);
+  att_geo_shared(c, layer);
+  const AttGeo& g = c.S->ag;
   const int R = c.st.Tq * P->G;
   const int mt = (R + 15) / 16;
   const int ngroups = (mt + MT - 1) / MT; /* 1 or 2 */
@@ -1298,8 +1342,8 @@ MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
 MSK_DEV void phase_attc(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const int lane = threadIdx.x & 31, hd = P->hd, per = hd / 32;
-  AttGeo g;
-  att_geo(c, layer, g);
+  const AttGeo& g = c.S->ag; /* set by this layer's attention phase */
+  (void)layer;
   for (int item = gwarp(c); item < c.st.T * P->hq; item += nwarps(c)) {
     const int t = item / P->hq, h = item % P->hq;
     const int b = t / c.st.Tq, ti = t % c.st.Tq;
