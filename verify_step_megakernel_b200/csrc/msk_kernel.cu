@@ -89,6 +89,7 @@ struct Smem {
   uint64_t tfin;            /* every tensor-core op issued complete */
   uint32_t tmem_base;
   AttGeo ag;                /* this layer's attention key split (consumers) */
+  AttGeo agp;               /* the producer warp's copy */
   uint4 sfb_one[32];        /* 128 rows x 4 ue4m3 scales of 1.0, the activation terms' scales */
   volatile int issuer_done; /* the MMA-issuing warp has committed its last work */
   uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
@@ -293,32 +294,14 @@ MSK_DEV void dense_mat(const MskParams* P, const MskLayer& Ly, bool qkv, int row
 
 /* attention key space of one layer: pairs (seq, kv head) in order, each
  * with the union of its rows' key ranges; CTA c owns [c N / n, (c+1) N / n) */
-MSK_DEV void att_geo(const Ctx& c, int layer, AttGeo& g) {
+/* the same geometry computed by one warp into shared memory (per-thread
+ * copies of the arrays would live in local memory): att_geo_shared for the
+ * consumers (warp 0 computes, every consumer warp passes the barrier); the
+ * producer warp keeps its own copy, as it runs ahead of them */
+MSK_DEV void att_geo_warp(const Ctx& c, int layer, AttGeo& g) {
   const MskParams* P = c.P;
-  g.npairs = c.st.S * P->hkv;
-  g.off[0] = 0;
-  for (int p = 0; p < g.npairs; ++p) {
-    int b = p / P->hkv;
-    int64_t first = c.S->pos0[b];
-    int64_t last = first + c.st.Tq - 1;
-    int64_t lo = 0;
-    if (P->layers[layer].sliding) { lo = first - P->W + 1; if (lo < 0) lo = 0; }
-    g.lo[p] = lo;
-    g.off[p + 1] = g.off[p] + (last - lo + 1);
-  }
-  g.N = g.off[g.npairs];
-  const int64_t C = P->hd == 128 ? 128 : 256;
-  int64_t parts = (g.N + 2 * C - 1) / (2 * C);
-  g.nparts = (int)(parts < 1 ? 1 : (parts > c.ncta ? c.ncta : parts));
-}
-/* the same geometry, computed once per layer by consumer warp 0 into
- * shared memory (per-thread copies of the arrays would live in local
- * memory); every consumer warp passes the barrier */
-MSK_DEV void att_geo_shared(const Ctx& c, int layer) {
-  const MskParams* P = c.P;
-  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
-  if (cw == 0) {
-    AttGeo& g = c.S->ag;
+  const int lane = threadIdx.x & 31;
+  {
     const int npairs = c.st.S * P->hkv;
     const bool sliding = P->layers[layer].sliding != 0;
     int64_t run = 0;
@@ -352,6 +335,10 @@ MSK_DEV void att_geo_shared(const Ctx& c, int layer) {
       g.nparts = (int)(parts < 1 ? 1 : (parts > c.ncta ? c.ncta : parts));
     }
   }
+  __syncwarp();
+}
+MSK_DEV void att_geo_shared(const Ctx& c, int layer) {
+  if ((threadIdx.x >> 5) == CONS_WARP0) att_geo_warp(c, layer, c.S->ag);
   named_sync(BAR_CONS, NCT);
 }
 MSK_DEV int att_owner(const AttGeo& g, int64_t x) {
@@ -381,7 +368,6 @@ MSK_DEV void for_each_att_stage(const Ctx& c, const AttGeo& g, F&& f) {
 struct Prod {
   Ctx* c;
   uint32_t it;
-  uint32_t last_parity_for_slot[MSK_NST];
   uint32_t xpar;  /* bit s: parity of the fills of expert slot s so far */
   uint32_t xused; /* bit s: expert slot s filled at least once */
   uint32_t dpar;  /* bit 2w+s: parity of the fills of warp w's dense slot s */
@@ -403,7 +389,6 @@ MSK_DEV bool prod_acquire(Prod& p, int layer, int phase, uint8_t** stg, uint64_t
   if (round > 0 && !pwait_bar(c, &c.S->empty[slot], (round - 1) & 1, layer, phase)) return false;
   *stg = c.ring + (size_t)slot * MSK_STAGE;
   *bar = &c.S->full[slot];
-  p.last_parity_for_slot[slot] = round & 1;
   p.it++;
   return true;
 }
@@ -666,8 +651,8 @@ MSK_DEV void producer(Ctx& c) {
      * past keys stream at once, chunks holding this step's keys wait until
      * every CTA has written them */
     if (!pwait_flag(c, &c.S->dense_done, 2 * l + 1, l, PH_ATT)) { p.ok = false; break; }
-    AttGeo g;
-    att_geo(c, l, g);
+    att_geo_warp(c, l, c.S->agp);
+    const AttGeo& g = c.S->agp;
     for_each_att_stage(c, g, [&](int pr, int slot, int64_t k0, int n, bool, bool) {
       int b = pr / P->hkv, h = pr % P->hkv;
       if (k0 + C > c.S->pos0[b]) {
