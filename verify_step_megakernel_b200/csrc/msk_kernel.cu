@@ -82,6 +82,7 @@ struct Smem {
   uint64_t dfull[MSK_NCW][2];  /* dense weight slot of a warp landed */
   uint64_t dempty[MSK_NCW][2]; /* dense weight slot read by its warp */
   uint64_t bfull;              /* dense activation slice landed */
+  uint64_t rfull;              /* the step's router logits landed (top-k) */
   uint64_t sfdone[4];       /* tensor-core ops up to the last chunk using scale staging b done */
   uint64_t sfready[4];      /* scale staging b written by every consumer warp */
   uint64_t dfull2[2];       /* accumulator buffer 0/1 holds a finished item */
@@ -1424,49 +1425,79 @@ MSK_DEV void phase_router(const Ctx& c, int layer) {
   }
 }
 
+static_assert(MSK_MAX_TOKENS * 256 * 4 <= MSK_NST * MSK_STAGE, "top-k copies every logit into the stage ring");
+
+/* order-preserving map of a non-NaN float to u32, -0 taken as +0 */
+MSK_DEV uint32_t ord_key(float x) {
+  const uint32_t b = x == 0.f ? 0u : __float_as_uint(x);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+MSK_DEV float ord_val(uint32_t k) { return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k); }
+
 /* top-k of every token (value desc, index asc), softmax weights, and the
  * expert work list grouped by expert; every CTA computes the same lists */
-MSK_DEV void phase_topk(Ctx& c, int layer) {
+MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
   const MskParams* P = c.P;
   Route& R = c.S->route;
   const int lane = threadIdx.x & 31, cw = (threadIdx.x >> 5) - CONS_WARP0;
-  const int E = P->E, k = P->k, per = E / 32;
+  const int E = P->E, k = P->k, per = E / 32, ctid = threadIdx.x - CONS0;
+  /* every token's logits into the (idle) stage ring by one bulk copy */
+  const float* lg = reinterpret_cast<const float*>(c.ring);
+  {
+    const uint32_t par = (dpar >> 9) & 1u, bytes = (uint32_t)(c.st.T * E * 4);
+    dpar ^= 1u << 9;
+    fence_proxy_async_shared();
+    if (ctid == 0) mbar_arrive_tx(&c.S->rfull, bytes);
+    named_sync(BAR_CONS, NCT);
+    if (ctid == 0) {
+      fence_proxy_async_global();
+      bulk_g2s(c.ring, P->logits, bytes, &c.S->rfull);
+    }
+    if (!wait_bar(c, &c.S->rfull, par, layer, PH_TOPK)) {
+      if (ctid == 0) { /* the copy must land before the CTA may exit */
+        const uint64_t t0 = gtimer();
+        while (!mbar_try(&c.S->rfull, par) && gtimer() - t0 < 2 * (uint64_t)P->timeout_ns) {
+        }
+      }
+      c.S->abort = 1;
+    }
+    if (named_sync_or(BAR_CONS, NCT, c.S->abort != 0)) return false;
+  }
   for (int t = cw; t < c.st.T; t += NCW) {
-    float v[8];
+    uint32_t key[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const float x = i < per ? P->logits[(size_t)t * E + lane * per + i] : -INFINITY;
-      v[i] = x == x ? x : -INFINITY; /* a NaN logit ranks last */
+      key[i] = 0u; /* below every real key: never picked while k <= E */
+      if (i < per) {
+        const float x = lg[(size_t)t * E + lane * per + i];
+        key[i] = ord_key(x == x ? x : -INFINITY); /* a NaN logit ranks last */
+      }
     }
     uint32_t taken = 0;
-    float sel[8];
-    float vmax = 0.f;
+#pragma unroll 1
     for (int s = 0; s < k; ++s) {
-      float bv = -INFINITY;
-      int bi = 0x7FFFFFFF;
+      /* this lane's best untaken logit (equal keys: lower index), then the
+       * warp's largest key and, among lanes holding it, the lowest index */
+      uint32_t bk = 0;
+      int bi = 0;
 #pragma unroll
       for (int i = 0; i < 8; ++i)
-        /* ties (-inf included) go to the lower index, so every pick is a
-         * valid expert even when all remaining logits are -inf */
-        if (i < per && !(taken >> i & 1) && (v[i] > bv || (v[i] == bv && lane * per + i < bi))) {
-          bv = v[i];
-          bi = lane * per + i;
-        }
-#pragma unroll
-      for (int o = 16; o; o >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+        if (!((taken >> i) & 1u) && key[i] > bk) { bk = key[i]; bi = i; }
+      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t cand = bk == wk ? (uint32_t)(lane * per + bi) : 0xFFFFFFFFu;
+      const uint32_t wi = __reduce_min_sync(0xffffffffu, cand);
+      if (cand == wi) taken |= 1u << bi;
+      if (lane == 0) {
+        R.ids[t * k + s] = (int16_t)wi;
+        R.w[t * k + s] = ord_val(wk);
       }
-      if (bi / per == lane) taken |= 1u << (bi % per);
-      if (s == 0) vmax = bv;
-      sel[s] = bv;
-      if (lane == 0) R.ids[t * k + s] = (int16_t)bi;
     }
-    if (lane == 0) {
+    if (lane == 0) { /* softmax of the k picks (the first is the largest) */
+      float* w = R.w + t * k;
+      const float vmax = w[0];
       float sum = 0.f;
-      for (int s = 0; s < k; ++s) { sel[s] = expf(sel[s] - vmax); sum += sel[s]; }
-      for (int s = 0; s < k; ++s) R.w[t * k + s] = sel[s] / sum;
+      for (int s = 0; s < k; ++s) { w[s] = expf(w[s] - vmax); sum += w[s]; }
+      for (int s = 0; s < k; ++s) w[s] = w[s] / sum;
     }
   }
   named_sync(BAR_CONS, NCT);
@@ -1540,10 +1571,14 @@ MSK_DEV void phase_topk(Ctx& c, int layer) {
     if (P->dbg_logits)
       for (int i = ctid; i < c.st.T * E; i += NCT) P->dbg_logits[(size_t)layer * c.st.T * E + i] = P->logits[i];
   }
+  /* the ring's next writer is the copy engine (the expert tiles) */
+  fence_proxy_async_shared();
+  named_sync(BAR_CONS, NCT);
   if (threadIdx.x == CONS0) {
     __threadfence_block();
     c.S->route_ready = layer + 1;
   }
+  return true;
 }
 
 /* h += sum_slot w * y (slot order); then the next layer's attention norm, or
@@ -1821,7 +1856,7 @@ MSK_DEV void consumer(Ctx& c) {
     if (!grid_sync(c, l, PH_MOENORM)) return;
     phase_router(c, l);
     if (!grid_sync(c, l, PH_ROUTER)) return;
-    phase_topk(c, l);
+    if (!phase_topk(c, l, dpar)) return;
     if (!(tc_experts(P) ? expert_gu_tc(c, l, xpar) : expert_mma<true>(c, l, xpar))) return;
     if (!grid_sync(c, l, PH_GU)) return;
     if (threadIdx.x == CONS0) c.S->dn_ready = l + 1;
@@ -1868,6 +1903,7 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
         mbar_init(&c.S->dempty[w][i], 1);
       }
     mbar_init(&c.S->bfull, 1);
+    mbar_init(&c.S->rfull, 1);
     for (int i = 0; i < XNS_MAX; ++i) {
       mbar_init(&c.S->xfull[i], 1);
       mbar_init(&c.S->xempty[i], 1);
