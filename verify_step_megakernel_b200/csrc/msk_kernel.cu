@@ -1463,37 +1463,56 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
     }
     if (named_sync_or(BAR_CONS, NCT, c.S->abort != 0)) return false;
   }
-  for (int t = cw; t < c.st.T; t += NCW) {
-    uint32_t key[8];
+  /* four tokens per warp at a time (t = t0 + 8 q), their picks interleaved */
+  constexpr int TQ = 4;
+  for (int t0 = cw; t0 < c.st.T; t0 += TQ * NCW) {
+    uint32_t key[TQ][8], taken[TQ];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      key[i] = 0u; /* below every real key: never picked while k <= E */
-      if (i < per) {
-        const float x = lg[(size_t)t * E + lane * per + i];
-        key[i] = ord_key(x == x ? x : -INFINITY); /* a NaN logit ranks last */
+    for (int q = 0; q < TQ; ++q) {
+      const int t = t0 + q * NCW;
+      taken[q] = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        key[q][i] = 0u; /* below every real key: never picked while k <= E */
+        if (t < c.st.T && i < per) {
+          const float x = lg[(size_t)t * E + lane * per + i];
+          key[q][i] = ord_key(x == x ? x : -INFINITY); /* a NaN logit ranks last */
+        }
       }
     }
-    uint32_t taken = 0;
 #pragma unroll 1
     for (int s = 0; s < k; ++s) {
-      /* this lane's best untaken logit (equal keys: lower index), then the
-       * warp's largest key and, among lanes holding it, the lowest index */
-      uint32_t bk = 0;
-      int bi = 0;
+      /* per token: this lane's best untaken logit (equal keys: lower index),
+       * then the warp's largest key and, among lanes holding it, the lowest
+       * index */
+      uint32_t bk[TQ], wk[TQ], cand[TQ];
+      int bi[TQ];
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (!((taken >> i) & 1u) && key[i] > bk) { bk = key[i]; bi = i; }
-      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
-      const uint32_t cand = bk == wk ? (uint32_t)(lane * per + bi) : 0xFFFFFFFFu;
-      const uint32_t wi = __reduce_min_sync(0xffffffffu, cand);
-      if (cand == wi) taken |= 1u << bi;
-      if (lane == 0) {
-        R.ids[t * k + s] = (int16_t)wi;
-        R.w[t * k + s] = ord_val(wk);
+      for (int q = 0; q < TQ; ++q) {
+        bk[q] = 0;
+        bi[q] = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          if (!((taken[q] >> i) & 1u) && key[q][i] > bk[q]) { bk[q] = key[q][i]; bi[q] = i; }
+      }
+#pragma unroll
+      for (int q = 0; q < TQ; ++q) wk[q] = __reduce_max_sync(0xffffffffu, bk[q]);
+#pragma unroll
+      for (int q = 0; q < TQ; ++q) cand[q] = bk[q] == wk[q] ? (uint32_t)(lane * per + bi[q]) : 0xFFFFFFFFu;
+#pragma unroll
+      for (int q = 0; q < TQ; ++q) {
+        const uint32_t wi = __reduce_min_sync(0xffffffffu, cand[q]);
+        if (cand[q] == wi) taken[q] |= 1u << bi[q];
+        const int t = t0 + q * NCW;
+        if (lane == 0 && t < c.st.T) {
+          R.ids[t * k + s] = (int16_t)wi;
+          R.w[t * k + s] = ord_val(wk[q]);
+        }
       }
     }
-    if (lane == 0) { /* softmax of the k picks (the first is the largest) */
-      float* w = R.w + t * k;
+    __syncwarp(); /* lane 0's picks, read by lanes 0 .. TQ-1 */
+    if (lane < TQ && t0 + lane * NCW < c.st.T) { /* softmax of a token's k picks (the first is the largest) */
+      float* w = R.w + (t0 + lane * NCW) * k;
       const float vmax = w[0];
       float sum = 0.f;
       for (int s = 0; s < k; ++s) { w[s] = expf(w[s] - vmax); sum += w[s]; }
