@@ -747,7 +747,7 @@ MSK_DEV void cons_release(Cons& q, uint32_t slot) {
  * slice.  Same lane layout as the expert tiles: lane (g, cq) owns the NVFP4
  * blocks 4 qb + cq, decodes them once and feeds every column tile.
  */
-template <int NT>
+template <int NT, bool FULL>
 MSK_DEV void dgemm(uint32_t codes, uint32_t scales, uint32_t cpitch, uint32_t spitch, uint32_t bsm, uint32_t bpitch,
                    int KS, int ntl, float (*acc)[4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
@@ -776,7 +776,7 @@ MSK_DEV void dgemm(uint32_t codes, uint32_t scales, uint32_t cpitch, uint32_t sp
     }
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt) {
-      if (nt < ntl) {
+      if (FULL || nt < ntl) {
         const uint32_t bt = b + nt * 8 * bpitch + 128 * qb;
         const uint4 b0 = lds128(bt), b1 = lds128(bt + 16);
         mma_f16(acc[nt], a[0], b0.x, b0.y);
@@ -836,7 +836,12 @@ MSK_DEV bool dense_phase(Ctx& c, int layer, uint32_t& dpar) {
 #pragma unroll
       for (int nt = 0; nt < MSK_NT_DENSE; ++nt) acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.f;
       const uint32_t slot = ring + DB_BYTES + (uint32_t)(cw * DNS + sl) * DSLOT;
-      dgemm<MSK_NT_DENSE>(slot, slot + 16 * G.cpitch, G.cpitch, G.spitch, ring, G.bpitch, G.KS, ntl, acc);
+      /* all n-tiles present: a copy without the per-tile guard, which the
+       * compiler can schedule across tiles */
+      if (ntl == MSK_NT_DENSE)
+        dgemm<MSK_NT_DENSE, true>(slot, slot + 16 * G.cpitch, G.cpitch, G.spitch, ring, G.bpitch, G.KS, ntl, acc);
+      else
+        dgemm<MSK_NT_DENSE, false>(slot, slot + 16 * G.cpitch, G.cpitch, G.spitch, ring, G.bpitch, G.KS, ntl, acc);
       __syncwarp();
       if (lane == 0) mbar_arrive(&c.S->dempty[cw][sl]);
       int map, lrow;
