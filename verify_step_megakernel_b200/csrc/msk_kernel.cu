@@ -992,12 +992,17 @@ MSK_DEV void att_stage(const Ctx& c, AttState<HD, MT>& A, const uint8_t* stg, in
 #pragma unroll
       for (int n2 = 0; n2 < 2; ++n2) {
         float p[4];
+        if (full) { /* the whole block inside every row's window: no per-score test */
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int kl = kb * 16 + n2 * 8 + 2 * cq + (e & 1);
-          const int kp = k0 + kl, hf = e >> 1;
-          const bool ok = full || (kl < nkeys && kp >= A.lo[m][hf] && kp <= A.hi[m][hf]);
-          p[e] = ok ? fast_exp2(sacc[m][n2][e] * scale_log2 - bound_log2) : 0.f;
+          for (int e = 0; e < 4; ++e) p[e] = fast_exp2(sacc[m][n2][e] * scale_log2 - bound_log2);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int kl = kb * 16 + n2 * 8 + 2 * cq + (e & 1);
+            const int kp = k0 + kl, hf = e >> 1;
+            const bool ok = kl < nkeys && kp >= A.lo[m][hf] && kp <= A.hi[m][hf];
+            p[e] = ok ? fast_exp2(sacc[m][n2][e] * scale_log2 - bound_log2) : 0.f;
+          }
         }
         A.l[m][0] += p[0] + p[1];
         A.l[m][1] += p[2] + p[3];
