@@ -1294,6 +1294,7 @@ MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
     /* the projection: its K slices' partials added in slice order */
     const int S = P->d <= DKS_MAX ? 1 : P->d / DKS_MAX;
     float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 4
     for (int sl = 0; sl < S; ++sl) {
       const float* raw = P->qkv + ((size_t)sl * c.st.T + t) * nqkv + hh * hd + lane * per;
       if (per == 4) {
@@ -1347,9 +1348,15 @@ MSK_DEV void phase_attc(const Ctx& c, int layer) {
     const int rho = ti * P->G + h % P->G;
     const int cf = att_owner(g, g.off[pair]), cl = att_owner(g, g.off[pair + 1] - 1);
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, l = 0.f;
+#pragma unroll 4
     for (int cc = cf; cc <= cl; ++cc) {
       const float* row = P->part + (size_t)(cc + pair) * P->part_stride + (size_t)rho * (hd + 4);
-      for (int i = 0; i < per; ++i) acc[i] += row[lane * per + i];
+      if (per == 4) {
+        const float4 q = *reinterpret_cast<const float4*>(row + lane * 4);
+        acc[0] += q.x; acc[1] += q.y; acc[2] += q.z; acc[3] += q.w;
+      } else {
+        for (int i = 0; i < per; ++i) acc[i] += row[lane * per + i];
+      }
       l += row[hd];
     }
     const float inv = 1.0f / l;
@@ -1378,6 +1385,7 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
         /* residual + W_o o, the projection's K slices added in order */
         float4* hp = reinterpret_cast<float4*>(P->h + (size_t)t * d + i);
         v[u] = *hp;
+#pragma unroll 4
         for (int s = 0; s < So; ++s) {
           const float4 q = *reinterpret_cast<const float4*>(P->qkv + ((size_t)s * c.st.T + t) * d + i);
           v[u].x += q.x; v[u].y += q.y; v[u].z += q.z; v[u].w += q.w;
@@ -1627,6 +1635,7 @@ MSK_DEV void phase_comb(const Ctx& c, int layer) {
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (i < (cw + 1) * sl) {
         float4 acc = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
+#pragma unroll 4
         for (int s = 0; s < k; ++s) {
           const float w = R.w[t * k + s];
           const float4 y = *reinterpret_cast<const float4*>(P->y + (size_t)(t * k + s) * d + i);
