@@ -324,6 +324,74 @@ def run_msk(args, w):
     return 0
 
 
+def run_sweep(args, w):
+    """Step time of the workload's model over a range of batch shapes (S
+    sequences x Tq draft tokens, S*Tq <= 64): one JSON line per shape, timed
+    like the main line (warm-up, CUDA events per step, L2 flushed when the
+    step's bytes would fit in it).  One handle serves all shapes with the
+    same token limit per sequence; Tq = 8 needs a second one (at most 8
+    sequences), built after the first is released."""
+    import torch
+
+    import synth.gpu as sg
+    import verify_step_megakernel_b200 as msk
+    from tests._gpu import Engine
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    groups = [(4, [(1, 1), (2, 1), (4, 1), (8, 1), (16, 1), (1, 4), (4, 4), (16, 4)]), (8, [(1, 8), (4, 8), (8, 8)])]
+    for tps, shapes in groups:
+        max_s = min(64 // tps, max(s for s, _ in shapes))
+        eng = Engine(w.with_(n_seqs=max_s, tokens_per_seq=tps), device=0)
+        eng.fill_past()
+        stream = torch.cuda.Stream(dev)
+        msk.msk_set_debug(eng.h)
+        for S, Tq in shapes:
+            ws = w.with_(n_seqs=S, tokens_per_seq=Tq)
+            hid = sg.hidden(ws, 0)
+            pos = torch.tensor(ws.positions(), dtype=torch.int32, device=dev)
+            out = torch.empty((ws.T, ws.d_model), dtype=torch.int16, device=dev)
+
+            def launch():
+                msk.msk_step(eng.h, hid.data_ptr(), pos.data_ptr(), S, Tq, eng.kv, out.data_ptr(),
+                             stream.cuda_stream)
+
+            for _ in range(args.warmup):
+                launch()
+            stream.synchronize()
+            if msk.msk_step_status(eng.h) != 0:
+                raise RuntimeError(f"sweep step {S}x{Tq} failed")
+            stats = msk.msk_query(eng.h)
+            nbytes = int(stats.algorithmic_bytes)
+            flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev) if nbytes < 4 * 126e6 else None
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(args.steps)]
+            torch.cuda.synchronize(dev)
+            with torch.cuda.stream(stream):
+                for i in range(args.steps):
+                    if flush is not None:
+                        flush.fill_(i & 0xFF)
+                    ev[i][0].record(stream)
+                    launch()
+                    ev[i][1].record(stream)
+            stream.synchronize()
+            if msk.msk_step_status(eng.h) != 0:
+                raise RuntimeError(f"sweep step {S}x{Tq} failed")
+            ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+            nd = list(stats.n_distinct[:w.n_layers])
+            print(json.dumps({"sweep": w.name, "n_seqs": S, "tokens_per_seq": Tq, "T": S * Tq,
+                              "step_us": round(ms * 1e3, 1), "tokens_per_s": round(S * Tq / (ms * 1e-3), 1),
+                              "algorithmic_bytes_per_step": nbytes, "hbm_gbs": round(nbytes / (ms * 1e-3) / 1e9, 1),
+                              "frac_of_measured": round(nbytes / (ms * 1e-3) / 1e9 / measured_peak()[0], 4),
+                              "distinct_experts_per_layer_mean": round(sum(nd) / len(nd), 1),
+                              "l2": "flushed" if flush is not None else "inputs larger than L2"}), flush=True)
+            del flush
+        eng.close()
+        del eng
+        torch.cuda.empty_cache()
+    return 0
+
+
 PHASES = ["in", "qkv", "qknorm", "attention", "attn_combine", "wo", "moe_norm", "router", "topk", "gate_up",
           "down", "combine"]
 
@@ -371,6 +439,8 @@ def main():
     ap.add_argument("--trace", action="store_true", help="print a per-phase device-time breakdown instead")
     ap.add_argument("--tc-experts", action="store_true",
                     help="gate/up on the block-scaled tensor cores (MSK_F_TC_EXPERTS) instead of the default path")
+    ap.add_argument("--sweep", action="store_true",
+                    help="step time of the workload's model over batch shapes (one JSON line per shape)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -378,6 +448,8 @@ def main():
     w = synth.WORKLOADS.get(args.workload) or synth.PROFILE_WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.sweep:
+        return run_sweep(args, w)
     return run_msk(args, w)
 
 
