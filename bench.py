@@ -172,6 +172,27 @@ def run_reference(args, w):
     return 0
 
 
+def max_over_ranks(value, device="cpu"):
+    """The largest of each rank's `value` (a float) over the default process
+    group; the value itself when there is no group or one rank.  Every rank
+    must call it, in the same order."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, units_per_rank, ms_max):
+    """Whole-job throughput: the units all ranks processed per second, over
+    the slowest rank's step time (replicas: each rank processes the same
+    units per step)."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
 def run_msk(args, w):
     import numpy as np
     import torch
@@ -252,10 +273,7 @@ def run_msk(args, w):
     per = [a.elapsed_time(b) for a, b in ev]
     ms = statistics.mean(per)
     total_ms = t0.elapsed_time(t1)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, dev)
 
     # end to end through the C ABI: pinned host input -> device, step, output -> host
     h_in_host = hid.cpu().pin_memory()
@@ -278,23 +296,20 @@ def run_msk(args, w):
         e1.record(stream)
     stream.synchronize()
     e2e_ms = e1.elapsed_time(e0) if False else e0.elapsed_time(e1)
-    e2e_t = torch.tensor([e2e_ms / args.steps], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(e2e_t, op=dist.ReduceOp.MAX)
-    e2e_step_ms = float(e2e_t.item())
+    e2e_step_ms = max_over_ranks(e2e_ms / args.steps, dev)
     if msk.msk_step_status(eng.h) != 0:
         raise RuntimeError("e2e step failed")
 
     peak, peak_kind = measured_peak()
     achieved = bytes_step / (ms * 1e-3) / 1e9  # this rank's kernel, GB/s
-    value = world * bytes_step / (ms_max * 1e-3) / 1e9
+    value = job_rate(world, bytes_step, ms_max) / 1e9
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms_max, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f16 x f16 -> fp32 (NVFP4/fp8 storage)", "data": "synthetic",
         "config": dict(workload_config(w), parallelism=f"{world} independent replicas", l2=l2_note),
         "step_us": round(ms_max * 1e3, 2),
-        "tokens_per_s": round(world * w.T / (ms_max * 1e-3), 1),
+        "tokens_per_s": round(job_rate(world, w.T, ms_max), 1),
         "hbm_gbs_per_gpu": round(achieved, 1),
         "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
         "step_over_stream_time": round((ms * 1e-3) / (bytes_step / (NOMINAL_HBM_GBS * 1e9)), 3),
@@ -303,7 +318,7 @@ def run_msk(args, w):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_kind": f"{peak_kind} copy bandwidth",
                      "traffic": ncu_traffic(w.name)},
-        "e2e": {"value": round(world * bytes_step / (e2e_step_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+        "e2e": {"value": round(job_rate(world, bytes_step, e2e_step_ms) / 1e9, 2), "unit": "GB/s",
                 "h2d_bytes_per_step": int(hid.numel() * 2 + pos.numel() * 4),
                 "d2h_bytes_per_step": int(out.numel() * 2), "ms_per_step": round(e2e_step_ms, 4)},
         "gpu_launches": world * args.steps,
