@@ -114,12 +114,14 @@ def gpu_kv_codes(eng, w, positions, seqs):
     return K, V
 
 
-def run_parity(w, eng, gpu_hidden, positions, seqs=None, threads=None, max_replays=4):
+def run_parity(w, eng, gpu_hidden, positions, seqs=None, threads=None, max_replays=4, src=None):
     """Oracle on sequences `seqs` (default all) of the step; returns (report,
     gpu outputs, oracle outputs).  Decisions with two valid answers (routing
     near-ties, fp8 codes at a rounding midpoint) are replayed in the oracle
     with the GPU's choice so the layers after them stay comparable; every
-    other difference counts against the tolerances."""
+    other difference counts against the tolerances.  src: the oracle's input
+    source (default the workload's generator; an array source where a test
+    changed the device weights)."""
     seqs = list(range(len(positions))) if seqs is None else seqs
     tps = len(positions[0])
     h_bits = gpu_hidden.cpu().numpy().view(np.uint16)
@@ -127,7 +129,7 @@ def run_parity(w, eng, gpu_hidden, positions, seqs=None, threads=None, max_repla
     assert gpu["status"] == 0, msk.STATUS.get(gpu["status"])
     rows = [b * tps + i for b in seqs for i in range(tps)]
     gk, gv = gpu_kv_codes(eng, w, positions, seqs)
-    src = synth.LazySource(w)
+    src = synth.LazySource(w) if src is None else src
     pos_s = [positions[b] for b in seqs]
     ww = w.with_(n_seqs=len(seqs))
     kw = dict(seq_ids=seqs, threads=threads)

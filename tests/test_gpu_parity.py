@@ -184,3 +184,46 @@ def test_parity_largest_sampled():
     _report("large", rep)
     assert_parity(rep)
     eng.close()
+
+
+def test_routing_exact_ties_break_by_lower_index():
+    # router rows equal in groups of three (row r = row 3 (r // 3)), so every
+    # token's logits come in exactly equal triples and the cut after the 8th
+    # pick falls inside a triple: only the tie rule (lower expert index
+    # first) decides which two of its three experts are taken.  The device
+    # router is overwritten in place (the handle borrows it); the oracle reads
+    # the same values from an array source.
+    from tests._models import ExtendableSource
+
+    w = synth.WORKLOADS["tiny"].with_(n_seqs=1, tokens_per_seq=1)
+    eng = Engine(w)
+    eng.fill_past()
+    src = ExtendableSource(w)
+    E, d = w.n_experts, w.d_model
+    for l in range(w.n_layers):
+        r = src.arrays["vec"][(l, "router")].reshape(E, d)
+        tied = np.ascontiguousarray(r[(np.arange(E) // 3) * 3].reshape(-1)).astype(np.float32)
+        src.arrays["vec"][(l, "router")] = tied
+        ptr = eng.wts.layers[l]["router"]
+        dev_t = next(t for t in eng.wts.keep if t.data_ptr() == ptr)
+        dev_t.copy_(torch.from_numpy(tied))
+    src.rebuild()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions(), src=src.src)
+    _report("ties", rep)
+    # the oracle's 8th-9th gap is exactly 0 here, so compare the picks
+    # themselves instead of exempting them
+    for l in range(w.n_layers):
+        assert ref["route_gap"][l, 0] == 0.0  # the 8th and 9th logits are equal
+        got = sorted(int(x) for x in gpu["route_ids"][l, 0])
+        assert got == sorted(int(x) for x in ref["route_ids"][l, 0]), (l, got, ref["route_ids"][l, 0])
+        # among the experts tied with the 8th logit, the lowest indices won
+        lg = gpu["logits"][l, 0]
+        v8 = min(lg[e] for e in got)
+        tied = sorted(int(e) for e in np.nonzero(lg == v8)[0])
+        taken = [e for e in got if lg[e] == v8]
+        assert len(tied) > len(taken) and taken == tied[:len(taken)], (l, tied, taken)
+    assert rep["forced"] == 0
+    assert rep["h_abs"] <= 2e-2 and rep["h_rel"] <= 1e-2, rep
+    assert max(rep["attn_rel"]) <= 5e-3
+    eng.close()
