@@ -227,3 +227,55 @@ def test_routing_exact_ties_break_by_lower_index():
     assert rep["h_abs"] <= 2e-2 and rep["h_rel"] <= 1e-2, rep
     assert max(rep["attn_rel"]) <= 5e-3
     eng.close()
+
+
+def _set_router(eng, w, fn):
+    """Overwrite every layer's device router [E][d] with fn(original)."""
+    E, d = w.n_experts, w.d_model
+    for l in range(w.n_layers):
+        ptr = eng.wts.layers[l]["router"]
+        dev_t = next(t for t in eng.wts.keep if t.data_ptr() == ptr)
+        r = dev_t.view(E, d).cpu().numpy()
+        dev_t.copy_(torch.from_numpy(np.ascontiguousarray(fn(r), dtype=np.float32).reshape(-1)))
+
+
+def test_routing_all_logits_equal_picks_the_first_k():
+    # one router row for every expert: all logits of a token are equal, so
+    # the picks are experts 0 .. k-1 with weights exactly 1/k
+    w = synth.WORKLOADS["tiny"].with_(n_seqs=2, tokens_per_seq=2)
+    eng = Engine(w)
+    eng.fill_past()
+    _set_router(eng, w, lambda r: np.repeat(r[:1], r.shape[0], axis=0))
+    out = eng.step(sg.hidden(w), w.positions())
+    assert out["status"] == 0
+    k = w.top_k
+    for l in range(w.n_layers):
+        for t in range(w.T):
+            assert sorted(int(x) for x in out["route_ids"][l, t]) == list(range(k))
+            assert np.all(out["route_w"][l, t] == np.float32(1.0 / k))
+    assert np.isfinite(bf16_to_f64(out["hidden_out"])).all()
+    eng.close()
+
+
+def test_routing_nan_logit_is_never_picked():
+    # a NaN router row makes that expert's logit NaN for every token; it
+    # ranks last, so it is never among the picks and nothing NaN reaches
+    # the hidden state
+    w = synth.WORKLOADS["tiny"].with_(n_seqs=2, tokens_per_seq=2)
+    eng = Engine(w)
+    eng.fill_past()
+    bad = 5
+
+    def poison(r):
+        r = r.copy()
+        r[bad] = np.nan
+        return r
+
+    _set_router(eng, w, poison)
+    out = eng.step(sg.hidden(w), w.positions())
+    assert out["status"] == 0
+    assert np.isnan(out["logits"][:, :, bad]).all()
+    assert not (out["route_ids"] == bad).any()
+    assert np.isfinite(out["route_w"]).all()
+    assert np.isfinite(bf16_to_f64(out["hidden_out"])).all()
+    eng.close()
