@@ -62,3 +62,28 @@ def test_status_strings_for_every_code():
         assert isinstance(s, str) and s, name
         seen.add(s)
     assert len(seen) == len(codes)  # one distinct message per code
+
+
+def test_null_handles_are_refused_without_device_work():
+    lib = ctypes.CDLL(_build.build())
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    lib.msk_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp]
+    lib.msk_step_static.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp]
+    lib.msk_kv_create.argtypes = [vp, i32, i64, vp]
+    lib.msk_kv_append.argtypes = [vp, vp, i32, i32, i64, i64, vp, vp, vp]
+    lib.msk_kv_read.argtypes = [vp, vp, i32, i32, i64, i64, vp, vp]
+    for f in ("msk_step_status", "msk_set_debug", "msk_query", "msk_destroy", "msk_kv_destroy"):
+        getattr(lib, f).argtypes = [vp] if f in ("msk_step_status", "msk_destroy", "msk_kv_destroy") else [vp, vp]
+    fake = 0x10000
+    out = ctypes.c_void_p()
+    assert lib.msk_create(None, None, 0, ctypes.byref(out)) == 1
+    assert lib.msk_step(None, fake, fake, 1, 1, fake, fake, None) == 1
+    assert lib.msk_step_static(None, fake, fake, 1, 1, fake, fake, None) == 1
+    assert lib.msk_kv_create(None, 1, 16, ctypes.byref(out)) == 1
+    assert lib.msk_kv_append(None, fake, 0, 0, 0, 1, fake, fake, None) == 1
+    assert lib.msk_kv_read(None, fake, 0, 0, 0, 1, fake, fake) == 1
+    assert lib.msk_step_status(None) == 1
+    assert lib.msk_set_debug(None, None) == 1
+    assert lib.msk_query(None, None) == 1
+    lib.msk_destroy(None)     # no-ops
+    lib.msk_kv_destroy(None)
