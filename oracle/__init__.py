@@ -49,6 +49,8 @@ def lib():
         L.msk_or_e4m3_decode.restype = C.c_double
         L.msk_or_e4m3_encode.argtypes = [C.c_double]
         L.msk_or_e4m3_encode.restype = C.c_int
+        L.msk_or_e4m3_encode_n.argtypes = [P, C.c_int64, P]
+        L.msk_or_e4m3_encode_n.restype = None
         L.msk_or_bf16_encode.argtypes = [C.c_double]
         L.msk_or_bf16_encode.restype = C.c_uint16
         L.msk_or_bf16_decode.argtypes = [C.c_uint16]
@@ -129,6 +131,14 @@ def attend(q, K, V, scale):
     lib().msk_or_attend(q.ctypes.data, K.ctypes.data, V.ctypes.data, K.shape[0], q.shape[0], scale,
                         o.ctypes.data, C.byref(smax))
     return o, smax.value
+
+
+def e4m3_encode(x):
+    """The oracle's fp8 e4m3 encoder (nearest even, saturating) over an array."""
+    x = np.ascontiguousarray(x, np.float64)
+    out = np.zeros(x.shape, np.uint8)
+    lib().msk_or_e4m3_encode_n(x.ctypes.data, x.size, out.ctypes.data)
+    return out
 
 
 def rmsnorm(x, g, eps):

@@ -72,18 +72,27 @@ static double round_sig(double x, int bits) {
   return ldexp(nearbyint(ldexp(m, bits)), e - bits);
 }
 
-/* fp64 -> e4m3fn code: nearest even, saturating to +-448. */
+/* fp64 -> e4m3fn code: nearest even, saturating to +-448.  The sign bit is
+ * the operand's (so -0 and negative values that round to zero give the
+ * signed zero S.0000.000 = 0x80, as IEEE rounding keeps the operand's sign);
+ * NaN gives the NaN code S.1111.111. */
 int msk_or_e4m3_encode(double x) {
   double a = fabs(x), r;
+  int base = signbit(x) ? 128 : 0;
+  if (isnan(x)) return base | 0x7F;
   if (a < ldexp(1.0, -6)) r = ldexp(nearbyint(ldexp(a, 9)), -9); /* subnormal spacing 2^-9 */
   else r = round_sig(a, 4);
   if (r > 448.0) r = 448.0;
-  int base = x < 0 ? 128 : 0;
   if (r == 0.0) return base;
   pthread_once(&g_tab_once, build_tables);
   for (int c = 1; c < 127; ++c)
     if (g_e4m3[c] == r) return base | c;
   return -1; /* unreachable */
+}
+
+/* msk_or_e4m3_encode over an array (codes of n values). */
+void msk_or_e4m3_encode_n(const double* x, int64_t n, uint8_t* codes) {
+  for (int64_t i = 0; i < n; ++i) codes[i] = (uint8_t)msk_or_e4m3_encode(x[i]);
 }
 
 /* fp64 -> bf16 bits: nearest even (finite, normal-range inputs). */

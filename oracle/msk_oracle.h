@@ -62,6 +62,7 @@ int msk_oracle_step(const msk_or_cfg* cfg, const msk_source* src, int n_seqs, in
 double msk_or_e2m1_decode(int nib);
 double msk_or_e4m3_decode(int code);
 int msk_or_e4m3_encode(double x);
+void msk_or_e4m3_encode_n(const double* x, int64_t n, uint8_t* codes);
 uint16_t msk_or_bf16_encode(double x);
 double msk_or_bf16_decode(uint16_t b);
 void msk_or_rmsnorm(const double* x, const float* g, int n, double eps, double* y);

@@ -80,6 +80,14 @@ def test_e4m3_encode_round_trip_and_saturation():
         assert L.msk_or_e4m3_encode(x) == 0x7E
         assert L.msk_or_e4m3_encode(-x) == 0xFE
     assert L.msk_or_e4m3_encode(0.0) == 0
+    # OFP8 E4M3 has a signed zero (S.0000.000) and one NaN pattern per sign
+    # (S.1111.111): -0 and negative values that round to zero keep the sign
+    # bit, NaN stays NaN, infinities saturate
+    assert L.msk_or_e4m3_encode(-0.0) == 0x80
+    assert L.msk_or_e4m3_encode(-2.0 ** -11) == 0x80
+    assert L.msk_or_e4m3_encode(float("nan")) & 0x7F == 0x7F
+    assert L.msk_or_e4m3_encode(float("inf")) == 0x7E
+    assert L.msk_or_e4m3_encode(float("-inf")) == 0xFE
 
 
 def test_e4m3_encode_ties_and_random_vs_brute_force():
@@ -106,9 +114,7 @@ def test_e4m3_encode_matches_torch_in_range():
     x = x[np.abs(x) < 440]
     ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     got = np.array([L.msk_or_e4m3_encode(float(v)) for v in x])
-    ref = np.where(ref == 128, 0, ref)  # -0 encodes as +0 here
-    got = np.where(got == 128, 0, got)
-    assert np.array_equal(got, ref)
+    assert np.array_equal(got, ref)  # signed zeros included
 
 
 def test_bf16_encode_matches_torch():
