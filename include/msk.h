@@ -121,13 +121,24 @@ typedef struct msk_kv msk_kv_t;
  * pointers, any may be NULL; T = n_seqs * tokens_per_seq of the step):
  *  route_ids [L][T][top_k] int16, route_w [L][T][top_k] fp32,
  *  logits [L][T][n_experts] fp32, attn_out [L][T][Hq*hd] fp32 (attention
- *  output before W_o), trace [L][16] uint64 %globaltimer stamps of CTA 0. */
+ *  output before W_o), trace [L][16] uint64 %globaltimer stamps of CTA 0,
+ *  k_pre, v_pre [L][T][Hkv*hd] fp32: this step's keys after QK-norm and
+ *  values, each exactly as the step holds it just before the fp8 e4m3
+ *  encoding that writes it into the cache.
+ * hold_barrier (a test hook of this library, not part of the method): when
+ * n > 0, CTA 0 withholds its arrival at the step's n-th grid barrier, so
+ * every CTA's wait there runs out after wait_timeout_us and the step ends
+ * with MSK_ERR_TIMEOUT (no trap, no fault: copies in flight land first and
+ * the kernel returns).  0 = off. */
 typedef struct msk_debug {
   int16_t* route_ids;
   float* route_w;
   float* logits;
   float* attn_out;
   uint64_t* trace;
+  float* k_pre;
+  float* v_pre;
+  int32_t hold_barrier;
 } msk_debug_t;
 
 typedef struct msk_stats {
@@ -162,6 +173,15 @@ void msk_kv_destroy(msk_kv_t* kv);
  * (e4m3 codes; 0x7F/0xFF NaN codes are not allowed).  Async on `stream`. */
 msk_status_t msk_kv_append(msk_handle_t* h, msk_kv_t* kv, int layer, int seq, int64_t pos0, int64_t n,
                            const uint8_t* k_fp8, const uint8_t* v_fp8, void* stream);
+
+/* Encode n fp32 values into fp8 e4m3 codes with the rounding the step uses
+ * when it writes this step's keys and values into the cache: round to
+ * nearest, ties to even, saturating to +-448 (the OFP8 "E4M3" format the
+ * post's fp8 KV cache stores; NaN stays NaN).  in: dev fp32 [n], out: dev
+ * uint8 [n]; both 16-byte aligned, on the current device.  For callers
+ * that build past K/V for msk_kv_append from wider values.  Async on
+ * `stream`. */
+msk_status_t msk_kv_encode(const float* in, uint8_t* out, int64_t n, void* stream);
 
 /* Read n positions back out of the cache into device or host arrays
  * laid out [n][n_kv_heads][head_dim]; synchronous. */
@@ -201,8 +221,10 @@ msk_status_t msk_step(msk_handle_t* h, const uint16_t* hidden_in, const int32_t*
  * into the library, shared by every handle on a device.  The call allocates
  * nothing: no cudaMalloc, no cudaFree, no allocating library routine.
  *  - First call on a device: looks the array's device address up
- *    (cudaGetSymbolAddress) with that device current, once; later calls
- *    reuse it.  Make that first call before any stream capture begins.
+ *    (cudaGetSymbolAddress) with that device current; later calls reuse it.
+ *    A lookup that fails is not remembered: the call returns MSK_ERR_CUDA
+ *    and the next call tries again.  Make the first call before any stream
+ *    capture begins.
  *  - Enqueues one small kernel that copies the handle's parameter block into
  *    the array and zeroes the barrier words (the only bytes that must start
  *    at zero), then the step kernel; no host synchronisation.
@@ -221,6 +243,15 @@ msk_status_t msk_step_static(msk_handle_t* h, const uint16_t* hidden_in, const i
 /* Device status of the steps since the last call (call after synchronising
  * the stream); clears it. */
 msk_status_t msk_step_status(msk_handle_t* h);
+
+/* msk_step_status, plus where the device recorded its first error: the
+ * layer, the phase (0 input norm, 1 QKV projection, 2 QK-norm and KV write,
+ * 3 attention, 4 attention combine, 5 W_o, 6 MoE norm, 7 router, 8 top-k,
+ * 9 gate/up, 10 down, 11 combine) and the CTA; all -1 when the status is
+ * MSK_OK or the error carries no site (positions refused before the layer
+ * loop).  Any out pointer may be NULL.  Clears the status like
+ * msk_step_status. */
+msk_status_t msk_step_status_at(msk_handle_t* h, int32_t* layer, int32_t* phase, int32_t* cta);
 
 /* Set (or, with NULL, clear) the capture buffers used by later steps. */
 msk_status_t msk_set_debug(msk_handle_t* h, const msk_debug_t* dbg);

@@ -61,6 +61,8 @@ def lib():
         L.sy_dev_init.restype = C.c_int
         L.sy_dev_fill_nvfp4.argtypes = [M, C.c_int, C.c_int, C.c_int, P, P, C.POINTER(C.c_float), P]
         L.sy_dev_fill_nvfp4.restype = C.c_int
+        L.sy_dev_fill_nvfp4_experts.argtypes = [M, C.c_int, C.c_int, C.c_int, P, P, P, C.POINTER(C.c_float), P]
+        L.sy_dev_fill_nvfp4_experts.restype = C.c_int
         L.sy_dev_fill_vec.argtypes = [M, C.c_int, C.c_int, P, P]
         L.sy_dev_fill_vec.restype = C.c_int
         L.sy_dev_fill_hidden.argtypes = [M, C.c_int, C.c_int, C.c_int, P, P, P]
@@ -201,6 +203,18 @@ def dev_nvfp4(w, role, layer, expert, codes_ptr, scales_ptr, stream=0):
                                  C.byref(gs), stream)
     if rc:
         raise RuntimeError(f"sy_dev_fill_nvfp4: {rc}")
+    return gs.value
+
+
+def dev_nvfp4_experts(w, role, layer, keys_ptr, codes_ptr, scales_ptr, stream=0):
+    """All n_experts tensors of an expert role in one launch; keys_ptr is
+    device scratch of n_experts uint64."""
+    gs = C.c_float()
+    m = model(w)
+    rc = lib().sy_dev_fill_nvfp4_experts(C.byref(m), ROLES[role], layer, w.n_experts, keys_ptr, codes_ptr,
+                                         scales_ptr, C.byref(gs), stream)
+    if rc:
+        raise RuntimeError(f"sy_dev_fill_nvfp4_experts: {rc}")
     return gs.value
 
 

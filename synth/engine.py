@@ -1,6 +1,8 @@
-"""GPU-side harness shared by the tests and bench.py: synthetic weights and
-KV on the device (synth.gpu), one msk handle and KV cache, and a step
-through the C ABI with the capture buffers set."""
+"""A synthetic workload on one GPU behind one msk handle: the seeded
+weights and past KV filled on the device (synth.gpu), the handle and KV
+cache created through the C ABI, and a step with the capture buffers set.
+Used by the GPU tests, bench.py and the smoke check; it holds none of the
+step's arithmetic (every step runs in libmsk.so's kernel)."""
 import numpy as np
 import torch
 
@@ -67,8 +69,10 @@ class Engine:
                     msk.msk_kv_append(self.h, self.kv, l, b, p0, n, kb.data_ptr(), vb.data_ptr(), stream)
         torch.cuda.synchronize(self.dev)
 
-    def step(self, hidden, positions, capture=True, stream=None):
-        """hidden: int16 [T][d] device tensor of bf16 bits; positions: int list [S][Tq]."""
+    def step(self, hidden, positions, capture=True, stream=None, hold_barrier=0):
+        """hidden: int16 [T][d] device tensor of bf16 bits; positions: int list [S][Tq].
+        hold_barrier: the library's test hook (CTA 0 withholds its arrival at
+        that grid barrier, so the step ends with a timeout)."""
         w = self.w
         pos = torch.tensor(positions, dtype=torch.int32, device=self.dev)
         S, Tq = pos.shape
@@ -77,14 +81,18 @@ class Engine:
         cap = {}
         if capture:
             L, k, E, qd = w.n_layers, w.top_k, w.n_experts, w.n_q_heads * w.head_dim
+            kvd = w.n_kv_heads * w.head_dim
             cap = {"route_ids": torch.full((L, T, k), -1, dtype=torch.int16, device=self.dev),
                    "route_w": torch.zeros((L, T, k), dtype=torch.float32, device=self.dev),
                    "logits": torch.zeros((L, T, E), dtype=torch.float32, device=self.dev),
-                   "attn_out": torch.zeros((L, T, qd), dtype=torch.float32, device=self.dev)}
+                   "attn_out": torch.zeros((L, T, qd), dtype=torch.float32, device=self.dev),
+                   "k_pre": torch.zeros((L, T, kvd), dtype=torch.float32, device=self.dev),
+                   "v_pre": torch.zeros((L, T, kvd), dtype=torch.float32, device=self.dev)}
             msk.msk_set_debug(self.h, cap["route_ids"].data_ptr(), cap["route_w"].data_ptr(),
-                              cap["logits"].data_ptr(), cap["attn_out"].data_ptr())
+                              cap["logits"].data_ptr(), cap["attn_out"].data_ptr(), k_pre=cap["k_pre"].data_ptr(),
+                              v_pre=cap["v_pre"].data_ptr(), hold_barrier=hold_barrier)
         else:
-            msk.msk_set_debug(self.h)
+            msk.msk_set_debug(self.h, hold_barrier=hold_barrier)
         st = stream if stream is not None else torch.cuda.current_stream(self.dev).cuda_stream
         msk.msk_step(self.h, hidden.data_ptr(), pos.data_ptr(), S, Tq, self.kv, out.data_ptr(), st)
         torch.cuda.synchronize(self.dev)

@@ -5,7 +5,7 @@ so the oracle can regenerate any tensor on the host.
 """
 import torch
 
-from . import ROLES, dev_init, dev_nvfp4, dev_past, dev_vec, dev_hidden, nvfp4_shape
+from . import ROLES, dev_init, dev_nvfp4, dev_nvfp4_experts, dev_past, dev_vec, dev_hidden, nvfp4_shape
 
 _inited = set()
 
@@ -31,6 +31,7 @@ class DeviceWeights:
         stream = torch.cuda.current_stream(dev).cuda_stream
         qd, kvd = w.n_q_heads * w.head_dim, w.n_kv_heads * w.head_dim
         self.bytes = 0
+        keys = torch.empty(w.n_experts, dtype=torch.int64, device=dev)  # per-expert generator keys
         with torch.cuda.device(device):
             for l in range(w.n_layers):
                 L = {}
@@ -53,9 +54,7 @@ class DeviceWeights:
                     per_c, per_s = rows * K // 2, rows * K // 16
                     c = torch.empty(w.n_experts * per_c, dtype=torch.uint8, device=dev)
                     s = torch.empty(w.n_experts * per_s, dtype=torch.uint8, device=dev)
-                    gs = None
-                    for e in range(w.n_experts):
-                        gs = dev_nvfp4(w, role, l, e, c.data_ptr() + e * per_c, s.data_ptr() + e * per_s, stream)
+                    gs = dev_nvfp4_experts(w, role, l, keys.data_ptr(), c.data_ptr(), s.data_ptr(), stream)
                     self.keep += [c, s]
                     L[role] = (c.data_ptr(), s.data_ptr(), gs)
                     self.bytes += c.numel() + s.numel()

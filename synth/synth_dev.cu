@@ -42,6 +42,27 @@ static __global__ void k_fill_nvfp4(uint64_t key, uint32_t K, int64_t nblocks, f
   }
 }
 
+/* the same fill for n experts' tensors stacked [E][rows][K]: expert e's
+ * blocks use keys[e] (one launch for a whole expert role) */
+static __global__ void k_fill_nvfp4_experts(const uint64_t* __restrict__ keys, uint32_t K, int64_t blocks_per_expert,
+                                            int64_t nblocks, float sigma, float gs, uint8_t* __restrict__ codes,
+                                            uint8_t* __restrict__ scales) {
+  const uint32_t nkb = K / 16;
+  for (int64_t blk = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; blk < nblocks;
+       blk += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t e = blk / blocks_per_expert, in_e = blk - e * blocks_per_expert;
+    const int64_t r = in_e / nkb;
+    const uint32_t kb = (uint32_t)(in_e - r * nkb);
+    uint8_t c8[8];
+    uint8_t sc = sy_nvfp4_gen_block(&g_dev_tab, keys[e], (uint64_t)r, K, kb, sigma, gs, c8);
+    uint2 w;
+    w.x = (uint32_t)c8[0] | ((uint32_t)c8[1] << 8) | ((uint32_t)c8[2] << 16) | ((uint32_t)c8[3] << 24);
+    w.y = (uint32_t)c8[4] | ((uint32_t)c8[5] << 8) | ((uint32_t)c8[6] << 16) | ((uint32_t)c8[7] << 24);
+    *reinterpret_cast<uint2*>(codes + blk * 8) = w;
+    scales[blk] = sc;
+  }
+}
+
 static __global__ void k_fill_vec(uint64_t key, int64_t n, int gauss, float sigma, float* __restrict__ out) {
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     uint64_t h = sy_u64(key, (uint64_t)i);
@@ -102,6 +123,33 @@ int sy_dev_fill_nvfp4(const sy_model* m, int role, int layer, int expert, void* 
   k_fill_nvfp4<<<grid_for(nb), 256, 0, (cudaStream_t)stream>>>(sy_nvfp4_key(m, role, layer, expert),
                                                                 (uint32_t)K, nb, sigma, gs,
                                                                 (uint8_t*)codes, (uint8_t*)scales);
+  if (gs_out) *gs_out = gs;
+  return (int)cudaGetLastError();
+}
+
+/* Every expert of one role: codes[E][rows][K/2], scales[E][rows][K/16] in
+ * one launch.  keys_dev is caller-provided device scratch of n_experts
+ * uint64. */
+int sy_dev_fill_nvfp4_experts(const sy_model* m, int role, int layer, int n_experts, void* keys_dev, void* codes,
+                              void* scales, float* gs_out, void* stream) {
+  int64_t rows, K;
+  float sigma, gs;
+  sy_nvfp4_shape(m, role, &rows, &K);
+  sy_nvfp4_params(m, role, &sigma, &gs);
+  if (K % 16 || n_experts < 1) return -1;
+  if (((uintptr_t)codes & 7u) != 0) return -2;
+  uint64_t* hk = (uint64_t*)malloc(sizeof(uint64_t) * (size_t)n_experts);
+  if (!hk) return -3;
+  for (int e = 0; e < n_experts; ++e) hk[e] = sy_nvfp4_key(m, role, layer, e);
+  cudaError_t err = cudaMemcpyAsync(keys_dev, hk, sizeof(uint64_t) * (size_t)n_experts, cudaMemcpyHostToDevice,
+                                    (cudaStream_t)stream);
+  if (err == cudaSuccess) err = cudaStreamSynchronize((cudaStream_t)stream);
+  free(hk);
+  if (err != cudaSuccess) return (int)err;
+  const int64_t per = rows * (K / 16), nb = per * n_experts;
+  k_fill_nvfp4_experts<<<grid_for(nb), 256, 0, (cudaStream_t)stream>>>((const uint64_t*)keys_dev, (uint32_t)K, per,
+                                                                      nb, sigma, gs, (uint8_t*)codes,
+                                                                      (uint8_t*)scales);
   if (gs_out) *gs_out = gs;
   return (int)cudaGetLastError();
 }

@@ -15,7 +15,7 @@ import torch
 
 import synth
 import verify_step_megakernel_b200 as msk
-from tests._gpu import config_struct
+from synth.engine import config_struct
 
 INVALID, UNSUPPORTED = 1, 2
 FAKE = 0x10000  # aligned, never read

@@ -18,16 +18,20 @@ import synth
 import synth.gpu as sg
 import verify_step_megakernel_b200 as msk
 from synth.configs import Workload
-from tests._gpu import Engine
+from synth.engine import Engine
 from tests._parity import assert_parity, bf16_to_f64, run_parity
 
 pytestmark = pytest.mark.gpu
 
 
 def _report(name, rep):
+    k, v = rep["kv_k"], rep["kv_v"]
     print(f"\n[{name}] attn_rel max {max(rep['attn_rel']):.2e}  h_abs {rep['h_abs']:.2e}  h_rel {rep['h_rel']:.2e}"
           f"  dh_rel {rep['dh_rel']:.2e}  route exempt {rep['n_exempt']} forced {rep['forced']}"
-          f"  kv midpoint {rep['forced_kv']}/{rep['kv_codes']} invalid {rep['kv_invalid']}")
+          f"  route_w abs {rep['route_w_abs']:.2e} rel {rep['route_w_rel']:.2e}"
+          f"  kv straddles {rep['forced_kv']}/{rep['kv_codes']} (expected {k['expected_diff'] + v['expected_diff']:.0f})"
+          f"  encoder mismatches {k['enc_mismatch'] + v['enc_mismatch']}"
+          f"  pre rel-L2 max K {max(k['pre_rel']):.2e} V {max(v['pre_rel']):.2e}  invalid {rep['kv_invalid']}")
 
 
 def _kv_written_match(w, eng, ref, positions, seqs):
@@ -137,7 +141,7 @@ def test_bad_positions_are_reported():
 def test_invalid_arguments_and_bound():
     w = synth.WORKLOADS["tiny"]
     wts = sg.DeviceWeights(w)
-    from tests._gpu import config_struct, layer_structs
+    from synth.engine import config_struct, layer_structs
     cfg = config_struct(w)
     cfg.head_dim = 96
     with pytest.raises(msk.MskError) as e:

@@ -23,13 +23,16 @@ def test_device_fill_equals_host_fill():
         assert np.array_equal(dc.cpu().numpy(), hc.ravel()) and np.array_equal(ds.cpu().numpy(), hs.ravel())
         assert gs == hgs
     # one expert of each expert tensor, from the stacked device copy
-    for role in ("w_gate", "w_down"):
+    # (the stacked tensors are filled by one launch per role)
+    for role in ("w_gate", "w_up", "w_down"):
         c, s, gs = wts.layers[0][role]
-        hc, hs, _ = synth.host_nvfp4(w, role, 0, 201)
         dev_c = wts.keep[[i for i, t in enumerate(wts.keep) if t.data_ptr() == c][0]]
         dev_s = wts.keep[[i for i, t in enumerate(wts.keep) if t.data_ptr() == s][0]]
-        assert np.array_equal(dev_c[201 * hc.size:202 * hc.size].cpu().numpy(), hc.ravel())
-        assert np.array_equal(dev_s[201 * hs.size:202 * hs.size].cpu().numpy(), hs.ravel())
+        for e in (0, 201, w.n_experts - 1):
+            hc, hs, hgs = synth.host_nvfp4(w, role, 0, e)
+            assert np.array_equal(dev_c[e * hc.size:(e + 1) * hc.size].cpu().numpy(), hc.ravel())
+            assert np.array_equal(dev_s[e * hs.size:(e + 1) * hs.size].cpu().numpy(), hs.ravel())
+            assert gs == hgs
     for name in ("router", "q_norm_g", "moe_norm_g"):
         ptr = wts.layers[1][name]
         host = synth.host_vec(w, name, 1).ravel()

@@ -48,7 +48,8 @@ class LayerWeights(C.Structure):
 
 class Debug(C.Structure):
     _fields_ = [("route_ids", C.c_void_p), ("route_w", C.c_void_p), ("logits", C.c_void_p),
-                ("attn_out", C.c_void_p), ("trace", C.c_void_p)]
+                ("attn_out", C.c_void_p), ("trace", C.c_void_p), ("k_pre", C.c_void_p), ("v_pre", C.c_void_p),
+                ("hold_barrier", C.c_int32)]
 
 
 class Stats(C.Structure):
@@ -58,8 +59,9 @@ class Stats(C.Structure):
 
 
 _lib = None
-EXPORTS = ["msk_create", "msk_destroy", "msk_kv_create", "msk_kv_destroy", "msk_kv_append", "msk_kv_read",
-           "msk_step", "msk_step_static", "msk_step_status", "msk_set_debug", "msk_query", "msk_status_string"]
+EXPORTS = ["msk_create", "msk_destroy", "msk_kv_create", "msk_kv_destroy", "msk_kv_append", "msk_kv_encode",
+           "msk_kv_read", "msk_step", "msk_step_static", "msk_step_status", "msk_step_status_at", "msk_set_debug",
+           "msk_query", "msk_status_string"]
 STATIC_SCRATCH_BYTES = 8 << 20
 
 
@@ -78,15 +80,17 @@ def lib():
         L.msk_kv_destroy.restype = None
         L.msk_kv_append.argtypes = [P, P, I, I, I64, I64, P, P, P]
         L.msk_kv_read.argtypes = [P, P, I, I, I64, I64, P, P]
+        L.msk_kv_encode.argtypes = [P, P, I64, P]
         L.msk_step.argtypes = [P, P, P, I, I, P, P, P]
         L.msk_step_static.argtypes = [P, P, P, I, I, P, P, P]
         L.msk_step_status.argtypes = [P]
+        L.msk_step_status_at.argtypes = [P, C.POINTER(C.c_int32), C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
         L.msk_set_debug.argtypes = [P, C.POINTER(Debug)]
         L.msk_query.argtypes = [P, C.POINTER(Stats)]
         L.msk_status_string.argtypes = [I]
         L.msk_status_string.restype = C.c_char_p
-        for name in ("msk_create", "msk_kv_create", "msk_kv_append", "msk_kv_read", "msk_step",
-                     "msk_step_static", "msk_step_status", "msk_set_debug", "msk_query"):
+        for name in ("msk_create", "msk_kv_create", "msk_kv_append", "msk_kv_encode", "msk_kv_read", "msk_step",
+                     "msk_step_static", "msk_step_status", "msk_step_status_at", "msk_set_debug", "msk_query"):
             getattr(L, name).restype = C.c_int
         _lib = L
     return _lib
@@ -122,6 +126,10 @@ def msk_kv_append(h, kv, layer, seq, pos0, n, k_fp8, v_fp8, stream=0):
     _check(lib().msk_kv_append(h, kv, layer, seq, pos0, n, k_fp8, v_fp8, stream), "msk_kv_append")
 
 
+def msk_kv_encode(in_f32, out_u8, n, stream=0):
+    _check(lib().msk_kv_encode(in_f32, out_u8, n, stream), "msk_kv_encode")
+
+
 def msk_kv_read(h, kv, layer, seq, pos0, n, k_out, v_out):
     _check(lib().msk_kv_read(h, kv, layer, seq, pos0, n, k_out, v_out), "msk_kv_read")
 
@@ -141,8 +149,16 @@ def msk_step_status(h) -> int:
     return lib().msk_step_status(h)
 
 
-def msk_set_debug(h, route_ids=0, route_w=0, logits=0, attn_out=0, trace=0):
-    d = Debug(route_ids or None, route_w or None, logits or None, attn_out or None, trace or None)
+def msk_step_status_at(h):
+    """(status, layer, phase, cta) of the steps since the last status call."""
+    a, b, c = C.c_int32(), C.c_int32(), C.c_int32()
+    st = lib().msk_step_status_at(h, C.byref(a), C.byref(b), C.byref(c))
+    return st, a.value, b.value, c.value
+
+
+def msk_set_debug(h, route_ids=0, route_w=0, logits=0, attn_out=0, trace=0, k_pre=0, v_pre=0, hold_barrier=0):
+    d = Debug(route_ids or None, route_w or None, logits or None, attn_out or None, trace or None, k_pre or None,
+              v_pre or None, int(hold_barrier))
     _check(lib().msk_set_debug(h, C.byref(d)), "msk_set_debug")
 
 

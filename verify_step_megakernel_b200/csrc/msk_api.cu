@@ -16,6 +16,7 @@
 
 extern "C" size_t msk_kernel_smem_bytes();
 extern "C" cudaError_t msk_kernel_setup(int hd, int* ctas_per_sm);
+extern "C" cudaError_t msk_kernel_kv_encode(const float* in, uint8_t* out, int64_t n, cudaStream_t stream);
 extern "C" cudaError_t msk_kernel_launch(int hd, const MskParams* P_dev, const MskStep* st, const CUtensorMap* map,
                                          int ncta, cudaStream_t stream);
 
@@ -112,12 +113,11 @@ static msk_status_t check_config(const msk_config_t* c) {
 static __device__ __align__(256) uint8_t g_static_scratch[MSK_STATIC_SCRATCH_BYTES];
 
 #define MSK_STATIC_MAX_DEVICES 64
-struct StaticSlot {
-  std::once_flag once;
-  uint8_t* ptr;
-  cudaError_t err;
-};
-static StaticSlot g_static_slots[MSK_STATIC_MAX_DEVICES];
+/* the array's device address per device, found on the first call that
+ * succeeds in looking it up (a failed lookup leaves the slot empty, so a
+ * later call tries again) */
+static std::mutex g_static_mu;
+static uint8_t* g_static_ptr[MSK_STATIC_MAX_DEVICES];
 
 /* where the step's buffers sit inside g_static_scratch */
 struct StaticLayout {
@@ -521,6 +521,12 @@ msk_status_t msk_kv_append(msk_handle_t* h, msk_kv_t* kv, int layer, int seq, in
   return e == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
 }
 
+msk_status_t msk_kv_encode(const float* in, uint8_t* out, int64_t n, void* stream) {
+  if (n < 0 || (n > 0 && (!in || !out || !aligned16(in) || !aligned16(out)))) return MSK_ERR_INVALID_ARG;
+  if (n == 0) return MSK_OK;
+  return msk_kernel_kv_encode(in, out, n, (cudaStream_t)stream) == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
+}
+
 msk_status_t msk_kv_read(msk_handle_t* h, msk_kv_t* kv, int layer, int seq, int64_t pos0, int64_t n, uint8_t* k_out,
                          uint8_t* v_out) {
   if (!h || !kv || kv->h != h || !k_out || !v_out) return MSK_ERR_INVALID_ARG;
@@ -571,7 +577,10 @@ msk_status_t msk_step(msk_handle_t* h, const uint16_t* hidden_in, const int32_t*
   return e == cudaSuccess ? MSK_OK : MSK_ERR_CUDA;
 }
 
-msk_status_t msk_step_status(msk_handle_t* h) {
+msk_status_t msk_step_status_at(msk_handle_t* h, int32_t* layer, int32_t* phase, int32_t* cta) {
+  if (layer) *layer = -1;
+  if (phase) *phase = -1;
+  if (cta) *cta = -1;
   if (!h) return MSK_ERR_INVALID_ARG;
   int prev = 0;
   cudaGetDevice(&prev);
@@ -581,8 +590,17 @@ msk_status_t msk_step_status(msk_handle_t* h) {
   if (e == cudaSuccess) e = cudaMemset(h->host.status, 0, sizeof w);
   cudaSetDevice(prev);
   if (e != cudaSuccess) return MSK_ERR_CUDA;
+  /* the site word is (layer << 16) | (phase << 8) | cta, plus one in the top
+   * bit when set (a site-less error leaves it zero) */
+  if (w[ST_CODE] != 0 && (w[ST_WHERE] & 0x80000000u)) {
+    if (layer) *layer = (int32_t)((w[ST_WHERE] >> 16) & 0x7FFF);
+    if (phase) *phase = (int32_t)((w[ST_WHERE] >> 8) & 0xFF);
+    if (cta) *cta = (int32_t)(w[ST_WHERE] & 0xFF);
+  }
   return (msk_status_t)w[ST_CODE];
 }
+
+msk_status_t msk_step_status(msk_handle_t* h) { return msk_step_status_at(h, nullptr, nullptr, nullptr); }
 
 msk_status_t msk_set_debug(msk_handle_t* h, const msk_debug_t* dbg) {
   if (!h) return MSK_ERR_INVALID_ARG;
@@ -595,6 +613,9 @@ msk_status_t msk_set_debug(msk_handle_t* h, const msk_debug_t* dbg) {
   P.dbg_logits = d.logits;
   P.dbg_attn = d.attn_out;
   P.dbg_trace = d.trace;
+  P.dbg_kpre = d.k_pre;
+  P.dbg_vpre = d.v_pre;
+  P.dbg_hold = d.hold_barrier > 0 ? d.hold_barrier : 0;
   h->dbg = d;
   int prev = 0;
   cudaGetDevice(&prev);
@@ -658,16 +679,22 @@ msk_status_t msk_step_static(msk_handle_t* h, const uint16_t* hidden_in, const i
   int prev = 0;
   cudaGetDevice(&prev);
   if (prev != h->device && cudaSetDevice(h->device) != cudaSuccess) return MSK_ERR_CUDA;
-  /* first call on this device, with the device current: look up the
-   * array's device address once */
-  StaticSlot& slot = g_static_slots[h->device];
-  std::call_once(slot.once, [&slot]() {
-    slot.ptr = nullptr;
-    slot.err = cudaGetSymbolAddress((void**)&slot.ptr, g_static_scratch);
-  });
-  cudaError_t e = (slot.err == cudaSuccess && slot.ptr) ? cudaSuccess : cudaErrorInvalidSymbol;
+  /* with the device current: the array's device address, looked up on the
+   * first call that succeeds */
+  uint8_t* base = nullptr;
+  cudaError_t e = cudaSuccess;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[h->device]) {
+      uint8_t* p = nullptr;
+      e = cudaGetSymbolAddress((void**)&p, g_static_scratch);
+      if (e == cudaSuccess && p) g_static_ptr[h->device] = p;
+      else if (e == cudaSuccess) e = cudaErrorInvalidSymbol;
+    }
+    base = g_static_ptr[h->device];
+  }
   if (e == cudaSuccess) {
-    uint8_t* b = slot.ptr;
+    uint8_t* b = base;
     StaticPtrs p;
     p.h = (float*)(b + Lo.h);
     p.x = (uint16_t*)(b + Lo.x);

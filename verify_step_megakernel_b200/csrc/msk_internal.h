@@ -85,6 +85,10 @@ typedef struct MskParams {
   float* dbg_logits;
   float* dbg_attn;
   uint64_t* dbg_trace;
+  float* dbg_kpre;  /* [L][T][kvd] keys after QK-norm, before fp8 */
+  float* dbg_vpre;  /* [L][T][kvd] values before fp8 */
+  int32_t dbg_hold; /* > 0: CTA 0 withholds its arrival at grid barrier number dbg_hold (test hook) */
+  int32_t dbg_pad;
   MskLayer layers[MSK_MAX_LAYERS];
 } MskParams;
 

@@ -127,20 +127,24 @@ MSK_DEV bool aborted(const Ctx& c) {
 
 MSK_DEV void raise_err(const Ctx& c, uint32_t code, int layer, int phase) {
   if (atomicCAS(&c.P->status[ST_CODE], 0u, code) == 0u)
-    c.P->status[ST_WHERE] = ((uint32_t)layer << 16) | ((uint32_t)phase << 8) | (uint32_t)(c.cta & 0xFF);
+    c.P->status[ST_WHERE] =
+        0x80000000u | ((uint32_t)(layer & 0x7FFF) << 16) | ((uint32_t)phase << 8) | (uint32_t)(c.cta & 0xFF);
   atomicExch(&c.P->ctrl[CTRL_ABORT], 1u);
   c.S->abort = 1;
 }
 
-/* bounded mbarrier wait; false on timeout or abort */
-MSK_DEV bool wait_bar(const Ctx& c, uint64_t* bar, uint32_t parity, int layer, int phase) {
+/* bounded mbarrier wait; false on timeout or abort.  `mult` scales the
+ * limit: the producer's waits on the consumers' progress take twice the
+ * limit of the consumers' own waits, so that when a step stalls, the wait
+ * nearest the cause gives up first and its site is the one recorded. */
+MSK_DEV bool wait_bar(const Ctx& c, uint64_t* bar, uint32_t parity, int layer, int phase, uint32_t mult = 1) {
   if (mbar_try(bar, parity)) return true;
   uint64_t t0 = gtimer();
   for (uint32_t it = 0;; ++it) {
     if (mbar_try(bar, parity)) return true;
     if ((it & 63) == 0) {
       if (aborted(c)) return false;
-      if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+      if (gtimer() - t0 > mult * (uint64_t)c.P->timeout_ns) {
         raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
         return false;
       }
@@ -157,8 +161,11 @@ MSK_DEV bool grid_sync(Ctx& c, int layer, int phase) {
     if (ok) {
       /* release: the CTA's writes (ordered before this thread by the CTA
        * barrier above) become visible before the count moves; acquire on
-       * the poll orders the other CTAs' writes before ours */
-      red_release_add_u32(&c.P->ctrl[CTRL_BARRIER], 1u);
+       * the poll orders the other CTAs' writes before ours.  The test hook
+       * dbg_hold makes CTA 0 withhold one arrival, so that every wait at
+       * that barrier runs out. */
+      if (!(c.cta == 0 && c.P->dbg_hold > 0 && c.nbar + 1 == (uint32_t)c.P->dbg_hold))
+        red_release_add_u32(&c.P->ctrl[CTRL_BARRIER], 1u);
       const uint32_t target = (c.nbar + 1) * (uint32_t)c.ncta;
       uint64_t t0 = 0;
       for (uint32_t it = 0; ld_acquire_u32(&c.P->ctrl[CTRL_BARRIER]) < target; ++it) {
@@ -381,7 +388,7 @@ struct Prod {
  * flow stays uniform.  Lane 0 posts each barrier's byte count, then the
  * lanes issue the copies in parallel. */
 MSK_DEV bool pwait_bar(const Ctx& c, uint64_t* bar, uint32_t parity, int layer, int phase) {
-  return __all_sync(0xffffffffu, wait_bar(c, bar, parity, layer, phase)) != 0;
+  return __all_sync(0xffffffffu, wait_bar(c, bar, parity, layer, phase, 2)) != 0;
 }
 
 MSK_DEV bool prod_acquire(Prod& p, int layer, int phase, uint8_t** stg, uint64_t** bar) {
@@ -403,12 +410,13 @@ MSK_DEV bool prod_drain(Prod& p, int layer, int phase) {
   return true;
 }
 
+/* a flag the consumers set: twice the consumers' limit (see wait_bar) */
 MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, int phase) {
   uint64_t t0 = gtimer();
   for (uint32_t it = 0; *flag < want; ++it) {
     if ((it & 15) == 0) {
       if (aborted(c)) return false;
-      if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+      if (gtimer() - t0 > 2 * (uint64_t)c.P->timeout_ns) {
         raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
         return false;
       }
@@ -1320,6 +1328,11 @@ MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
     } else {
       const int isv = hh >= P->hq + P->hkv;
       const int kvh = hh - P->hq - (isv ? P->hkv : 0);
+      float* pre = isv ? P->dbg_vpre : P->dbg_kpre;
+      if (pre) {
+        pre += ((size_t)layer * c.st.T + t) * P->kvd + kvh * hd + lane * per;
+        for (int i = 0; i < per; ++i) pre[i] = v[i];
+      }
       const int64_t pos = c.S->pos0[b] + ti;
       int64_t row = (((int64_t)layer * c.st.kv_seqs + b) * P->hkv + kvh) * c.st.kv_cap + pos;
       if (isv) row += c.st.kv_half_rows;
@@ -2007,8 +2020,32 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
   }
 }
 
+/* fp32 -> fp8 e4m3 codes with the KV write's conversion (RNE, satfinite),
+ * four values per thread */
+__global__ void msk_kv_encode_kernel(const float4* __restrict__ in, uint32_t* __restrict__ out, int64_t n4) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 v = in[i];
+    out[i] = f32x2_to_e4m3x2(v.x, v.y) | (f32x2_to_e4m3x2(v.z, v.w) << 16);
+  }
+}
+__global__ void msk_kv_encode_tail(const float* __restrict__ in, uint8_t* __restrict__ out, int64_t i0, int64_t n) {
+  const int64_t i = i0 + threadIdx.x;
+  if (i < n) out[i] = (uint8_t)f32x2_to_e4m3x2(in[i], 0.f);
+}
+
 /* ---- launch ---------------------------------------------------------------------------- */
 extern "C" size_t msk_kernel_smem_bytes() { return SMEM_BYTES; }
+
+extern "C" cudaError_t msk_kernel_kv_encode(const float* in, uint8_t* out, int64_t n, cudaStream_t stream) {
+  const int64_t n4 = n / 4;
+  if (n4 > 0) {
+    const int64_t blocks = (n4 + 255) / 256;
+    msk_kv_encode_kernel<<<(unsigned)(blocks < 148 * 16 ? blocks : 148 * 16), 256, 0, stream>>>(
+        reinterpret_cast<const float4*>(in), reinterpret_cast<uint32_t*>(out), n4);
+  }
+  if (n % 4) msk_kv_encode_tail<<<1, 32, 0, stream>>>(in, out, n4 * 4, n);
+  return cudaGetLastError();
+}
 
 static const void* kernel_for(int hd) {
   return hd == 128 ? (const void*)msk_step_kernel<128> : (const void*)msk_step_kernel<64>;
