@@ -243,7 +243,7 @@ def run_msk(args, w):
             dist.barrier()
 
     t_setup = time.perf_counter()
-    eng = Engine(w, device=local, flags=msk.F_TC_EXPERTS if args.tc_experts else 0)
+    eng = Engine(w, device=local, flags=msk.F_TC_EXPERTS if args.tc_experts else 0, tau=args.tau)
     eng.fill_past()
     hid = sg.hidden(w, local)
     pos = torch.tensor(w.positions(), dtype=torch.int32, device=dev)
@@ -486,6 +486,9 @@ def main():
     ap.add_argument("--trace", action="store_true", help="print a per-phase device-time breakdown instead")
     ap.add_argument("--tc-experts", action="store_true",
                     help="gate/up on the block-scaled tensor cores (MSK_F_TC_EXPERTS) instead of the default path")
+    ap.add_argument("--tau", type=int, default=0,
+                    help="expert_mma_min_tokens: units with at least this many tokens take the block-scaled path "
+                         "(0 = never)")
     ap.add_argument("--sweep", action="store_true",
                     help="step time of the workload's model over batch shapes (one JSON line per shape)")
     args = ap.parse_args()

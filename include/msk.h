@@ -86,15 +86,23 @@ typedef struct msk_config {
                                  <= 64 */
   uint32_t flags;         /* MSK_F_* */
   int32_t wait_timeout_us; /* limit of every device wait; 0 = 2,000,000 */
+  int32_t expert_mma_min_tokens; /* tau: the gate/up projection of an expert
+                             unit (up to 8 of an expert's tokens) with at
+                             least tau tokens runs on the block-scaled tensor
+                             cores, the others on the CUDA-core path (the
+                             post's "Expert Weight Quantization": NVFP4 GEMV
+                             at one token, a dense contraction where several
+                             tokens share an expert).  0 = never (unless
+                             MSK_F_TC_EXPERTS), 1 = always */
 } msk_config_t;
 
 #define MSK_F_TRACE 1u /* record per-phase %globaltimer stamps (msk_query) */
-/* Gate/up projections on the block-scaled tensor cores (tcgen05.mma
- * kind::mxf4nvf4): the NVFP4 weights are consumed as stored, the moe-norm
+/* Gate/up projections of every expert unit on the block-scaled tensor cores
+ * (tcgen05.mma kind::mxf4nvf4), the same as expert_mma_min_tokens = 1: the
+ * NVFP4 weights are consumed as stored (their block scales from a copy
+ * msk_create repacks into the tensor cores' layout), the moe-norm
  * activations as eight e2m1 terms (relative error ~1e-5 of the row's
- * largest value).  Default off: with units of 2-3 tokens per expert the
- * per-instruction cost of the tensor-core path exceeds the CUDA-core
- * decode it saves (see the design notes for the measurements). */
+ * largest value). */
 #define MSK_F_TC_EXPERTS 2u
 
 /* Per-layer weights, all device pointers, borrowed.
@@ -151,6 +159,10 @@ typedef struct msk_stats {
   int64_t weight_bytes;       /* the weight part of algorithmic_bytes */
   int64_t kv_bytes;           /* the KV part */
   int64_t scratch_bytes;      /* device scratch the handle owns */
+  int64_t repacked_bytes;     /* library-owned copies of weight data in
+                                 another layout (the gate/up block scales in
+                                 the block-scaled tensor cores' layout, when
+                                 that expert path is enabled) */
 } msk_stats_t;
 
 /* Create a handle on `device`: validates the shapes, computes the per-layer

@@ -10,7 +10,7 @@ import synth.gpu as sg
 import verify_step_megakernel_b200 as msk
 
 
-def config_struct(w, max_seqs=None, max_tps=None, timeout_us=0, flags=0):
+def config_struct(w, max_seqs=None, max_tps=None, timeout_us=0, flags=0, tau=0):
     c = msk.Config()
     c.n_layers, c.d_model, c.n_q_heads, c.n_kv_heads = w.n_layers, w.d_model, w.n_q_heads, w.n_kv_heads
     c.head_dim, c.n_experts, c.top_k, c.expert_dim, c.window = (w.head_dim, w.n_experts, w.top_k, w.expert_dim,
@@ -22,6 +22,7 @@ def config_struct(w, max_seqs=None, max_tps=None, timeout_us=0, flags=0):
     c.max_tokens_per_seq = max_tps or w.tokens_per_seq
     c.flags = flags
     c.wait_timeout_us = timeout_us
+    c.expert_mma_min_tokens = tau
     return c
 
 
@@ -42,12 +43,12 @@ class Engine:
     """Weights + handle + KV cache of one workload on cuda:device."""
 
     def __init__(self, w, device=0, capacity=None, max_seqs=None, max_tps=None, timeout_us=0, flags=0,
-                 past_per_seq=None):
+                 past_per_seq=None, tau=0):
         self.w = w
         self.device = device
         self.dev = torch.device("cuda", device)
         self.wts = sg.DeviceWeights(w, device)
-        self.cfg = config_struct(w, max_seqs, max_tps, timeout_us, flags)
+        self.cfg = config_struct(w, max_seqs, max_tps, timeout_us, flags, tau)
         self.h = msk.msk_create(self.cfg, layer_structs(self.wts), device)
         self.n_seqs = max_seqs or w.n_seqs
         self.past = past_per_seq or [w.past] * self.n_seqs

@@ -81,6 +81,26 @@ def test_parity_workload(name):
     eng.close()
 
 
+@pytest.mark.parametrize("tau", [2, 3])
+def test_parity_mixed_expert_paths(tau):
+    """expert_mma_min_tokens = tau: in one step, the gate/up of expert units
+    with at least tau tokens runs on the block-scaled tensor cores and the
+    rest on the CUDA-core path; both kinds occur in every layer here."""
+    w = synth.WORKLOADS["ver8"]
+    eng = Engine(w, tau=tau)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions())
+    _report(f"ver8 tau {tau}", rep)
+    assert_parity(rep)
+    # both paths ran: per layer, experts chosen by at least tau tokens and by fewer
+    for l in range(w.n_layers):
+        cnt = np.bincount(gpu["route_ids"][l].ravel().astype(np.int64), minlength=w.n_experts)
+        assert (cnt >= tau).any() and ((cnt > 0) & (cnt < tau)).any(), (l, np.bincount(cnt))
+    assert msk.msk_query(eng.h).repacked_bytes > 0
+    eng.close()
+
+
 RAGGED = Workload("ragged", 3, 256, 4, 2, 64, 128, [1, 0, 1], 3, 3, 0, 0x5EED + 40, n_experts=32, top_k=4,
                   window=100)
 

@@ -36,7 +36,7 @@ class Config(C.Structure):
                 ("top_k", C.c_int32), ("expert_dim", C.c_int32), ("window", C.c_int32),
                 ("layer_is_sliding", C.c_uint8 * MAX_LAYERS), ("rms_eps", C.c_float),
                 ("max_seqs", C.c_int32), ("max_tokens_per_seq", C.c_int32), ("flags", C.c_uint32),
-                ("wait_timeout_us", C.c_int32)]
+                ("wait_timeout_us", C.c_int32), ("expert_mma_min_tokens", C.c_int32)]
 
 
 class LayerWeights(C.Structure):
@@ -55,7 +55,7 @@ class Debug(C.Structure):
 class Stats(C.Structure):
     _fields_ = [("n_layers", C.c_int32), ("n_distinct", C.c_int32 * MAX_LAYERS),
                 ("algorithmic_bytes", C.c_int64), ("weight_bytes", C.c_int64), ("kv_bytes", C.c_int64),
-                ("scratch_bytes", C.c_int64)]
+                ("scratch_bytes", C.c_int64), ("repacked_bytes", C.c_int64)]
 
 
 _lib = None

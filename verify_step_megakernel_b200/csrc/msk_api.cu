@@ -16,6 +16,7 @@
 
 extern "C" size_t msk_kernel_smem_bytes();
 extern "C" cudaError_t msk_kernel_setup(int hd, int* ctas_per_sm);
+extern "C" cudaError_t msk_kernel_sf_repack(const uint8_t* in, uint8_t* out, int64_t rows, int k16, cudaStream_t st);
 extern "C" cudaError_t msk_kernel_kv_encode(const float* in, uint8_t* out, int64_t n, cudaStream_t stream);
 extern "C" cudaError_t msk_kernel_launch(int hd, const MskParams* P_dev, const MskStep* st, const CUtensorMap* map,
                                          int ncta, cudaStream_t stream);
@@ -29,6 +30,8 @@ struct msk_handle {
   MskParams* dev;   /* device copy */
   void* scratch;    /* one allocation for every scratch buffer */
   CUtensorMap* emaps; /* [L][MSK_NMAPS] weight tensor maps (device) */
+  uint8_t* repack;    /* gate/up scale-factor atoms of every layer (block-scaled expert path), or null */
+  size_t repack_bytes;
   size_t scratch_bytes;
   uint32_t* words;  /* ctrl + status */
   msk_debug_t dbg;
@@ -97,7 +100,7 @@ static msk_status_t check_config(const msk_config_t* c) {
   if (c->max_seqs * c->max_tokens_per_seq > MSK_MAX_TOKENS) return MSK_ERR_UNSUPPORTED;
   if (c->max_tokens_per_seq * (c->n_q_heads / c->n_kv_heads) > 64) return MSK_ERR_UNSUPPORTED;
   if (c->max_seqs * c->n_kv_heads > MSK_MAX_PAIRS) return MSK_ERR_UNSUPPORTED;
-  if (c->wait_timeout_us < 0) return MSK_ERR_INVALID_ARG;
+  if (c->wait_timeout_us < 0 || c->expert_mma_min_tokens < 0) return MSK_ERR_INVALID_ARG;
   return MSK_OK;
 }
 
@@ -254,6 +257,9 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)P.hd));
   P.timeout_ns = (int64_t)(c.wait_timeout_us ? c.wait_timeout_us : 2000000) * 1000;
   P.flags = c.flags;
+  /* tau: 0 = never (2^30), MSK_F_TC_EXPERTS = every unit */
+  P.tau = (c.flags & MSK_F_TC_EXPERTS) ? 1 : (c.expert_mma_min_tokens > 0 ? c.expert_mma_min_tokens : (1 << 30));
+  if (P.tau < 1) P.tau = 1;
 
   /* the fixed softmax shift of each layer, from its QK-norm gains */
   float* gq = (float*)malloc(sizeof(float) * P.hd);
@@ -339,7 +345,7 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       for (int m = 0; m < 3 && ok; ++m) {
         const int64_t K = m < 2 ? P.d : P.f, rows = (int64_t)P.E * (m < 2 ? P.f : P.d);
         /* K chunks: 256 for gate/up on the tensor cores, else 512 (or all of K) */
-        const int KC = (m < 2 && (c.flags & MSK_F_TC_EXPERTS)) ? 256 : (K <= 512 ? (int)K : 512);
+        const int KC = K <= 512 ? (int)K : 512; /* the CUDA-core path's chunks */
         /* K not a multiple of 256 (128, 384): whole rows go as bulk copies
          * and the maps stay zero */
         if (K % 256) continue;
@@ -400,7 +406,32 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       return MSK_ERR_CUDA;
     }
   }
+  /* the block-scaled expert path reads the gate/up block scales in the
+   * tensor cores' scale-factor layout: repack them once (library-owned
+   * copy; the borrowed weights are not touched) */
+  if (P.tau <= MSK_UNIT_TOK) { /* some unit can take the block-scaled path */
+    const size_t per = (size_t)P.E * P.f * (P.d / 16); /* bytes of one matrix's scales */
+    h->repack_bytes = 2 * per * P.L;
+    bool ok = cudaMalloc(&h->repack, h->repack_bytes) == cudaSuccess;
+    for (int l = 0; l < P.L && ok; ++l) {
+      uint8_t* g = h->repack + (size_t)2 * l * per;
+      ok = msk_kernel_sf_repack(layers[l].w_gate.scales, g, (int64_t)P.E * P.f, P.d / 16, 0) == cudaSuccess &&
+           msk_kernel_sf_repack(layers[l].w_up.scales, g + per, (int64_t)P.E * P.f, P.d / 16, 0) == cudaSuccess;
+      P.layers[l].sfg = g;
+      P.layers[l].sfu = g + per;
+    }
+    if (ok) ok = cudaDeviceSynchronize() == cudaSuccess;
+    if (!ok) {
+      if (h->repack) cudaFree(h->repack);
+      cudaFree(h->emaps);
+      cudaFree(h->scratch);
+      delete h;
+      cudaSetDevice(prev);
+      return MSK_ERR_OOM;
+    }
+  }
   if (cudaMalloc(&h->dev, sizeof(MskParams)) != cudaSuccess) {
+    if (h->repack) cudaFree(h->repack);
     cudaFree(h->emaps);
     cudaFree(h->scratch);
     delete h;
@@ -410,6 +441,7 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   if (cudaMemcpy(h->dev, &P, sizeof(MskParams), cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaDeviceSynchronize() != cudaSuccess) {
     cudaFree(h->dev);
+    if (h->repack) cudaFree(h->repack);
     cudaFree(h->emaps);
     cudaFree(h->scratch);
     delete h;
@@ -430,6 +462,7 @@ void msk_destroy(msk_handle_t* h) {
   cudaFree(h->dev);
   cudaFree(h->scratch);
   cudaFree(h->emaps);
+  if (h->repack) cudaFree(h->repack);
   cudaSetDevice(prev);
   delete h;
 }
@@ -631,6 +664,7 @@ msk_status_t msk_query(msk_handle_t* h, msk_stats_t* out) {
   const MskParams& P = h->host;
   out->n_layers = P.L;
   out->scratch_bytes = (int64_t)h->scratch_bytes;
+  out->repacked_bytes = (int64_t)h->repack_bytes;
   if (!h->have_last) return MSK_OK;
   int prev = 0;
   cudaGetDevice(&prev);

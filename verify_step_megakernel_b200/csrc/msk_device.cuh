@@ -99,6 +99,22 @@ MSK_DEV void tc_mma_nvf4(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(tmem_sfa), "r"(tmem_sfb)
       : "memory");
 }
+/* D (+)= A B^T with 8-bit operands (kind::f8f6f4; types in the instruction descriptor) */
+MSK_DEV void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+/* D (+)= A B^T with 16-bit operands (kind::f16: f16 or bf16, fp32 accumulate) */
+MSK_DEV void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 /* arrive on an mbarrier once every tcgen05 operation this thread issued has completed */
 MSK_DEV void tc_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
@@ -114,6 +130,12 @@ MSK_DEV void tc_ld32(uint32_t taddr, uint32_t* r) {
         "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
+}
+/* 8 consecutive TMEM columns of this warp's 32 lanes */
+MSK_DEV void tc_ld8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
 }
 MSK_DEV void tc_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
@@ -155,6 +177,11 @@ MSK_DEV uint32_t lds32(uint32_t addr) {
   asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr));
   return v;
 }
+MSK_DEV void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+MSK_DEV void sts32(uint32_t addr, uint32_t v) { asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory"); }
+MSK_DEV void sts16(uint32_t addr, uint16_t v) { asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v) : "memory"); }
 MSK_DEV uint2 lds64(uint32_t addr) {
   uint2 v;
   asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr));
@@ -200,6 +227,12 @@ MSK_DEV uint32_t e4m3pair_to_bf16x2_scaled(uint32_t w0, uint32_t w1, uint32_t se
   uint32_t t = __byte_perm(w0, w1, sel); /* [b, b, b', b'] */
   return (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
 }
+/* bytes 2i and 2i+1 (i = half) of a word of e4m3 codes -> bf16x2 of value *
+ * 2^-120 (exact; the same bit move as e4m3pair_to_bf16x2_scaled) */
+MSK_DEV uint32_t e4m3x2_to_bf16x2_scaled(uint32_t w, int half) {
+  const uint32_t t = __byte_perm(w, w, half ? 0x3322u : 0x1100u); /* [b, b, b', b'] */
+  return (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
+}
 /* the low / high f16 of an f16x2 word as fp32 (exact) */
 MSK_DEV float f16lo_f32(uint32_t w) {
   float f;
@@ -210,6 +243,13 @@ MSK_DEV float f16hi_f32(uint32_t w) {
   float f;
   asm("{\n .reg .b16 l, h;\n mov.b32 {l, h}, %1;\n cvt.f32.f16 %0, h;\n}" : "=f"(f) : "r"(w));
   return f;
+}
+/* an e4m3 code's value as fp32 (exact) */
+MSK_DEV float e4m3_to_f32(uint32_t code) {
+  uint32_t h;
+  const uint16_t two = (uint16_t)(code & 0xFFu);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(two));
+  return f16lo_f32(h);
 }
 /* two floats -> e2m1x2 byte (low nibble = a, high = b), round to nearest
  * even on the e2m1 grid, saturating at 6 */

@@ -50,6 +50,11 @@ typedef struct MskLayer {
    * codes, gate scales, up codes, up scales, down codes, down scales, then
    * (from MSK_MAP_DENSE) codes and scales of wq, wk, wv, wo */
   const CUtensorMap* emap;
+  /* gate and up block scales repacked (library-owned) in the block-scaled
+   * tensor cores' scale-factor atoms: [E][f/128][d/64][512 B], atom byte
+   * 16 r + 4 m + b = scale of row 128 g + r + 32 m, block 4 s + b */
+  const uint8_t* sfg;
+  const uint8_t* sfu;
   float bound_log2; /* M * log2(e), M = sqrt(hd) max|g_q| max|g_k| */
   int32_t sliding;
 } MskLayer;
@@ -60,6 +65,7 @@ typedef struct MskParams {
   float eps, scale_log2; /* 1/sqrt(hd) * log2(e) */
   int64_t timeout_ns;
   uint32_t flags;
+  int32_t tau;      /* expert units with at least tau tokens: gate/up on the block-scaled tensor cores */
   /* scratch (device) */
   float* h;         /* [T][d] residual */
   uint16_t* x;      /* [T][d] f16 attention-norm input of the projections */

@@ -51,6 +51,7 @@ enum Phase {
 
 struct Route {
   int n_units, n_distinct;
+  int n_units_tc; /* units [0, n_units_tc) take the block-scaled gate/up path, the rest the CUDA-core path */
   int16_t ids[MSK_MAX_TOKENS * 8];
   float w[MSK_MAX_TOKENS * 8];
   int16_t cnt[256];
@@ -83,8 +84,6 @@ struct Smem {
   uint64_t dempty[MSK_NCW][2]; /* dense weight slot read by its warp */
   uint64_t bfull;              /* dense activation slice landed */
   uint64_t rfull;              /* the step's router logits landed (top-k) */
-  uint64_t sfdone[4];       /* tensor-core ops up to the last chunk using scale staging b done */
-  uint64_t sfready[4];      /* scale staging b written by every consumer warp */
   uint64_t dfull2[2];       /* accumulator buffer 0/1 holds a finished item */
   uint64_t dempty2[2];      /* accumulator buffer 0/1 read by every consumer warp */
   uint64_t tfin;            /* every tensor-core op issued complete */
@@ -101,6 +100,18 @@ struct Smem {
   volatile int dn_ready;    /* layer+1 whose gate/up outputs all CTAs finished */
   volatile int dense_done;  /* dense phases this CTA finished (2 per layer) */
   volatile int abort;
+  /* attention on the tensor cores (head dim 128): stage ring, score and
+   * probability buffers, Q terms, output accumulator handoff */
+  uint64_t afull[5];        /* K and V of a stage landed (producer's expect-tx) */
+  uint64_t aempty[5];       /* the stage's P.V products completed (tensor-core commit) */
+  uint64_t s_ready[2];      /* scores S^T of buffer b computed */
+  uint64_t s_free[2];       /* S^T of buffer b read by every consumer warp */
+  uint64_t p_ready[2];      /* P^T of buffer b and the stage's bf16 V written by every consumer warp */
+  uint64_t pv_done[2];      /* the P.V products of buffer b completed */
+  uint64_t q_ready;         /* the segment's Q terms written */
+  uint64_t o_free;          /* the segment's output accumulator read */
+  volatile int ag_ready;    /* layer+1 whose attention key split (ag) the consumers computed */
+  float qfac[64];           /* per query row: softmax scale / its Q-term factor */
   int pos0[MSK_MAX_TOKENS];
   float lbuf[4][32][2];
   float red8[MSK_NCW];
@@ -108,6 +119,7 @@ struct Smem {
 };
 
 constexpr size_t SMEM_BYTES = 1024 + (size_t)MSK_NST * MSK_STAGE + MSK_SCR + sizeof(Smem);
+static_assert(SMEM_BYTES <= 232448, "227 KB of shared memory per CTA");
 
 /* ---- context ---------------------------------------------------------------------- */
 struct Ctx {
@@ -208,7 +220,7 @@ MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
  * (1024-byte aligned, four slots in the ring):
  * [GU_A]  codes of gate, up: one 128-row x 128-byte box each (256 codes per
  *         row), 128-byte swizzled — the K-major SW128 layout
- * [GU_AS] scales of gate, up: [128 rows][16] each
+ * [GU_AS] scales of gate, up: their scale-factor atoms [matrix][4 k steps][512 B]
  * [GU_B]  the unit's tokens' activation terms: token t at t*1024, its chunk's
  *         [8 core-matrix columns][8 term rows][16 B] (all term scales are 1) */
 constexpr int GU_KC = 256;
@@ -216,28 +228,28 @@ constexpr uint32_t GU_A = 0, GU_AS = 32768, GU_B = 36864, GU_SLOT = 45056;
 /* TMEM columns: two buffers of gate and up accumulators (128 lanes x 64
  * each), then the scale factors of two chunks in flight */
 constexpr uint32_t TM_D = 0, TM_DU = 64, TM_SFA = 256, TM_SFB = 384, TM_COLS = 512;
-/* scale-factor buffers: four chunks in flight, so that waiting for the
- * copies of chunk j-4 (a commit covers every earlier op) does not
- * serialise the consumers' staging with the tensor pipe */
+/* scale-factor buffers in TMEM: four chunks in rotation */
 constexpr int NSF = 4;
 constexpr uint32_t TM_SFA_BUF = 32; /* columns per buffer: 2 matrices x 4 steps x 4; SFB: 4 columns of ones */
-/* per-chunk staging of the scale factors in the interleaved block layout
- * (scratch region): SFA [matrix][k step][512 B], SFB [k step][512 B] */
-constexpr uint32_t SF_STAGE = 4096; /* SFA [matrix][4 k steps][512 B] */
-static_assert(NSF * SF_STAGE <= MSK_SCR, "scale staging fits the scratch region");
 static_assert(TM_SFA + NSF * TM_SFA_BUF <= TM_SFB && TM_SFB + 4 <= TM_COLS, "TMEM columns");
 
 struct XGeo {
   int K, KC, nkc, rows_unit, ngroups, NM, tma, ns;
   uint32_t cpitch, spitch, bpitch, mat_bytes, b_off, slot_bytes;
-  int a, b; /* this CTA's items [a, b) */
+  int u0;   /* first unit of the part */
+  int a, b; /* this CTA's items [a, b) of the part (item i: unit u0 + i / ngroups) */
 };
 
-MSK_DEV bool tc_experts(const MskParams* P) { return (P->flags & MSK_F_TC_EXPERTS) != 0; }
+/* some expert unit can take the block-scaled gate/up path */
+MSK_DEV bool tc_experts(const MskParams* P) { return P->tau <= MSK_UNIT_TOK; }
 
-MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
+/* the parts of an expert phase: gate/up of the block-scaled units, gate/up
+ * of the CUDA-core units, the down projection of every unit */
+enum { XP_TC = 0, XP_CC = 1, XP_DN = 2 };
+
+MSK_DEV void xgeo(const Ctx& c, int part, XGeo& x) {
   const MskParams* P = c.P;
-  const bool tc = gu && tc_experts(P);
+  const bool gu = part != XP_DN, tc = part == XP_TC;
   x.K = gu ? P->d : P->f;
   x.rows_unit = gu ? P->f : P->d;
   x.KC = tc ? GU_KC : (x.K <= XKC_MAX ? x.K : XKC_MAX);
@@ -252,7 +264,25 @@ MSK_DEV void xgeo(const Ctx& c, bool gu, XGeo& x) {
   x.slot_bytes = tc ? GU_SLOT : (x.b_off + MSK_UNIT_TOK * x.bpitch + 127) & ~127u;
   x.ns = min(XNS_MAX, (int)((uint32_t)(MSK_NST * MSK_STAGE) / x.slot_bytes));
   x.ngroups = x.rows_unit / XROWS;
-  item_range(c.S->route.n_units * x.ngroups, c.cta, c.ncta, &x.a, &x.b);
+  const Route& R = c.S->route;
+  x.u0 = part == XP_CC ? R.n_units_tc : 0;
+  const int nu = part == XP_TC ? R.n_units_tc : (part == XP_CC ? R.n_units - R.n_units_tc : R.n_units);
+  item_range(nu * x.ngroups, c.cta, c.ncta, &x.a, &x.b);
+}
+/* bit s set where the phase's fills of expert slot s are odd in number */
+MSK_DEV uint32_t fill_parity(const XGeo& x) {
+  const int n = (x.b - x.a) * x.nkc;
+  uint32_t m = 0;
+  for (int s = 0; s < x.ns; ++s)
+    if (((n / x.ns) + (s < n % x.ns ? 1 : 0)) & 1) m |= 1u << s;
+  return m;
+}
+/* the slot parities flipped by the fills of item i (0-based in this CTA's
+ * range): chunks i nkc .. (i+1) nkc - 1 of the phase */
+MSK_DEV uint32_t fill_parity_run(const XGeo& x, int i) {
+  uint32_t m = 0;
+  for (int j = i * x.nkc; j < (i + 1) * x.nkc; ++j) m ^= 1u << (j % x.ns);
+  return m;
 }
 /* gate+up with K = 512 is the largest slot: two must fit the ring */
 static_assert(2 * ((2 * XROWS * (XKC_MAX / 2 + 32 + XKC_MAX / 16) + MSK_UNIT_TOK * (2 * XKC_MAX + 16) + 127) & ~127) <=
@@ -372,10 +402,27 @@ MSK_DEV void for_each_att_stage(const Ctx& c, const AttGeo& g, F&& f) {
   }
 }
 
+/* tensor-core attention geometry (see attention_phase_tc) */
+constexpr uint32_t ATC_STAGE = 32768;
+constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64;
+MSK_DEV int atc_ns(int RP) { return RP > 32 ? 4 : 5; }
+MSK_DEV uint32_t atc_pt_off(int RP) { return (uint32_t)atc_ns(RP) * ATC_STAGE; }
+MSK_DEV uint32_t atc_q_off(int RP) { return atc_pt_off(RP) + 2u * (uint32_t)RP * 256u; }
+MSK_DEV int atc_rp(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 64); }
+static_assert(4 * ATC_STAGE + 2 * 64 * 256 + 3 * 64 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
+static_assert(5 * ATC_STAGE + 2 * 32 * 256 + 3 * 32 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
+/* instruction descriptors: fp32 accumulators, M = 128, N = RP; QK e4m3 x e4m3
+ * both K-major; PV bf16 x bf16 with A MN-major */
+MSK_DEV uint32_t atc_idesc_qk(int RP) { return (1u << 4) | ((uint32_t)(RP >> 3) << 17) | ((128u >> 4) << 24); }
+MSK_DEV uint32_t atc_idesc_pv(int RP) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(RP >> 3) << 17) | ((128u >> 4) << 24);
+}
+
 /* ---- producer ---------------------------------------------------------------------- */
 struct Prod {
   Ctx* c;
   uint32_t it;
+  uint32_t ait;   /* tensor-core attention stages issued */
   uint32_t xpar;  /* bit s: parity of the fills of expert slot s so far */
   uint32_t xused; /* bit s: expert slot s filled at least once */
   uint32_t dpar;  /* bit 2w+s: parity of the fills of warp w's dense slot s */
@@ -481,23 +528,24 @@ MSK_DEV void prefetch_dense(const Ctx& c, int layer, bool qkv) {
 /* Fill the expert ring for one phase: for each of this CTA's items and
  * each K chunk, the 128-row tiles of the unit's expert (gate and up, or
  * down) and the unit's activation rows, all on the slot's full barrier. */
-MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
+MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
   Ctx& c = *p.c;
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
   const Route& R = c.S->route;
+  const bool gu = part != XP_DN;
   const int phase = gu ? PH_GU : PH_DN;
   XGeo x;
-  xgeo(c, gu, x);
+  xgeo(c, part, x);
   const MskNv* mat[2] = {gu ? &Ly.wg : &Ly.wd, &Ly.wu};
   const CUtensorMap* cmap[2] = {Ly.emap + (gu ? 0 : 4), Ly.emap + 2};
   const CUtensorMap* smap[2] = {Ly.emap + (gu ? 1 : 5), Ly.emap + 3};
   const int lane = threadIdx.x & 31;
   int j = 0;
-  if (gu && tc_experts(P)) { /* block-scaled tensor cores: swizzled code boxes, raw scales, the tokens' terms */
+  if (part == XP_TC) { /* block-scaled tensor cores: swizzled code boxes, scale atoms, the tokens' terms */
     const size_t xqb = MSK_XQ_BYTES(P->d);
     for (int item = x.a; item < x.b; ++item) {
-      const int unit = item / x.ngroups, grp = item % x.ngroups;
+      const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups;
       const int n = R.unit_n[unit], st0 = R.unit_start[unit];
       const int64_t grow = (int64_t)R.unit_e[unit] * x.rows_unit + (int64_t)grp * XROWS;
       const int tl = lane - 8; /* lanes 8-15 copy token tl's terms */
@@ -517,9 +565,10 @@ MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
         __syncwarp();
         if (lane < 2) {
           tma_2d_g2s(dst + GU_A + lane * 16384, Ly.emap + MSK_MAP_GUSW + lane, kc * (GU_KC / 2), (int32_t)grow, bar);
-        } else if (lane == 4 || lane == 5) {
+        } else if (lane == 4 || lane == 5) { /* the chunk's scale-factor atoms, as the tensor core reads them */
           const int m = lane - 4;
-          tma_2d_g2s(dst + GU_AS + m * (XROWS * GU_KC / 16), smap[m], kc * (GU_KC / 16), (int32_t)grow, bar);
+          const int64_t atom = (grow / XROWS) * (P->d / 64) + (int64_t)kc * (GU_KC / 64);
+          bulk_g2s(dst + GU_AS + m * (XROWS * GU_KC / 16), (m ? Ly.sfu : Ly.sfg) + atom * 512, XROWS * GU_KC / 16, bar);
         } else if (tq) {
           bulk_g2s(dst + GU_B + tl * (8 * GU_KC / 2), tq + (size_t)kc * (8 * GU_KC / 2), 8 * GU_KC / 2, bar);
         }
@@ -531,7 +580,7 @@ MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
   const int act_ld = gu ? P->d : P->f;
   const uint32_t brow = (uint32_t)(2 * x.KC);
   for (int item = x.a; item < x.b; ++item) {
-    const int unit = item / x.ngroups, grp = item % x.ngroups;
+    const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
     const int64_t grow = (int64_t)R.unit_e[unit] * x.rows_unit + (int64_t)grp * XROWS;
     int my_row = 0; /* lanes 8.. : the activation row of the unit's entry lane-8 (token, or pair) */
@@ -568,19 +617,32 @@ MSK_DEV bool prod_experts(Prod& p, int layer, bool gu) {
   return true;
 }
 
+/* wait until the last fill of every expert slot has been released */
+MSK_DEV bool prod_xdrain(Prod& p, int layer) {
+  Ctx& c = *p.c;
+  for (int s = 0; s < XNS_MAX; ++s)
+    if (((p.xused >> s) & 1u) && !pwait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, PH_GU)) return false;
+  return true;
+}
+
 /* The MMA-issuing warp (one elected lane does the issuing): walks the same
  * gate/up chunk sequence as the consumers; per chunk it waits for the
  * consumers' scale staging, copies the scales into TMEM, issues the
  * block-scaled MMAs into the item's accumulator buffer (after the
  * consumers released that buffer) and commits (see expert_gu_tc). */
+MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg);
+
 MSK_DEV void issuer(Ctx& c) {
   const MskParams* P = c.P;
   const int lane = threadIdx.x & 31;
   const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(64 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
-  uint32_t bits = 0; /* 0-3 sfready parities, 4-5 dempty parities, 6-7 accumulator buffer used */
+  uint32_t bits = 0; /* 0-3 expert-slot fill parities, 4-5 dempty parities, 6-7 accumulator buffer used */
   bool ok = true;
   uint32_t tb = 0;
-  for (int l = 0; l < P->L && ok && tc_experts(P); ++l) {
+  uint32_t ait = 0, aseg = 0; /* attention stages and segments issued */
+  for (int l = 0; l < P->L && ok; ++l) {
+    if (P->hd == 128 && !issuer_att(c, l, ait, aseg)) { ok = false; break; }
+    if (!tc_experts(P)) continue;
     if (!pwait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { ok = false; break; }
     tb = c.S->tmem_base;
     if (l == 0) { /* the activation terms' block scales, all 1.0 (ue4m3 0x38), once */
@@ -593,25 +655,27 @@ MSK_DEV void issuer(Ctx& c) {
       }
       __syncwarp();
     }
-    XGeo x;
-    xgeo(c, true, x);
+    XGeo x, xc, xd;
+    xgeo(c, XP_TC, x);
+    xgeo(c, XP_CC, xc); /* (read while this layer's routing is current) */
+    xgeo(c, XP_DN, xd);
     const int nsteps = x.KC / 64;
-    const uint32_t ring = smem_u32(c.ring), sfs = smem_u32(c.scr);
+    const uint32_t ring = smem_u32(c.ring);
     int j = 0;
     for (int item = x.a; item < x.b && ok; ++item) {
       const int db = (item - x.a) & 1;
       for (int kc = 0; kc < x.nkc; ++kc, ++j) {
         const int s = j % x.ns, buf = j & (NSF - 1);
-        if (!pwait_bar(c, &c.S->sfready[buf], (bits >> buf) & 1u, l, PH_GU)) { ok = false; break; }
-        bits ^= 1u << buf;
+        if (!pwait_bar(c, &c.S->xfull[s], (bits >> s) & 1u, l, PH_GU)) { ok = false; break; }
+        bits ^= 1u << s;
         if (kc == 0 && ((bits >> (6 + db)) & 1u)) {
           if (!pwait_bar(c, &c.S->dempty2[db], (bits >> (4 + db)) & 1u, l, PH_GU)) { ok = false; break; }
           bits ^= 1u << (4 + db);
         }
         if (lane == 0) {
           tc_fence_after();
-          const uint32_t slot = ring + (uint32_t)s * x.slot_bytes, stg = sfs + (uint32_t)buf * SF_STAGE;
-          const uint64_t sd = umma_desc(stg, 16, 128, 0), ad = umma_desc(slot + GU_A, 16, 1024, 2),
+          const uint32_t slot = ring + (uint32_t)s * x.slot_bytes;
+          const uint64_t sd = umma_desc(slot + GU_AS, 16, 128, 0), ad = umma_desc(slot + GU_A, 16, 1024, 2),
                          bd = umma_desc(slot + GU_B, 128, 8 * GU_KC / 2, 0);
           const uint32_t sfa = tb + TM_SFA + buf * TM_SFA_BUF, sfb = tb + TM_SFB, dg = tb + TM_D + db * 128;
 #pragma unroll 1
@@ -625,13 +689,16 @@ MSK_DEV void issuer(Ctx& c) {
             tc_mma_nvf4(dg + TM_DU, a + (uint64_t)(16384 >> 4), b, idesc, acc, sfa + 16 + 4 * st, sfb);
           }
           tc_commit(&c.S->xempty[s]);
-          tc_commit(&c.S->sfdone[buf]);
           if (kc == x.nkc - 1) tc_commit(&c.S->dfull2[db]);
         }
         __syncwarp();
         if (kc == x.nkc - 1) bits |= 1u << (6 + db);
       }
     }
+    /* the producer fills the same slots for the CUDA-core units and the
+     * down projection: count those fills too, so the next layer's waits
+     * take the right parity */
+    bits ^= fill_parity(xc) ^ fill_parity(xd);
   }
   if (lane == 0) {
     tc_commit(&c.S->tfin);
@@ -640,11 +707,15 @@ MSK_DEV void issuer(Ctx& c) {
   }
 }
 
+MSK_DEV bool prod_att_tc(Prod& p, int layer, uint32_t& ait);
+MSK_DEV bool prod_att_tc_drain(Prod& p, int layer, uint32_t ait);
+
 MSK_DEV void producer(Ctx& c) {
   const MskParams* P = c.P;
   Prod p;
   p.c = &c;
   p.it = 0;
+  p.ait = 0;
   p.xpar = 0;
   p.xused = 0;
   p.dpar = 0;
@@ -662,6 +733,11 @@ MSK_DEV void producer(Ctx& c) {
     if (!pwait_flag(c, &c.S->dense_done, 2 * l + 1, l, PH_ATT)) { p.ok = false; break; }
     att_geo_warp(c, l, c.S->agp);
     const AttGeo& g = c.S->agp;
+    if (hd == 128) {
+      /* tensor-core attention: its own stage ring; W_o tiles once every
+       * stage's products have completed */
+      if (!prod_att_tc(p, l, p.ait) || !prod_att_tc_drain(p, l, p.ait)) { p.ok = false; break; }
+    } else
     for_each_att_stage(c, g, [&](int pr, int slot, int64_t k0, int n, bool, bool) {
       int b = pr / P->hkv, h = pr % P->hkv;
       if (k0 + C > c.S->pos0[b]) {
@@ -693,10 +769,17 @@ MSK_DEV void producer(Ctx& c) {
     }
     if (!pwait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { p.ok = false; break; }
     fence_proxy_async_global();
-    if (!prod_experts(p, l, true)) { p.ok = false; break; }
+    {
+      const Route& R = c.S->route;
+      if (R.n_units_tc > 0 && !prod_experts(p, l, XP_TC)) { p.ok = false; break; }
+      /* the CUDA-core units' slots are laid out differently: every
+       * block-scaled slot must be free first */
+      if (R.n_units_tc > 0 && R.n_units > R.n_units_tc && !prod_xdrain(p, l)) { p.ok = false; break; }
+      if (R.n_units > R.n_units_tc && !prod_experts(p, l, XP_CC)) { p.ok = false; break; }
+    }
     if (!pwait_flag(c, &c.S->dn_ready, l + 1, l, PH_DN)) { p.ok = false; break; }
     fence_proxy_async_global();
-    if (!prod_experts(p, l, false)) { p.ok = false; break; }
+    if (!prod_experts(p, l, XP_DN)) { p.ok = false; break; }
     if (!pwait_flag(c, &c.S->ring_free, l + 1, l, PH_DN)) { p.ok = false; break; }
   }
   if (!p.ok && (threadIdx.x & 31) == 0) {
@@ -723,6 +806,15 @@ MSK_DEV void producer(Ctx& c) {
       uint64_t t0 = gtimer();
       while (!mbar_try(&c.S->full[slot], (i / MSK_NST) & 1)) {
         if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+      }
+    }
+    if (hd == 128) {
+      const uint32_t ns = (uint32_t)atc_ns(atc_rp(c.st.Tq * P->G)), na = p.ait < ns ? p.ait : ns;
+      for (uint32_t i = p.ait - na; i < p.ait; ++i) {
+        uint64_t t0 = gtimer();
+        while (!mbar_try(&c.S->afull[i % ns], (i / ns) & 1)) {
+          if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+        }
       }
     }
   }
@@ -1163,6 +1255,323 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
   return R <= 16 ? attention_phase_mt<HD, 1>(q, layer) : attention_phase_mt<HD, 2>(q, layer);
 }
 
+/* ---- attention on the 5th-generation tensor cores (head dim 128) ------------------------ */
+/*
+ * Per (sequence, kv head) segment of keys, with R = Tq * G query rows padded
+ * to RP in {16, 32, 64}:
+ *   S^T[128 keys][RP] = K Q^T: tcgen05.mma kind::f8f6f4, A = the stage's K
+ *     exactly as the tensor copy lands it (e4m3, 128 keys x 128 bytes,
+ *     128-byte swizzle: the K-major canonical layout), B = Q as three e4m3
+ *     terms per value (q f = t0 + t1 + t2 with a power-of-two row factor f;
+ *     about 12 significant bits, as f16), the three term products
+ *     accumulated in TMEM: 3 x 4 MMAs of K = 32 per stage.
+ *   p = exp(s - M) under the key windows, on CUDA cores: each consumer
+ *     lane holds one key (TMEM lane), its rows' scores; l += p per lane;
+ *     P^T is written to shared memory as bf16 scaled by 2^120.
+ *   O^T[128 hd][RP] += V^T P^T: kind::f16 (bf16), A = the stage's V widened
+ *     in place to bf16 x 2^-120 (an exact bit move) and read MN-major
+ *     (head-dim contiguous, no transpose), B = P^T (K-major); 8 MMAs of
+ *     K = 16 keys per stage, accumulated in TMEM over the segment.
+ * The MMA-issuing warp runs one stage ahead: the QK products of stage j+1
+ * are in flight while the consumer warps turn the scores of stage j into
+ * probabilities.  Parties and barriers per stage j (buffer b = j mod 2):
+ *   producer -> afull -> issuer: QK(j) -> s_ready[b] -> consumers: widen V,
+ *   read S^T -> s_free[b] -> issuer (QK(j+2)); consumers: write P^T ->
+ *   p_ready[b] -> issuer: PV(j) -> aempty (stage refill) and pv_done[b]
+ *   (P^T buffer reuse; the segment's output read).
+ * Shared memory (from the ring base): NS stages of 32 KB (K at 0, V at 16 KB;
+ * after widening, bf16 V [key/8][hd/64][key%8][128 B], 128-byte swizzle),
+ * then two P^T buffers [2 key tiles][RP rows][128 B], then the Q terms
+ * [3][RP rows][128 B].  TMEM: O^T at column 0, S^T buffers at 64 and 128.
+ */
+/* The issuing warp's part of one layer's attention: this CTA's stages in
+ * the consumers' order; lane 0 issues.  ait / aseg: stages and segments
+ * issued so far (the consumers count the same). */
+MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31;
+  if (!pwait_flag(c, &c.S->ag_ready, layer + 1, layer, PH_ATT)) return false;
+  const AttGeo& g = c.S->ag;
+  const int RP = atc_rp(c.st.Tq * P->G), NS = atc_ns(RP);
+  const uint32_t tb = c.S->tmem_base, ring = smem_u32(c.ring);
+  const uint32_t qoff = ring + atc_q_off(RP), ptoff = ring + atc_pt_off(RP);
+  const uint32_t id_qk = atc_idesc_qk(RP), id_pv = atc_idesc_pv(RP);
+  bool ok = true;
+  auto qk = [&](uint32_t j) -> bool {
+    if (!pwait_bar(c, &c.S->afull[j % NS], (j / NS) & 1u, layer, PH_ATT)) return false;
+    if (j >= 2 && !pwait_bar(c, &c.S->s_free[j & 1u], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) return false;
+    if (lane == 0) {
+      tc_fence_after();
+      const uint32_t sk = ring + (j % NS) * ATC_STAGE, d = tb + ATC_TM_S + 64u * (j & 1u);
+#pragma unroll 1
+      for (int t = 0; t < 3; ++t)
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+          tc_mma_f8(d, umma_desc(sk + 32u * s, 16, 1024, 2), umma_desc(qoff + (uint32_t)(t * RP * 128 + 32 * s), 16, 1024, 2),
+                    id_qk, (t > 0 || s > 0) ? 1u : 0u);
+      tc_commit(&c.S->s_ready[j & 1u]);
+    }
+    __syncwarp();
+    return true;
+  };
+  auto pv = [&](uint32_t j, bool first) -> bool {
+    if (!pwait_bar(c, &c.S->p_ready[j & 1u], (j >> 1) & 1u, layer, PH_ATT)) return false;
+    if (first && aseg > 0 && !pwait_bar(c, &c.S->o_free, (aseg - 1u) & 1u, layer, PH_ATT)) return false;
+    if (lane == 0) {
+      tc_fence_after();
+      const uint32_t sv = ring + (j % NS) * ATC_STAGE, pt = ptoff + (j & 1u) * (uint32_t)RP * 256u;
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        tc_mma_f16(tb + ATC_TM_O, umma_desc(sv + 4096u * kk, 1024, 2048, 2),
+                   umma_desc(pt + (uint32_t)((kk >> 2) * RP * 128 + 32 * (kk & 3)), 16, 1024, 2), id_pv,
+                   (first && kk == 0) ? 0u : 1u);
+      tc_commit(&c.S->aempty[j % NS]);
+      tc_commit(&c.S->pv_done[j & 1u]);
+    }
+    __syncwarp();
+    return true;
+  };
+  for_each_att_stage(c, g, [&](int, int, int64_t, int, bool first, bool last) {
+    if (first) {
+      if (!pwait_bar(c, &c.S->q_ready, aseg & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (!qk(ait)) { ok = false; return false; }
+    }
+    if (!last && !qk(ait + 1)) { ok = false; return false; }
+    if (!pv(ait, first)) { ok = false; return false; }
+    ait++;
+    if (last) aseg++;
+    return true;
+  });
+  return ok;
+}
+
+/* The producer's part: this CTA's K and V boxes into the stage ring. */
+MSK_DEV bool prod_att_tc(Prod& p, int layer, uint32_t& ait) {
+  Ctx& c = *p.c;
+  const MskParams* P = c.P;
+  const AttGeo& g = c.S->agp;
+  const int RP = atc_rp(c.st.Tq * P->G), NS = atc_ns(RP);
+  const int lane = threadIdx.x & 31;
+  bool ok = true;
+  for_each_att_stage(c, g, [&](int pr, int, int64_t k0, int, bool, bool) {
+    const int b = pr / P->hkv, h = pr % P->hkv;
+    if (k0 + 128 > c.S->pos0[b]) {
+      if (!pwait_flag(c, &c.S->kv_ready, layer + 1, layer, PH_ATT)) { ok = false; return false; }
+      fence_proxy_async_global();
+    }
+    const uint32_t slot = ait % NS;
+    if (ait >= (uint32_t)NS && !pwait_bar(c, &c.S->aempty[slot], ((ait / NS) - 1u) & 1u, layer, PH_ATT)) {
+      ok = false;
+      return false;
+    }
+    uint8_t* stg = c.ring + (size_t)slot * ATC_STAGE;
+    uint64_t* bar = &c.S->afull[slot];
+    const int64_t row = (((int64_t)layer * c.st.kv_seqs + b) * P->hkv + h) * c.st.kv_cap + k0;
+    if (lane == 0) mbar_arrive_tx(bar, 2u * 128u * 128u);
+    __syncwarp();
+    if (lane == 0) tma_2d_g2s(stg, c.kvmap, 0, (int32_t)row, bar);
+    else if (lane == 1) tma_2d_g2s(stg + 16384, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), bar);
+    ait++;
+    return true;
+  });
+  return ok;
+}
+
+/* wait (bounded) until every tc attention stage issued so far is free again */
+MSK_DEV bool prod_att_tc_drain(Prod& p, int layer, uint32_t ait) {
+  Ctx& c = *p.c;
+  const int NS = atc_ns(atc_rp(c.st.Tq * c.P->G));
+  const uint32_t n = ait < (uint32_t)NS ? ait : (uint32_t)NS;
+  for (uint32_t i = ait - n; i < ait; ++i)
+    if (!pwait_bar(c, &c.S->aempty[i % NS], (i / NS) & 1u, layer, PH_WO)) return false;
+  return true;
+}
+
+/* Q of the pair's R rows as three e4m3 terms (B operand rows t RP + rho,
+ * 128-byte swizzle) and each row's softmax factor; one warp per row. */
+MSK_DEV void atc_q_terms(const Ctx& c, int pair, int RP, uint32_t qoff) {
+  const MskParams* P = c.P;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  const int b = pair / P->hkv, kvh = pair % P->hkv;
+  const int R = c.st.Tq * P->G;
+  for (int rho = cw; rho < RP; rho += NCW) {
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
+    if (rho < R) {
+      const int t = b * c.st.Tq + rho / P->G, h = kvh * P->G + rho % P->G;
+      const uint2 w = *reinterpret_cast<const uint2*>(P->qs + (size_t)t * P->qd + h * 128 + lane * 4);
+      x[0] = f16lo_f32(w.x); x[1] = f16hi_f32(w.x); x[2] = f16lo_f32(w.y); x[3] = f16hi_f32(w.y);
+    }
+    float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    /* f = 2^e with mx f in (224, 448] */
+    int e = 0;
+    if (mx > 0.f) e = max(-100, min(100, (int)floorf(log2f(448.0f / mx))));
+    const float f = __int_as_float((127 + e) << 23);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] *= f;
+    const uint32_t chunk = (uint32_t)(lane >> 2), within = 4u * (uint32_t)(lane & 3);
+#pragma unroll
+    for (int t = 0; t < 3; ++t) {
+      const uint32_t c01 = f32x2_to_e4m3x2(x[0], x[1]), c23 = f32x2_to_e4m3x2(x[2], x[3]);
+      x[0] -= e4m3_to_f32(c01);
+      x[1] -= e4m3_to_f32(c01 >> 8);
+      x[2] -= e4m3_to_f32(c23);
+      x[3] -= e4m3_to_f32(c23 >> 8);
+      const uint32_t n = (uint32_t)(t * RP + rho);
+      sts32(qoff + n * 128u + ((chunk ^ (n & 7u)) << 4) + within, c01 | (c23 << 16));
+    }
+    if (lane == 0) c.S->qfac[rho] = rho < R ? P->scale_log2 / f : 0.f;
+  }
+}
+
+template <int RP>
+MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  constexpr int NR = RP / 2; /* query rows per consumer warp */
+  constexpr int NS = RP > 32 ? 4 : 5;
+  att_geo_shared(c, layer);
+  if (threadIdx.x == CONS0) {
+    __threadfence_block();
+    c.S->ag_ready = layer + 1;
+  }
+  const AttGeo& g = c.S->ag;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, ctid = threadIdx.x - CONS0;
+  const int qd = cw & 3, hh = cw >> 2; /* TMEM lane quadrant (keys 32 qd ..), row half */
+  const int R = c.st.Tq * P->G;
+  const uint32_t ring = smem_u32(c.ring), tb = c.S->tmem_base;
+  const uint32_t ptoff = ring + atc_pt_off(RP), qoff = ring + atc_q_off(RP);
+  const float bound_log2 = Ly.bound_log2;
+  const float two120 = 1.329227995784916e36f; /* 2^120 */
+  const bool sliding = Ly.sliding != 0;
+  float* lred = reinterpret_cast<float*>(c.S->lbuf); /* [4 quadrants][64 rows] */
+  bool ok = true;
+  if (c.cta < g.nparts) {
+    const int64_t A0 = g.N * c.cta / g.nparts, B0 = g.N * (c.cta + 1) / g.nparts;
+    for (int pr = 0; pr < g.npairs; ++pr) {
+      const int64_t a = max(A0, g.off[pr]), bb = min(B0, g.off[pr + 1]);
+      if (a >= bb) continue;
+      const int k0 = (int)(g.lo[pr] + (a - g.off[pr])), k1 = (int)(g.lo[pr] + (bb - g.off[pr]));
+      const int b = pr / P->hkv;
+      const int T0 = c.S->pos0[b];
+      /* the window every valid row shares: [lo_max, hi_min] */
+      const int hi_min = T0, lo_max = sliding ? max(0, T0 + c.st.Tq - 1 - P->W + 1) : 0;
+      if (ok) atc_q_terms(c, pr, RP, qoff);
+      fence_proxy_async_shared();
+      named_sync(BAR_CONS, NCT);
+      if (ctid == 0) mbar_arrive(&c.S->q_ready);
+      float l[NR];
+#pragma unroll
+      for (int i = 0; i < NR; ++i) l[i] = 0.f;
+      for (int x = k0; x < k1; x += 128) {
+        const uint32_t j = ait, bf = j & 1u, slot = j % NS;
+        const int nkeys = min(128, k1 - x);
+        if (ok && j >= 2 && !wait_bar(c, &c.S->pv_done[bf], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) ok = false;
+        if (ok && !wait_bar(c, &c.S->afull[slot], (j / NS) & 1u, layer, PH_ATT)) ok = false;
+        if (ok && !wait_bar(c, &c.S->s_ready[bf], (j >> 1) & 1u, layer, PH_ATT)) ok = false;
+        ok = __all_sync(0xffffffffu, ok) != 0; /* warp-uniform: the TMEM loads below are warp-collective */
+        tc_fence_after();
+        /* V of the stage: 1024 16-byte chunks (key k, head-dim chunk ch), four
+         * per thread, read before any thread overwrites the stage */
+        const uint32_t sb = ring + slot * ATC_STAGE;
+        uint4 vv[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int ci = ctid + NCT * u, k = ci >> 3, ch = ci & 7;
+          vv[u] = ok ? lds128(sb + 16384u + (uint32_t)k * 128u + ((uint32_t)(ch ^ (k & 7)) << 4)) : make_uint4(0, 0, 0, 0);
+        }
+        named_sync(BAR_CONS, NCT);
+        if (ok) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int ci = ctid + NCT * u, k = ci >> 3, ch = ci & 7;
+            const uint32_t dst = sb + (uint32_t)(k >> 3) * 2048u + (uint32_t)(ch >> 2) * 1024u + (uint32_t)(k & 7) * 128u;
+            const uint32_t c0 = (uint32_t)(2 * (ch & 3)), c1 = c0 + 1u, sw = (uint32_t)(k & 7);
+            sts128(dst + ((c0 ^ sw) << 4), e4m3x2_to_bf16x2_scaled(vv[u].x, 0), e4m3x2_to_bf16x2_scaled(vv[u].x, 1),
+                   e4m3x2_to_bf16x2_scaled(vv[u].y, 0), e4m3x2_to_bf16x2_scaled(vv[u].y, 1));
+            sts128(dst + ((c1 ^ sw) << 4), e4m3x2_to_bf16x2_scaled(vv[u].z, 0), e4m3x2_to_bf16x2_scaled(vv[u].z, 1),
+                   e4m3x2_to_bf16x2_scaled(vv[u].w, 0), e4m3x2_to_bf16x2_scaled(vv[u].w, 1));
+          }
+        }
+        /* this warp's scores: its quadrant's 32 keys, its NR rows */
+        uint32_t sr[NR];
+        if (ok) {
+          const uint32_t ta = tb + ATC_TM_S + 64u * bf + (uint32_t)(hh * NR) + ((uint32_t)(qd * 32) << 16);
+#pragma unroll
+          for (int i = 0; i < NR; i += 8) tc_ld8(ta + (uint32_t)i, sr + i);
+          tc_wait_ld();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.S->s_free[bf]);
+        if (ok) {
+          const int key = qd * 32 + lane, kp = x + key;
+          const bool full = nkeys == 128 && x >= lo_max && x + 127 <= hi_min;
+          const uint32_t pt = ptoff + bf * (uint32_t)RP * 256u + (uint32_t)(key >> 6) * (uint32_t)RP * 128u;
+          const uint32_t kk = (uint32_t)(key & 63);
+#pragma unroll
+          for (int i = 0; i < NR; ++i) {
+            const int rho = hh * NR + i;
+            float pv = 0.f;
+            if (rho < R) {
+              bool valid = full;
+              if (!full) {
+                const int hi = T0 + rho / P->G, lo = sliding ? max(0, hi - P->W + 1) : 0;
+                valid = key < nkeys && kp >= lo && kp <= hi;
+              }
+              if (valid) pv = fast_exp2(__uint_as_float(sr[i]) * c.S->qfac[rho] - bound_log2);
+            }
+            l[i] += pv;
+            sts16(pt + (uint32_t)rho * 128u + (((kk >> 3) ^ ((uint32_t)rho & 7u)) << 4) + 2u * (kk & 7u),
+                  f32_to_bf16(pv * two120));
+          }
+        }
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&c.S->p_ready[bf]);
+        ait++;
+      }
+      /* segment end: the output accumulator after the last stage's products */
+      const uint32_t jl = ait - 1u;
+      if (ok && !wait_bar(c, &c.S->pv_done[jl & 1u], (jl >> 1) & 1u, layer, PH_ATT)) ok = false;
+      ok = __all_sync(0xffffffffu, ok) != 0;
+      tc_fence_after();
+      const int slotp = c.cta + pr;
+      float* base = P->part + (size_t)slotp * P->part_stride;
+      if (ok) {
+        uint32_t orr[NR];
+        const uint32_t ta = tb + ATC_TM_O + (uint32_t)(hh * NR) + ((uint32_t)(qd * 32) << 16);
+#pragma unroll
+        for (int i = 0; i < NR; i += 8) tc_ld8(ta + (uint32_t)i, orr + i);
+        tc_wait_ld();
+#pragma unroll
+        for (int i = 0; i < NR; ++i) {
+          const int rho = hh * NR + i;
+          if (rho < R) base[(size_t)rho * (128 + 4) + qd * 32 + lane] = __uint_as_float(orr[i]);
+        }
+      }
+      /* row sums: over the warp's 32 keys, then the four quadrants */
+#pragma unroll
+      for (int i = 0; i < NR; ++i) {
+        float v = l[i];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) lred[qd * 64 + hh * NR + i] = v;
+      }
+      tc_fence_before();
+      named_sync(BAR_CONS, NCT);
+      if (ctid < R && ok)
+        base[(size_t)ctid * (128 + 4) + 128] = lred[ctid] + lred[64 + ctid] + lred[128 + ctid] + lred[192 + ctid];
+      if (ctid == 0) mbar_arrive(&c.S->o_free);
+      aseg++;
+      named_sync(BAR_CONS, NCT); /* lred reused by the next segment */
+    }
+  }
+  if (!ok) c.S->abort = 1;
+  return !named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
+}
+
 /* ---- consumer: small phases (warp per item over the whole grid) --------------------- */
 MSK_DEV int gwarp(const Ctx& c) { return c.cta * NCW + (threadIdx.x >> 5) - CONS_WARP0; }
 MSK_DEV int nwarps(const Ctx& c) { return c.ncta * NCW; }
@@ -1408,12 +1817,8 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
       }
     }
     const float r = 1.0f / sqrtf(cta_sum(c, ss) / d + P->eps);
-    if (tc_experts(P)) {
-      row_norm_store(v, d, r, P->layers[layer].g_moe, nullptr, P->x2f + (size_t)t * d);
-      row_quant8(c, v, d, r, P->layers[layer].g_moe, P->xq + (size_t)t * MSK_XQ_BYTES(d));
-    } else {
-      row_norm_store(v, d, r, P->layers[layer].g_moe, P->x2h + (size_t)t * d, P->x2f + (size_t)t * d);
-    }
+    row_norm_store(v, d, r, P->layers[layer].g_moe, P->x2h + (size_t)t * d, P->x2f + (size_t)t * d);
+    if (tc_experts(P)) row_quant8(c, v, d, r, P->layers[layer].g_moe, P->xq + (size_t)t * MSK_XQ_BYTES(d));
   }
 }
 
@@ -1587,27 +1992,44 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
       const int pi = base + lane;
       if (pi < np) R.pairs[R.start[R.ids[pi]] + rank_local[ch]] = (int16_t)pi;
     }
-    /* units: experts with tokens, split into groups of <= MSK_UNIT_TOK */
-    int nu = 0, nd = 0;
+    /* units: experts with tokens, split into groups of <= MSK_UNIT_TOK;
+     * the units with at least tau tokens (block-scaled gate/up) first, in
+     * expert order, then the others */
+    const int tau = P->tau;
+    auto tc_units = [tau](int n) {
+      const int full = n / MSK_UNIT_TOK, rem = n % MSK_UNIT_TOK;
+      return (MSK_UNIT_TOK >= tau ? full : 0) + (rem > 0 && rem >= tau ? 1 : 0);
+    };
+    int ntc = 0;
+    for (int base = 0; base < E; base += 32) {
+      int v = tc_units(R.cnt[base + lane]);
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      ntc += v;
+    }
+    int nu = 0, nt = 0, nd = 0;
     for (int base = 0; base < E; base += 32) {
       const int e = base + lane, n = R.cnt[e];
-      const int mine = (n + MSK_UNIT_TOK - 1) / MSK_UNIT_TOK;
-      int x = mine;
+      const int mine = (n + MSK_UNIT_TOK - 1) / MSK_UNIT_TOK, mt = tc_units(n), mc = mine - mt;
+      int xt = mt, xc = mc;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+        const int yt = __shfl_up_sync(0xffffffffu, xt, o), yc = __shfl_up_sync(0xffffffffu, xc, o);
+        if (lane >= o) { xt += yt; xc += yc; }
       }
-      const int first = nu + x - mine;
+      int pt = nt + xt - mt, pc = ntc + (nu - nt) + xc - mc;
       for (int u = 0; u < mine; ++u) {
-        R.unit_e[first + u] = (int16_t)e;
-        R.unit_start[first + u] = (int16_t)(R.start[e] + u * MSK_UNIT_TOK);
-        R.unit_n[first + u] = (int16_t)min(MSK_UNIT_TOK, n - u * MSK_UNIT_TOK);
+        const int un = min(MSK_UNIT_TOK, n - u * MSK_UNIT_TOK);
+        const int at = un >= tau ? pt++ : pc++;
+        R.unit_e[at] = (int16_t)e;
+        R.unit_start[at] = (int16_t)(R.start[e] + u * MSK_UNIT_TOK);
+        R.unit_n[at] = (int16_t)un;
       }
-      nu += __shfl_sync(0xffffffffu, x, 31);
+      nt += __shfl_sync(0xffffffffu, xt, 31);
+      nu += __shfl_sync(0xffffffffu, xt + xc, 31);
       nd += __popc(__ballot_sync(0xffffffffu, n > 0));
     }
-    if (lane == 0) { R.n_units = nu; R.n_distinct = nd; }
+    if (lane == 0) { R.n_units = nu; R.n_units_tc = nt; R.n_distinct = nd; }
   }
   named_sync(BAR_CONS, NCT);
   if (c.cta == 0) {
@@ -1725,69 +2147,40 @@ MSK_DEV void xgemm(uint32_t codes, uint32_t scales, uint32_t mstride, uint32_t c
 
 /* Gate/up of the selected experts on the block-scaled tensor cores
  * (tcgen05.mma kind::mxf4nvf4, M = 128 weight rows, N = 8 tokens x 8 term
- * rows, K = 64 per instruction, fp32 accumulators in TMEM).  Three parties
- * per chunk: the producer warp lands the slot; each consumer warp lays its
- * share of the chunk's scales out in the interleaved block layout the
- * scale-factor copies read (staging buffer j mod 4) and arrives on
- * sfready; the issuing warp then copies the scales into TMEM, issues the
- * MMAs and commits to the slot's empty barrier, the staging barrier and,
- * after an item's last chunk, to that item's accumulator buffer (two
- * buffers, so an item's epilogue overlaps the next item's MMAs).  The
- * epilogue reads the accumulators (TMEM lane = weight row), sums each
- * token's four term columns, undoes the token's power-of-two factor and
- * applies the global scales and SwiGLU.
- * xpar: bits 0-3 weight-slot parities; 4-7 parity of the chunks handed
- * to each staging buffer, 8-11 whether any was; 12-13 accumulator-buffer
- * parities. */
+ * rows, K = 64 per instruction, fp32 accumulators in TMEM).  The producer
+ * lands each chunk's codes, its scale-factor atoms (repacked once by
+ * msk_create into the layout the scale copies read) and the unit's
+ * activation terms; the issuing warp copies the scales into TMEM, issues
+ * the MMAs, commits the slot back to the producer and, after an item's last
+ * chunk, to that item's accumulator buffer (two buffers, so an item's
+ * epilogue overlaps the next item's MMAs).  The consumer warps only run the
+ * epilogue: read the accumulators (TMEM lane = weight row), sum each token's
+ * eight term columns, undo the token's power-of-two factor, apply the global
+ * scales and SwiGLU.
+ * xpar: bits 0-3 weight-slot fill parities (the issuer waits for the fills;
+ * the consumers count them, for the down projection's waits); 12-13
+ * accumulator-buffer parities. */
 MSK_DEV bool expert_gu_tc(Ctx& c, int layer, uint32_t& xpar) {
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
   const Route& R = c.S->route;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
   XGeo x;
-  xgeo(c, true, x);
-  const int f = P->f, nsteps = x.KC / 64;
+  xgeo(c, XP_TC, x);
+  const int f = P->f;
   const float gs0 = Ly.wg.gs, gs1 = Ly.wu.gs;
   const size_t xqb = MSK_XQ_BYTES(P->d);
-  const uint32_t ring = smem_u32(c.ring), sfs = smem_u32(c.scr);
   const uint32_t tb = c.S->tmem_base;
   const int q = (threadIdx.x >> 5) & 3, th = cw >> 2; /* TMEM lane quadrant, token half of the epilogue */
   bool ok = true;
-  int j = 0;
   for (int item = x.a; item < x.b; ++item) {
-    const int unit = item / x.ngroups, grp = item % x.ngroups, db = (item - x.a) & 1;
+    const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups, db = (item - x.a) & 1;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
-    for (int kc = 0; kc < x.nkc; ++kc, ++j) {
-      const int s = j % x.ns, buf = j & (NSF - 1);
-      const uint32_t slot = ring + (uint32_t)s * x.slot_bytes, stg = sfs + (uint32_t)buf * SF_STAGE;
-      if (ok && !wait_bar(c, &c.S->xfull[s], (xpar >> s) & 1u, layer, PH_GU)) ok = false;
-      xpar ^= 1u << s;
-      /* the scale copies last issued from this staging buffer must be done */
-      if (ok && ((xpar >> (8 + buf)) & 1u) &&
-          !wait_bar(c, &c.S->sfdone[buf], ((xpar >> (4 + buf)) & 1u) ^ 1u, layer, PH_GU))
-        ok = false;
-      if (!ok) continue;
-      /* this warp's share: SFA block (m, k step st), 16-byte row r0 = rows
-       * r0 + 32 m1 (m1 = 0..3), 4 scales each */
-      for (int u = cw * 32 + lane; u < 2 * nsteps * 32; u += NCT) {
-        const int blk = u / 32, r0 = u % 32;
-        const int m = blk / nsteps, st = blk % nsteps;
-        const uint32_t src = slot + GU_AS + m * (XROWS * GU_KC / 16) + 4 * st;
-        uint32_t wv[4];
-#pragma unroll
-        for (int m1 = 0; m1 < 4; ++m1) wv[m1] = lds32(src + (r0 + 32 * m1) * (GU_KC / 16));
-        asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(stg + (m * 4 + st) * 512 + r0 * 16), "r"(wv[0]),
-                     "r"(wv[1]), "r"(wv[2]), "r"(wv[3]));
-      }
-      fence_proxy_async_shared();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&c.S->sfready[buf]);
-      xpar ^= 1u << (4 + buf);
-      xpar |= 1u << (8 + buf);
-    }
+    xpar ^= fill_parity_run(x, item - x.a);
     const uint32_t dp = (xpar >> (12 + db)) & 1u;
     xpar ^= 1u << (12 + db);
     if (ok && !wait_bar(c, &c.S->dfull2[db], dp, layer, PH_GU)) ok = false;
+    ok = __all_sync(0xffffffffu, ok) != 0; /* warp-uniform: the TMEM loads below are warp-collective */
     if (!ok) continue;
     tc_fence_after();
     uint32_t gr[32], ur[32];
@@ -1836,7 +2229,7 @@ MSK_DEV bool expert_mma(Ctx& c, int layer, uint32_t& xpar) {
   const int ctid = threadIdx.x - CONS0;
   const int phase = GU ? PH_GU : PH_DN;
   XGeo x;
-  xgeo(c, GU, x);
+  xgeo(c, GU ? XP_CC : XP_DN, x);
   const int d = P->d, f = P->f;
   const float gs0 = GU ? Ly.wg.gs : Ly.wd.gs, gs1 = Ly.wu.gs;
   const uint32_t ring = smem_u32(c.ring);
@@ -1844,7 +2237,7 @@ MSK_DEV bool expert_mma(Ctx& c, int layer, uint32_t& xpar) {
   int j = 0;
   bool ok = true;
   for (int item = x.a; item < x.b; ++item) {
-    const int unit = item / x.ngroups, grp = item % x.ngroups;
+    const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups;
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[0][e] = acc[1][e] = acc2[0][e] = acc2[1][e] = 0.f;
     for (int kc = 0; kc < x.nkc; ++kc, ++j) {
@@ -1888,6 +2281,7 @@ MSK_DEV void consumer(Ctx& c) {
   q.it = 0;
   uint32_t xpar = 0; /* this warp's expert-slot parities */
   uint32_t dpar = 0; /* this warp's dense-slot and activation-slice parities */
+  uint32_t ait = 0, aseg = 0; /* tensor-core attention stages and segments consumed */
   phase_in(c);
   if (!grid_sync(c, 0, PH_IN)) return;
   for (int l = 0; l < P->L; ++l) {
@@ -1896,7 +2290,14 @@ MSK_DEV void consumer(Ctx& c) {
     phase_qknorm(c, l);
     if (!grid_sync(c, l, PH_QKNORM)) return;
     if (threadIdx.x == CONS0) c.S->kv_ready = l + 1;
-    bool ok = attention_phase<HD>(q, l);
+    bool ok;
+    if constexpr (HD == 128) {
+      const int RP = atc_rp(c.st.Tq * P->G);
+      ok = RP == 16 ? attention_phase_tc<16>(c, l, ait, aseg)
+                    : (RP == 32 ? attention_phase_tc<32>(c, l, ait, aseg) : attention_phase_tc<64>(c, l, ait, aseg));
+    } else {
+      ok = attention_phase<HD>(q, l);
+    }
     if (!ok) return;
     if (!grid_sync(c, l, PH_ATT)) return;
     phase_attc(c, l);
@@ -1908,7 +2309,8 @@ MSK_DEV void consumer(Ctx& c) {
     phase_router(c, l);
     if (!grid_sync(c, l, PH_ROUTER)) return;
     if (!phase_topk(c, l, dpar)) return;
-    if (!(tc_experts(P) ? expert_gu_tc(c, l, xpar) : expert_mma<true>(c, l, xpar))) return;
+    if (tc_experts(P) && !expert_gu_tc(c, l, xpar)) return;
+    if (!expert_mma<true>(c, l, xpar)) return;
     if (!grid_sync(c, l, PH_GU)) return;
     if (threadIdx.x == CONS0) c.S->dn_ready = l + 1;
     if (!expert_mma<false>(c, l, xpar)) return;
@@ -1959,15 +2361,24 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
       mbar_init(&c.S->xfull[i], 1);
       mbar_init(&c.S->xempty[i], 1);
     }
-    for (int i = 0; i < NSF; ++i) {
-      mbar_init(&c.S->sfdone[i], 1);
-      mbar_init(&c.S->sfready[i], NCW);
-    }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.S->dfull2[i], 1);
       mbar_init(&c.S->dempty2[i], NCW);
     }
     mbar_init(&c.S->tfin, 1);
+    for (int i = 0; i < 5; ++i) {
+      mbar_init(&c.S->afull[i], 1);
+      mbar_init(&c.S->aempty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&c.S->s_ready[i], 1);
+      mbar_init(&c.S->s_free[i], NCW);
+      mbar_init(&c.S->p_ready[i], NCW);
+      mbar_init(&c.S->pv_done[i], 1);
+    }
+    mbar_init(&c.S->q_ready, 1);
+    mbar_init(&c.S->o_free, 1);
+    c.S->ag_ready = 0;
     c.S->issuer_done = 0;
     mbar_fence_init();
   }
@@ -2033,8 +2444,32 @@ __global__ void msk_kv_encode_tail(const float* __restrict__ in, uint8_t* __rest
   if (i < n) out[i] = (uint8_t)f32x2_to_e4m3x2(in[i], 0.f);
 }
 
+/* NVFP4 block scales [rows][k16] (k16 = K/16, rows a multiple of 128, k16 a
+ * multiple of 4) -> the block-scaled tensor cores' scale-factor atoms
+ * [rows/128][k16/4][512 B]: byte 16 r + 4 m + b of atom (g, s) is the scale
+ * of row 128 g + r + 32 m, block 4 s + b.  One 4-byte word per thread. */
+__global__ void msk_sf_repack_kernel(const uint8_t* __restrict__ in, uint32_t* __restrict__ out, int64_t nwords,
+                                     int k16) {
+  const int S = k16 / 4;
+  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords; w += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t a = w >> 7;
+    const int i = (int)(w & 127), r0 = i >> 2, m1 = i & 3;
+    const int64_t g = a / S, st = a - g * S;
+    const int64_t row = g * 128 + r0 + 32 * m1;
+    out[w] = *reinterpret_cast<const uint32_t*>(in + row * k16 + 4 * st);
+  }
+}
+
 /* ---- launch ---------------------------------------------------------------------------- */
 extern "C" size_t msk_kernel_smem_bytes() { return SMEM_BYTES; }
+
+extern "C" cudaError_t msk_kernel_sf_repack(const uint8_t* in, uint8_t* out, int64_t rows, int k16, cudaStream_t st) {
+  const int64_t nwords = rows * k16 / 4;
+  const int64_t blocks = (nwords + 255) / 256;
+  msk_sf_repack_kernel<<<(unsigned)(blocks < 148 * 32 ? blocks : 148 * 32), 256, 0, st>>>(
+      in, reinterpret_cast<uint32_t*>(out), nwords, k16);
+  return cudaGetLastError();
+}
 
 extern "C" cudaError_t msk_kernel_kv_encode(const float* in, uint8_t* out, int64_t n, cudaStream_t stream) {
   const int64_t n4 = n / 4;
