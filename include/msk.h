@@ -92,8 +92,9 @@ typedef struct msk_config {
                              cores, the others on the CUDA-core path (the
                              post's "Expert Weight Quantization": NVFP4 GEMV
                              at one token, a dense contraction where several
-                             tokens share an expert).  0 = never (unless
-                             MSK_F_TC_EXPERTS), 1 = always */
+                             tokens share an expert).  0 = the library's
+                             default, MSK_TAU_DEFAULT; above 8 = never (the
+                             CUDA-core path for every unit); 1 = always */
 } msk_config_t;
 
 #define MSK_F_TRACE 1u /* record per-phase %globaltimer stamps (msk_query) */
@@ -104,6 +105,11 @@ typedef struct msk_config {
  * activations as eight e2m1 terms (relative error ~1e-5 of the row's
  * largest value). */
 #define MSK_F_TC_EXPERTS 2u
+/* expert_mma_min_tokens when the config leaves it 0: every unit on the
+ * block-scaled tensor cores (measured faster than the CUDA-core decode at
+ * every unit size the workloads produce, 1-8 tokens) */
+#define MSK_TAU_DEFAULT 1
+#define MSK_TAU_NEVER 0x7FFFFFFF
 
 /* Per-layer weights, all device pointers, borrowed.
  *  attn_norm_g [d], moe_norm_g [d]      RMSNorm gains (fp32)

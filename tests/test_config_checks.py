@@ -70,6 +70,7 @@ CASES = [
     ("more than 64 tokens", dict(max_seqs=16, max_tokens_per_seq=5), UNSUPPORTED),
     ("query rows per kv head above 64", dict(max_seqs=1, max_tokens_per_seq=9), UNSUPPORTED),
     ("negative wait limit", dict(wait_timeout_us=-1), INVALID),
+    ("negative expert token threshold", dict(expert_mma_min_tokens=-1), INVALID),
 ]
 
 

@@ -68,6 +68,20 @@ def test_parity_tensor_core_experts(name):
 
 
 @pytest.mark.parametrize("name", ["tiny", "dec8", "ver8"])
+def test_parity_cuda_core_experts(name):
+    """Every expert unit's gate/up on the CUDA-core path (tau above the unit size)."""
+    w = synth.WORKLOADS[name]
+    eng = Engine(w, tau=msk.TAU_NEVER)
+    eng.fill_past()
+    hid = sg.hidden(w)
+    rep, gpu, ref = run_parity(w, eng, hid, w.positions())
+    _report(name + " cc", rep)
+    assert_parity(rep)
+    assert msk.msk_query(eng.h).repacked_bytes == 0
+    eng.close()
+
+
+@pytest.mark.parametrize("name", ["tiny", "dec8", "ver8"])
 def test_parity_workload(name):
     w = synth.WORKLOADS[name]
     eng = Engine(w)
@@ -105,11 +119,11 @@ RAGGED = Workload("ragged", 3, 256, 4, 2, 64, 128, [1, 0, 1], 3, 3, 0, 0x5EED + 
                   window=100)
 
 
-@pytest.mark.parametrize("flags", [0, msk.F_TC_EXPERTS], ids=["cuda_core", "tensor_core"])
-def test_parity_ragged_sequences(flags):
+@pytest.mark.parametrize("tau", [msk.TAU_NEVER, 1], ids=["cuda_core", "tensor_core"])
+def test_parity_ragged_sequences(tau):
     w = RAGGED
     past = [0, 130, 517]  # empty past, a chunk boundary crossed, window < context
-    eng = Engine(w, past_per_seq=past, flags=flags)
+    eng = Engine(w, past_per_seq=past, tau=tau)
     eng.fill_past()
     hid = sg.hidden(w)
     pos = [[p + i for i in range(w.tokens_per_seq)] for p in past]

@@ -44,10 +44,10 @@ def _held_step(eng, hid, pos, n):
     return msk.msk_step_status_at(eng.h)
 
 
-@pytest.mark.parametrize("flags", [0, msk.F_TC_EXPERTS], ids=["cuda_core", "tensor_core"])
-def test_withheld_barrier_times_out_and_the_next_step_is_exact(flags):
+@pytest.mark.parametrize("tau", [msk.TAU_NEVER, 1], ids=["cuda_core", "tensor_core"])
+def test_withheld_barrier_times_out_and_the_next_step_is_exact(tau):
     w = synth.WORKLOADS["tiny"]
-    eng = Engine(w, timeout_us=20000, flags=flags)
+    eng = Engine(w, timeout_us=20000, tau=tau)
     try:
         eng.fill_past()
         hid = sg.hidden(w)

@@ -18,6 +18,8 @@ STATUS = {0: "MSK_OK", 1: "MSK_ERR_INVALID_ARG", 2: "MSK_ERR_UNSUPPORTED", 3: "M
           5: "MSK_ERR_BOUND", 6: "MSK_ERR_KV_RANGE", 7: "MSK_ERR_TIMEOUT", 8: "MSK_ERR_DEVICE"}
 F_TRACE = 1
 F_TC_EXPERTS = 2  # gate/up on the block-scaled tensor cores
+TAU_DEFAULT = 1  # expert_mma_min_tokens when 0 is passed
+TAU_NEVER = 0x7FFFFFFF  # every unit's gate/up on the CUDA-core path
 
 
 class MskError(RuntimeError):

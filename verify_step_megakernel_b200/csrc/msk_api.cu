@@ -257,9 +257,9 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   P.scale_log2 = (float)(1.4426950408889634 / sqrt((double)P.hd));
   P.timeout_ns = (int64_t)(c.wait_timeout_us ? c.wait_timeout_us : 2000000) * 1000;
   P.flags = c.flags;
-  /* tau: 0 = never (2^30), MSK_F_TC_EXPERTS = every unit */
-  P.tau = (c.flags & MSK_F_TC_EXPERTS) ? 1 : (c.expert_mma_min_tokens > 0 ? c.expert_mma_min_tokens : (1 << 30));
-  if (P.tau < 1) P.tau = 1;
+  /* tau: 0 = the default, above the unit size = never, MSK_F_TC_EXPERTS = every unit */
+  P.tau = (c.flags & MSK_F_TC_EXPERTS) ? 1 : (c.expert_mma_min_tokens > 0 ? c.expert_mma_min_tokens : MSK_TAU_DEFAULT);
+  if (P.tau > MSK_UNIT_TOK) P.tau = MSK_TAU_NEVER;
 
   /* the fixed softmax shift of each layer, from its QK-norm gains */
   float* gq = (float*)malloc(sizeof(float) * P.hd);

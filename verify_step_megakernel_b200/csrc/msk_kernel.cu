@@ -404,7 +404,7 @@ MSK_DEV void for_each_att_stage(const Ctx& c, const AttGeo& g, F&& f) {
 
 /* tensor-core attention geometry (see attention_phase_tc) */
 constexpr uint32_t ATC_STAGE = 32768;
-constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64;
+constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64, ATC_TM_SSTRIDE = 192;
 MSK_DEV int atc_ns(int RP) { return RP > 32 ? 4 : 5; }
 MSK_DEV uint32_t atc_pt_off(int RP) { return (uint32_t)atc_ns(RP) * ATC_STAGE; }
 MSK_DEV uint32_t atc_q_off(int RP) { return atc_pt_off(RP) + 2u * (uint32_t)RP * 256u; }
@@ -413,7 +413,7 @@ static_assert(4 * ATC_STAGE + 2 * 64 * 256 + 3 * 64 * 128 <= MSK_NST * MSK_STAGE
 static_assert(5 * ATC_STAGE + 2 * 32 * 256 + 3 * 32 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
 /* instruction descriptors: fp32 accumulators, M = 128, N = RP; QK e4m3 x e4m3
  * both K-major; PV bf16 x bf16 with A MN-major */
-MSK_DEV uint32_t atc_idesc_qk(int RP) { return (1u << 4) | ((uint32_t)(RP >> 3) << 17) | ((128u >> 4) << 24); }
+MSK_DEV uint32_t atc_idesc_qk(int RP) { return (1u << 4) | ((uint32_t)((3 * RP) >> 3) << 17) | ((128u >> 4) << 24); }
 MSK_DEV uint32_t atc_idesc_pv(int RP) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(RP >> 3) << 17) | ((128u >> 4) << 24);
 }
@@ -645,21 +645,22 @@ MSK_DEV void issuer(Ctx& c) {
     if (!tc_experts(P)) continue;
     if (!pwait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { ok = false; break; }
     tb = c.S->tmem_base;
-    if (l == 0) { /* the activation terms' block scales, all 1.0 (ue4m3 0x38), once */
+    /* the activation terms' block scales, all 1.0 (ue4m3 0x38), into TMEM
+     * each layer (the attention phase reuses those columns) */
+    if (l == 0) {
       c.S->sfb_one[lane] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
       fence_proxy_async_shared();
       __syncwarp();
-      if (lane == 0) {
-        tc_fence_after();
-        tc_cp_sf(tb + TM_SFB, umma_desc(smem_u32(c.S->sfb_one), 16, 128, 0));
-      }
-      __syncwarp();
     }
+    if (lane == 0) {
+      tc_fence_after();
+      tc_cp_sf(tb + TM_SFB, umma_desc(smem_u32(c.S->sfb_one), 16, 128, 0));
+    }
+    __syncwarp();
     XGeo x, xc, xd;
     xgeo(c, XP_TC, x);
     xgeo(c, XP_CC, xc); /* (read while this layer's routing is current) */
     xgeo(c, XP_DN, xd);
-    const int nsteps = x.KC / 64;
     const uint32_t ring = smem_u32(c.ring);
     int j = 0;
     for (int item = x.a; item < x.b && ok; ++item) {
@@ -678,15 +679,15 @@ MSK_DEV void issuer(Ctx& c) {
           const uint64_t sd = umma_desc(slot + GU_AS, 16, 128, 0), ad = umma_desc(slot + GU_A, 16, 1024, 2),
                          bd = umma_desc(slot + GU_B, 128, 8 * GU_KC / 2, 0);
           const uint32_t sfa = tb + TM_SFA + buf * TM_SFA_BUF, sfb = tb + TM_SFB, dg = tb + TM_D + db * 128;
-#pragma unroll 1
-          for (int st = 0; st < 2 * nsteps; ++st) tc_cp_sf(sfa + 4 * st, sd + (uint64_t)((st * 512) >> 4));
-#pragma unroll 1
-          for (int st = 0; st < nsteps; ++st) {
+          /* descriptors advance by adding to their address field (16-byte units) */
+#pragma unroll
+          for (int st = 0; st < 2 * (GU_KC / 64); ++st) tc_cp_sf(sfa + 4 * st, sd + (uint64_t)(st * 32));
+#pragma unroll
+          for (int st = 0; st < GU_KC / 64; ++st) {
             const uint32_t acc = (kc > 0 || st > 0) ? 1u : 0u;
-            const uint64_t b = bd + (uint64_t)((256 * st) >> 4);
-            const uint64_t a = ad + (uint64_t)((32 * st) >> 4);
+            const uint64_t b = bd + (uint64_t)(16 * st), a = ad + (uint64_t)(2 * st);
             tc_mma_nvf4(dg, a, b, idesc, acc, sfa + 4 * st, sfb);
-            tc_mma_nvf4(dg + TM_DU, a + (uint64_t)(16384 >> 4), b, idesc, acc, sfa + 16 + 4 * st, sfb);
+            tc_mma_nvf4(dg + TM_DU, a + 1024u, b, idesc, acc, sfa + 16 + 4 * st, sfb);
           }
           tc_commit(&c.S->xempty[s]);
           if (kc == x.nkc - 1) tc_commit(&c.S->dfull2[db]);
@@ -1259,12 +1260,14 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
 /*
  * Per (sequence, kv head) segment of keys, with R = Tq * G query rows padded
  * to RP in {16, 32, 64}:
- *   S^T[128 keys][RP] = K Q^T: tcgen05.mma kind::f8f6f4, A = the stage's K
- *     exactly as the tensor copy lands it (e4m3, 128 keys x 128 bytes,
+ *   S^T[128 keys][3 RP] = K Q^T: tcgen05.mma kind::f8f6f4, A = the stage's
+ *     K exactly as the tensor copy lands it (e4m3, 128 keys x 128 bytes,
  *     128-byte swizzle: the K-major canonical layout), B = Q as three e4m3
  *     terms per value (q f = t0 + t1 + t2 with a power-of-two row factor f;
- *     about 12 significant bits, as f16), the three term products
- *     accumulated in TMEM: 3 x 4 MMAs of K = 32 per stage.
+ *     about 12 significant bits, as f16) stacked along N, so one MMA per
+ *     32-wide K step covers all three: 4 MMAs of N = 3 RP per stage (an MMA
+ *     costs about the same up to N = 128, and K is read once); the consumer
+ *     adds a row's three term columns.
  *   p = exp(s - M) under the key windows, on CUDA cores: each consumer
  *     lane holds one key (TMEM lane), its rows' scores; l += p per lane;
  *     P^T is written to shared memory as bf16 scaled by 2^120.
@@ -1280,9 +1283,11 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
  *   p_ready[b] -> issuer: PV(j) -> aempty (stage refill) and pv_done[b]
  *   (P^T buffer reuse; the segment's output read).
  * Shared memory (from the ring base): NS stages of 32 KB (K at 0, V at 16 KB;
- * after widening, bf16 V [key/8][hd/64][key%8][128 B], 128-byte swizzle),
+ * after widening, bf16 V: 8-key group g at 2 KB (g / 2) + 16 KB (g mod 2),
+ * each [hd/64][key%8][128 B] with 128-byte swizzle, read MN-major with the
+ * head-dim halves 1 KB apart and the two groups of an MMA 16 KB apart),
  * then two P^T buffers [2 key tiles][RP rows][128 B], then the Q terms
- * [3][RP rows][128 B].  TMEM: O^T at column 0, S^T buffers at 64 and 128.
+ * [3][RP rows][128 B].  TMEM: O^T at column 0, S^T buffers at 64 and 256.
  */
 /* The issuing warp's part of one layer's attention: this CTA's stages in
  * the consumers' order; lane 0 issues.  ait / aseg: stages and segments
@@ -1302,13 +1307,10 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg) {
     if (j >= 2 && !pwait_bar(c, &c.S->s_free[j & 1u], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) return false;
     if (lane == 0) {
       tc_fence_after();
-      const uint32_t sk = ring + (j % NS) * ATC_STAGE, d = tb + ATC_TM_S + 64u * (j & 1u);
-#pragma unroll 1
-      for (int t = 0; t < 3; ++t)
+      const uint32_t sk = ring + (j % NS) * ATC_STAGE, d = tb + ATC_TM_S + ATC_TM_SSTRIDE * (j & 1u);
+      const uint64_t ka = umma_desc(sk, 16, 1024, 2), qb = umma_desc(qoff, 16, 1024, 2);
 #pragma unroll
-        for (int s = 0; s < 4; ++s)
-          tc_mma_f8(d, umma_desc(sk + 32u * s, 16, 1024, 2), umma_desc(qoff + (uint32_t)(t * RP * 128 + 32 * s), 16, 1024, 2),
-                    id_qk, (t > 0 || s > 0) ? 1u : 0u);
+      for (int s = 0; s < 4; ++s) tc_mma_f8(d, ka + (uint64_t)(2 * s), qb + (uint64_t)(2 * s), id_qk, s > 0 ? 1u : 0u);
       tc_commit(&c.S->s_ready[j & 1u]);
     }
     __syncwarp();
@@ -1320,10 +1322,11 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg) {
     if (lane == 0) {
       tc_fence_after();
       const uint32_t sv = ring + (j % NS) * ATC_STAGE, pt = ptoff + (j & 1u) * (uint32_t)RP * 256u;
+      const uint64_t va = umma_desc(sv, 1024, 16384, 2), pb0 = umma_desc(pt, 16, 1024, 2),
+                     pb1 = umma_desc(pt + (uint32_t)RP * 128u, 16, 1024, 2);
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        tc_mma_f16(tb + ATC_TM_O, umma_desc(sv + 4096u * kk, 1024, 2048, 2),
-                   umma_desc(pt + (uint32_t)((kk >> 2) * RP * 128 + 32 * (kk & 3)), 16, 1024, 2), id_pv,
+        tc_mma_f16(tb + ATC_TM_O, va + (uint64_t)(128 * kk), (kk < 4 ? pb0 : pb1) + (uint64_t)(2 * (kk & 3)), id_pv,
                    (first && kk == 0) ? 0u : 1u);
       tc_commit(&c.S->aempty[j % NS]);
       tc_commit(&c.S->pv_done[j & 1u]);
@@ -1461,9 +1464,13 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
       fence_proxy_async_shared();
       named_sync(BAR_CONS, NCT);
       if (ctid == 0) mbar_arrive(&c.S->q_ready);
-      float l[NR];
+      float l[NR], qf[NR];
 #pragma unroll
-      for (int i = 0; i < NR; ++i) l[i] = 0.f;
+      for (int i = 0; i < NR; ++i) {
+        l[i] = 0.f;
+        qf[i] = c.S->qfac[hh * NR + i]; /* softmax scale / the row's Q-term factor */
+      }
+      const int nvalid = min(NR, max(0, R - hh * NR)); /* this warp's rows below R */
       for (int x = k0; x < k1; x += 128) {
         const uint32_t j = ait, bf = j & 1u, slot = j % NS;
         const int nkeys = min(128, k1 - x);
@@ -1472,21 +1479,28 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
         if (ok && !wait_bar(c, &c.S->s_ready[bf], (j >> 1) & 1u, layer, PH_ATT)) ok = false;
         ok = __all_sync(0xffffffffu, ok) != 0; /* warp-uniform: the TMEM loads below are warp-collective */
         tc_fence_after();
-        /* V of the stage: 1024 16-byte chunks (key k, head-dim chunk ch), four
-         * per thread, read before any thread overwrites the stage */
+        /* V of the stage, widened in place: warp w owns keys 16 w .. 16 w + 15,
+         * whose fp8 V (2 KB at 16 KB + 2 KB w) and fp8 K (2 KB at 2 KB w, free
+         * once the QK products are done) it overwrites with their bf16 V, so
+         * no other warp's bytes are touched and a warp barrier suffices.  Its
+         * lanes read 16-byte chunks (key 16 w + lane / 8 + 4 u, head-dim chunk
+         * lane mod 8). */
         const uint32_t sb = ring + slot * ATC_STAGE;
         uint4 vv[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          const int ci = ctid + NCT * u, k = ci >> 3, ch = ci & 7;
+          const int k = 16 * cw + (lane >> 3) + 4 * u, ch = lane & 7;
           vv[u] = ok ? lds128(sb + 16384u + (uint32_t)k * 128u + ((uint32_t)(ch ^ (k & 7)) << 4)) : make_uint4(0, 0, 0, 0);
         }
-        named_sync(BAR_CONS, NCT);
+        __syncwarp();
         if (ok) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int ci = ctid + NCT * u, k = ci >> 3, ch = ci & 7;
-            const uint32_t dst = sb + (uint32_t)(k >> 3) * 2048u + (uint32_t)(ch >> 2) * 1024u + (uint32_t)(k & 7) * 128u;
+            const int kl = (lane >> 3) + 4 * u, k = 16 * cw + kl, ch = lane & 7;
+            /* 8-key group 2 w (keys 16 w ..) in the K bytes, group 2 w + 1 in
+             * the V bytes; then [hd / 64][key mod 8][128 B], 128-byte swizzle */
+            const uint32_t dst = sb + (kl < 8 ? 0u : 16384u) + (uint32_t)cw * 2048u + (uint32_t)(ch >> 2) * 1024u +
+                                 (uint32_t)(k & 7) * 128u;
             const uint32_t c0 = (uint32_t)(2 * (ch & 3)), c1 = c0 + 1u, sw = (uint32_t)(k & 7);
             sts128(dst + ((c0 ^ sw) << 4), e4m3x2_to_bf16x2_scaled(vv[u].x, 0), e4m3x2_to_bf16x2_scaled(vv[u].x, 1),
                    e4m3x2_to_bf16x2_scaled(vv[u].y, 0), e4m3x2_to_bf16x2_scaled(vv[u].y, 1));
@@ -1494,13 +1508,21 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
                    e4m3x2_to_bf16x2_scaled(vv[u].w, 0), e4m3x2_to_bf16x2_scaled(vv[u].w, 1));
           }
         }
-        /* this warp's scores: its quadrant's 32 keys, its NR rows */
-        uint32_t sr[NR];
+        /* this warp's scores: its quadrant's 32 keys, its NR rows, the sum
+         * of each row's three term columns */
+        float sr[NR];
         if (ok) {
-          const uint32_t ta = tb + ATC_TM_S + 64u * bf + (uint32_t)(hh * NR) + ((uint32_t)(qd * 32) << 16);
+          const uint32_t ta = tb + ATC_TM_S + ATC_TM_SSTRIDE * bf + (uint32_t)(hh * NR) + ((uint32_t)(qd * 32) << 16);
 #pragma unroll
-          for (int i = 0; i < NR; i += 8) tc_ld8(ta + (uint32_t)i, sr + i);
-          tc_wait_ld();
+          for (int i = 0; i < NR; i += 8) {
+            uint32_t t0[8], t1[8], t2[8];
+            tc_ld8(ta + (uint32_t)i, t0);
+            tc_ld8(ta + (uint32_t)(RP + i), t1);
+            tc_ld8(ta + (uint32_t)(2 * RP + i), t2);
+            tc_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) sr[i + e] = __uint_as_float(t0[e]) + __uint_as_float(t1[e]) + __uint_as_float(t2[e]);
+          }
         }
         tc_fence_before();
         __syncwarp();
@@ -1508,23 +1530,28 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
         if (ok) {
           const int key = qd * 32 + lane, kp = x + key;
           const bool full = nkeys == 128 && x >= lo_max && x + 127 <= hi_min;
-          const uint32_t pt = ptoff + bf * (uint32_t)RP * 256u + (uint32_t)(key >> 6) * (uint32_t)RP * 128u;
-          const uint32_t kk = (uint32_t)(key & 63);
+          /* P^T element (row rho, key): tile key / 64, row rho (rho mod 8 = i mod 8
+           * since NR is a multiple of 8), 16-byte chunk (key mod 64) / 8 xor rho mod 8 */
+          const uint32_t kk = (uint32_t)(key & 63), c8 = kk >> 3;
+          const uint32_t pt = ptoff + bf * (uint32_t)RP * 256u + (uint32_t)(key >> 6) * (uint32_t)RP * 128u +
+                              (uint32_t)(hh * NR) * 128u + 2u * (kk & 7u);
+          float pv[NR];
+          if (full) {
+#pragma unroll
+            for (int i = 0; i < NR; ++i) pv[i] = i < nvalid ? fast_exp2(fmaf(sr[i], qf[i], -bound_log2)) : 0.f;
+          } else {
+            const int G = P->G, W = P->W;
+#pragma unroll
+            for (int i = 0; i < NR; ++i) {
+              const int hi = T0 + (hh * NR + i) / G, lo = sliding ? max(0, hi - W + 1) : 0;
+              const bool valid = i < nvalid && key < nkeys && kp >= lo && kp <= hi;
+              pv[i] = valid ? fast_exp2(fmaf(sr[i], qf[i], -bound_log2)) : 0.f;
+            }
+          }
 #pragma unroll
           for (int i = 0; i < NR; ++i) {
-            const int rho = hh * NR + i;
-            float pv = 0.f;
-            if (rho < R) {
-              bool valid = full;
-              if (!full) {
-                const int hi = T0 + rho / P->G, lo = sliding ? max(0, hi - P->W + 1) : 0;
-                valid = key < nkeys && kp >= lo && kp <= hi;
-              }
-              if (valid) pv = fast_exp2(__uint_as_float(sr[i]) * c.S->qfac[rho] - bound_log2);
-            }
-            l[i] += pv;
-            sts16(pt + (uint32_t)rho * 128u + (((kk >> 3) ^ ((uint32_t)rho & 7u)) << 4) + 2u * (kk & 7u),
-                  f32_to_bf16(pv * two120));
+            l[i] += pv[i];
+            sts16(pt + (uint32_t)i * 128u + ((c8 ^ (uint32_t)(i & 7)) << 4), f32_to_bf16(pv[i] * two120));
           }
         }
         fence_proxy_async_shared();
