@@ -18,7 +18,10 @@
  *  - "dev" pointers are CUDA device pointers on the handle's device; "host"
  *    pointers are read during the call only.
  *  - Weight pointers are BORROWED: they must stay valid and unchanged until
- *    msk_destroy.  All of them must be 16-byte aligned.
+ *    msk_destroy.  All of them must be 16-byte aligned.  msk_create reads
+ *    the expert weights once, to repack them into library-owned tiles that
+ *    each K chunk's weights stream from as one contiguous copy
+ *    (msk_query().repacked_bytes); the step reads those tiles.
  *  - msk_step enqueues work on the caller's stream and never synchronises the
  *    host.  Errors the device detects (a wait that gave up, a position
  *    outside the cache) are recorded in a device status word that

@@ -118,6 +118,8 @@ class Engine:
             msk.msk_destroy(self.h)
             self.h = None
         self.wts = None
+        if torch.cuda.is_available():
+            torch.cuda.empty_cache()  # give the weights back for the next handle's own allocations
 
     def __del__(self):
         try:

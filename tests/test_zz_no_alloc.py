@@ -53,25 +53,32 @@ def test_static_step_matches_step_twice():
 
 @pytest.mark.gpu
 def test_static_step_rejects_shapes_beyond_the_array():
-    # 16 x 4 tokens of d_model 4096 need about 17.7 MiB: refused before any
-    # device work, so the weights can be stand-in buffers that are never read
-    w = WORKLOADS["large"]
+    # 16 x 4 tokens of d_model 4096 need about 17.7 MiB of working memory:
+    # refused before any device work.  msk_create reads the expert weights
+    # (it repacks them into its own tiles), so they are real buffers of the
+    # right sizes (zeros), on a model with few small experts.
+    w = WORKLOADS["large"].with_(n_layers=1, sliding=[1], n_experts=32, expert_dim=128)
     dev = torch.device("cuda", 0)
-    d, hd, E = w.d_model, w.head_dim, w.n_experts
+    d, hd, E, f = w.d_model, w.head_dim, w.n_experts, w.expert_dim
+    qd, kvd = w.n_q_heads * hd, w.n_kv_heads * hd
+    keep = []
+
+    def nv(rows, K):
+        c = torch.zeros(rows * K // 2, dtype=torch.uint8, device=dev)
+        s = torch.zeros(rows * K // 16, dtype=torch.uint8, device=dev)
+        keep.extend([c, s])
+        return msk.Nvfp4(c.data_ptr(), s.data_ptr(), 1.0)
+
     ones_d = torch.ones(d, dtype=torch.float32, device=dev)
     ones_hd = torch.ones(hd, dtype=torch.float32, device=dev)
     router = torch.zeros((E, d), dtype=torch.float32, device=dev)
-    blob = torch.zeros(1 << 12, dtype=torch.uint8, device=dev)
-    layers = []
-    for _ in range(w.n_layers):
-        lw = msk.LayerWeights()
-        lw.attn_norm_g = lw.moe_norm_g = ones_d.data_ptr()
-        lw.q_norm_g = lw.k_norm_g = ones_hd.data_ptr()
-        lw.router = router.data_ptr()
-        for role in ("wq", "wk", "wv", "wo", "w_gate", "w_up", "w_down"):
-            setattr(lw, role, msk.Nvfp4(blob.data_ptr(), blob.data_ptr(), 1.0))
-        layers.append(lw)
-    h = msk.msk_create(config_struct(w), layers, 0)
+    lw = msk.LayerWeights()
+    lw.attn_norm_g = lw.moe_norm_g = ones_d.data_ptr()
+    lw.q_norm_g = lw.k_norm_g = ones_hd.data_ptr()
+    lw.router = router.data_ptr()
+    lw.wq, lw.wk, lw.wv, lw.wo = nv(qd, d), nv(kvd, d), nv(kvd, d), nv(d, qd)
+    lw.w_gate, lw.w_up, lw.w_down = nv(E * f, d), nv(E * f, d), nv(E * d, f)
+    h = msk.msk_create(config_struct(w), [lw], 0)
     kv = msk.msk_kv_create(h, w.n_seqs, 16)
     try:
         hid = torch.zeros((w.T, d), dtype=torch.int16, device=dev)

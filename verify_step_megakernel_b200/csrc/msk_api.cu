@@ -16,7 +16,10 @@
 
 extern "C" size_t msk_kernel_smem_bytes();
 extern "C" cudaError_t msk_kernel_setup(int hd, int* ctas_per_sm);
-extern "C" cudaError_t msk_kernel_sf_repack(const uint8_t* in, uint8_t* out, int64_t rows, int k16, cudaStream_t st);
+extern "C" size_t msk_kernel_xtile_gu_bytes(int E, int f, int d);
+extern "C" size_t msk_kernel_xtile_dn_bytes(int E, int rows_per_expert, int K);
+extern "C" cudaError_t msk_kernel_xtile(int kind, const uint8_t* c0, const uint8_t* c1, const uint8_t* s0, const uint8_t* s1,
+                                        uint8_t* out, int E, int rows_per_expert, int K, cudaStream_t st);
 extern "C" cudaError_t msk_kernel_kv_encode(const float* in, uint8_t* out, int64_t n, cudaStream_t stream);
 extern "C" cudaError_t msk_kernel_launch(int hd, const MskParams* P_dev, const MskStep* st, const CUtensorMap* map,
                                          int ncta, cudaStream_t stream);
@@ -406,19 +409,27 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       return MSK_ERR_CUDA;
     }
   }
-  /* the block-scaled expert path reads the gate/up block scales in the
-   * tensor cores' scale-factor layout: repack them once (library-owned
-   * copy; the borrowed weights are not touched) */
-  if (P.tau <= MSK_UNIT_TOK) { /* some unit can take the block-scaled path */
-    const size_t per = (size_t)P.E * P.f * (P.d / 16); /* bytes of one matrix's scales */
-    h->repack_bytes = 2 * per * P.L;
-    bool ok = cudaMalloc(&h->repack, h->repack_bytes) == cudaSuccess;
-    for (int l = 0; l < P.L && ok; ++l) {
-      uint8_t* g = h->repack + (size_t)2 * l * per;
-      ok = msk_kernel_sf_repack(layers[l].w_gate.scales, g, (int64_t)P.E * P.f, P.d / 16, 0) == cudaSuccess &&
-           msk_kernel_sf_repack(layers[l].w_up.scales, g + per, (int64_t)P.E * P.f, P.d / 16, 0) == cudaSuccess;
-      P.layers[l].sfg = g;
-      P.layers[l].sfu = g + per;
+  /* the expert weights as slot images, one contiguous bulk copy per K
+   * chunk (library-owned copies; the borrowed weights are not touched):
+   * gate/up for the block-scaled path when some unit can take it, down for
+   * the CUDA-core path when its K is a multiple of 256 */
+  {
+    const bool gu = P.tau <= MSK_UNIT_TOK, dn = (P.f % 256) == 0;
+    const size_t gub = gu ? msk_kernel_xtile_gu_bytes(P.E, P.f, P.d) : 0;
+    const size_t dnb = dn ? msk_kernel_xtile_dn_bytes(P.E, P.d, P.f) : 0;
+    h->repack_bytes = (gub + dnb) * P.L;
+    bool ok = h->repack_bytes == 0 || cudaMalloc(&h->repack, h->repack_bytes) == cudaSuccess;
+    for (int l = 0; l < P.L && ok && h->repack_bytes; ++l) {
+      uint8_t* g = h->repack + (gub + dnb) * l;
+      const msk_layer_weights_t& w = layers[l];
+      if (gu)
+        ok = msk_kernel_xtile(0, w.w_gate.codes, w.w_up.codes, w.w_gate.scales, w.w_up.scales, g, P.E, P.f, P.d, 0) ==
+             cudaSuccess;
+      if (ok && dn)
+        ok = msk_kernel_xtile(1, w.w_down.codes, nullptr, w.w_down.scales, nullptr, g + gub, P.E, P.d, P.f, 0) ==
+             cudaSuccess;
+      P.layers[l].xtgu = gu ? g : nullptr;
+      P.layers[l].xtdn = dn ? g + gub : nullptr;
     }
     if (ok) ok = cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {

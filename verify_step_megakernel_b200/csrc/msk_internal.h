@@ -50,11 +50,14 @@ typedef struct MskLayer {
    * codes, gate scales, up codes, up scales, down codes, down scales, then
    * (from MSK_MAP_DENSE) codes and scales of wq, wk, wv, wo */
   const CUtensorMap* emap;
-  /* gate and up block scales repacked (library-owned) in the block-scaled
-   * tensor cores' scale-factor atoms: [E][f/128][d/64][512 B], atom byte
-   * 16 r + 4 m + b = scale of row 128 g + r + 32 m, block 4 s + b */
-  const uint8_t* sfg;
-  const uint8_t* sfu;
+  /* expert weights repacked (library-owned) into slot images, one
+   * contiguous bulk copy per K chunk: gate/up tiles of the block-scaled path
+   * [E][f/128][d/256][36 KB] (swizzled codes of both matrices, then their
+   * scale-factor atoms), down tiles of the CUDA-core path
+   * [E][d/128][f/KC][128 (KC/2 + 32 + KC/16)] (null when K is not a
+   * multiple of 256: whole rows are copied then) */
+  const uint8_t* xtgu;
+  const uint8_t* xtdn;
   float bound_log2; /* M * log2(e), M = sqrt(hd) max|g_q| max|g_k| */
   int32_t sliding;
 } MskLayer;

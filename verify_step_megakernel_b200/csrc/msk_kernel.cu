@@ -90,10 +90,10 @@ struct Smem {
   uint32_t tmem_base;
   AttGeo ag;                /* this layer's attention key split (consumers) */
   AttGeo agp;               /* the producer warp's copy */
-  uint4 sfb_one[32];        /* 128 rows x 4 ue4m3 scales of 1.0, the activation terms' scales */
-  volatile int issuer_done; /* the MMA-issuing warp has committed its last work */
+  uint4 sfb_one[64];        /* per issuing role: 128 rows x 4 ue4m3 scales of 1.0, the activation terms' scales */
+  volatile int issuer_done; /* MMA-issuing warps that have committed their last work */
   uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
-  uint64_t xempty[XNS_MAX]; /* expert slot consumed (one arrival: a tensor-core commit or the consumers' last warp) */
+  uint64_t xempty[XNS_MAX]; /* expert slot consumed (two arrivals: both issuing roles' commits, or two consumer threads) */
   volatile int kv_ready;    /* layer+1 whose KV writes all CTAs finished */
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
@@ -225,13 +225,14 @@ MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
  *         [8 core-matrix columns][8 term rows][16 B] (all term scales are 1) */
 constexpr int GU_KC = 256;
 constexpr uint32_t GU_A = 0, GU_AS = 32768, GU_B = 36864, GU_SLOT = 45056;
+constexpr uint32_t GU_AS_END = GU_B; /* codes and scale atoms of a chunk: one repacked tile */
 /* TMEM columns: two buffers of gate and up accumulators (128 lanes x 64
  * each), then the scale factors of two chunks in flight */
 constexpr uint32_t TM_D = 0, TM_DU = 64, TM_SFA = 256, TM_SFB = 384, TM_COLS = 512;
 /* scale-factor buffers in TMEM: four chunks in rotation */
 constexpr int NSF = 4;
 constexpr uint32_t TM_SFA_BUF = 32; /* columns per buffer: 2 matrices x 4 steps x 4; SFB: 4 columns of ones */
-static_assert(TM_SFA + NSF * TM_SFA_BUF <= TM_SFB && TM_SFB + 4 <= TM_COLS, "TMEM columns");
+static_assert(TM_SFA + NSF * TM_SFA_BUF <= TM_SFB && TM_SFB + 8 <= TM_COLS, "TMEM columns");
 
 struct XGeo {
   int K, KC, nkc, rows_unit, ngroups, NM, tma, ns;
@@ -563,12 +564,9 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
         uint64_t* bar = &c.S->xfull[s];
         if (lane == 0) mbar_arrive_tx(bar, bytes);
         __syncwarp();
-        if (lane < 2) {
-          tma_2d_g2s(dst + GU_A + lane * 16384, Ly.emap + MSK_MAP_GUSW + lane, kc * (GU_KC / 2), (int32_t)grow, bar);
-        } else if (lane == 4 || lane == 5) { /* the chunk's scale-factor atoms, as the tensor core reads them */
-          const int m = lane - 4;
-          const int64_t atom = (grow / XROWS) * (P->d / 64) + (int64_t)kc * (GU_KC / 64);
-          bulk_g2s(dst + GU_AS + m * (XROWS * GU_KC / 16), (m ? Ly.sfu : Ly.sfg) + atom * 512, XROWS * GU_KC / 16, bar);
+        if (lane == 0) { /* the chunk's codes and scale atoms of both matrices: one tile, one copy */
+          const int64_t tile = (grow / XROWS) * (P->d / GU_KC) + kc;
+          bulk_g2s(dst, Ly.xtgu + tile * GU_AS_END, GU_AS_END, bar);
         } else if (tq) {
           bulk_g2s(dst + GU_B + tl * (8 * GU_KC / 2), tq + (size_t)kc * (8 * GU_KC / 2), 8 * GU_KC / 2, bar);
         }
@@ -599,7 +597,11 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
       uint64_t* bar = &c.S->xfull[s];
       if (lane == 0) mbar_arrive_tx(bar, x.b_off + (uint32_t)n * brow);
       __syncwarp();
-      if (lane < 2 * x.NM) { /* lane 2m: codes of matrix m, lane 2m+1: its scales */
+      if (!gu && Ly.xtdn && x.tma) { /* the down chunk's codes and scales: one repacked tile, one copy */
+        if (lane == 0) bulk_g2s(dst, Ly.xtdn + ((grow / XROWS) * x.nkc + kc) * (int64_t)x.mat_bytes, x.mat_bytes, bar);
+        else if (lane >= 8 && lane < 8 + n)
+          bulk_g2s(dst + x.b_off + (lane - 8) * x.bpitch, act + (size_t)my_row * act_ld + (size_t)kc * x.KC, brow, bar);
+      } else if (lane < 2 * x.NM) { /* lane 2m: codes of matrix m, lane 2m+1: its scales */
         const int m = lane >> 1;
         uint8_t* md = dst + (size_t)m * x.mat_bytes;
         if (x.tma) {
@@ -630,9 +632,14 @@ MSK_DEV bool prod_xdrain(Prod& p, int layer) {
  * consumers' scale staging, copies the scales into TMEM, issues the
  * block-scaled MMAs into the item's accumulator buffer (after the
  * consumers released that buffer) and commits (see expert_gu_tc). */
-MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg);
+MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& aseg);
 
-MSK_DEV void issuer(Ctx& c) {
+/* The two MMA-issuing warps (warps 1 and 2; lane 0 issues), role 0 and 1:
+ * attention QK and PV products respectively, and the gate and the up
+ * matrix of the block-scaled expert path respectively (each copies its
+ * matrix's scale atoms into TMEM and issues its MMAs; the slot and the
+ * accumulator buffer complete when both have committed). */
+MSK_DEV void issuer(Ctx& c, int role) {
   const MskParams* P = c.P;
   const int lane = threadIdx.x & 31;
   const uint32_t idesc = (1u << 7) | (1u << 10) | ((uint32_t)(64 >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
@@ -641,20 +648,21 @@ MSK_DEV void issuer(Ctx& c) {
   uint32_t tb = 0;
   uint32_t ait = 0, aseg = 0; /* attention stages and segments issued */
   for (int l = 0; l < P->L && ok; ++l) {
-    if (P->hd == 128 && !issuer_att(c, l, ait, aseg)) { ok = false; break; }
+    if (P->hd == 128 && !issuer_att(c, l, role, ait, aseg)) { ok = false; break; }
     if (!tc_experts(P)) continue;
     if (!pwait_flag(c, &c.S->route_ready, l + 1, l, PH_GU)) { ok = false; break; }
     tb = c.S->tmem_base;
     /* the activation terms' block scales, all 1.0 (ue4m3 0x38), into TMEM
-     * each layer (the attention phase reuses those columns) */
+     * each layer (the attention phase reuses those columns); each role
+     * copies its own, so its MMAs follow the copy in its issue order */
     if (l == 0) {
-      c.S->sfb_one[lane] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
+      c.S->sfb_one[role * 32 + lane] = make_uint4(0x38383838u, 0x38383838u, 0x38383838u, 0x38383838u);
       fence_proxy_async_shared();
       __syncwarp();
     }
     if (lane == 0) {
       tc_fence_after();
-      tc_cp_sf(tb + TM_SFB, umma_desc(smem_u32(c.S->sfb_one), 16, 128, 0));
+      tc_cp_sf(tb + TM_SFB + 4 * role, umma_desc(smem_u32(c.S->sfb_one + role * 32), 16, 128, 0));
     }
     __syncwarp();
     XGeo x, xc, xd;
@@ -678,17 +686,18 @@ MSK_DEV void issuer(Ctx& c) {
           const uint32_t slot = ring + (uint32_t)s * x.slot_bytes;
           const uint64_t sd = umma_desc(slot + GU_AS, 16, 128, 0), ad = umma_desc(slot + GU_A, 16, 1024, 2),
                          bd = umma_desc(slot + GU_B, 128, 8 * GU_KC / 2, 0);
-          const uint32_t sfa = tb + TM_SFA + buf * TM_SFA_BUF, sfb = tb + TM_SFB, dg = tb + TM_D + db * 128;
-          /* descriptors advance by adding to their address field (16-byte units) */
+          /* this role's matrix: its scale atoms (4 steps) into its TMEM
+           * columns, then its 4 MMAs; descriptors advance by adding to their
+           * address field (16-byte units) */
+          const uint32_t sfa = tb + TM_SFA + buf * TM_SFA_BUF + 16 * role, sfb = tb + TM_SFB + 4 * role;
+          const uint32_t dg = tb + TM_D + db * 128 + TM_DU * role;
+          const uint64_t sdr = sd + (uint64_t)(128 * role), adr = ad + (uint64_t)(1024 * role);
 #pragma unroll
-          for (int st = 0; st < 2 * (GU_KC / 64); ++st) tc_cp_sf(sfa + 4 * st, sd + (uint64_t)(st * 32));
+          for (int st = 0; st < GU_KC / 64; ++st) tc_cp_sf(sfa + 4 * st, sdr + (uint64_t)(st * 32));
 #pragma unroll
-          for (int st = 0; st < GU_KC / 64; ++st) {
-            const uint32_t acc = (kc > 0 || st > 0) ? 1u : 0u;
-            const uint64_t b = bd + (uint64_t)(16 * st), a = ad + (uint64_t)(2 * st);
-            tc_mma_nvf4(dg, a, b, idesc, acc, sfa + 4 * st, sfb);
-            tc_mma_nvf4(dg + TM_DU, a + 1024u, b, idesc, acc, sfa + 16 + 4 * st, sfb);
-          }
+          for (int st = 0; st < GU_KC / 64; ++st)
+            tc_mma_nvf4(dg, adr + (uint64_t)(2 * st), bd + (uint64_t)(16 * st), idesc, (kc > 0 || st > 0) ? 1u : 0u,
+                        sfa + 4 * st, sfb);
           tc_commit(&c.S->xempty[s]);
           if (kc == x.nkc - 1) tc_commit(&c.S->dfull2[db]);
         }
@@ -704,7 +713,7 @@ MSK_DEV void issuer(Ctx& c) {
   if (lane == 0) {
     tc_commit(&c.S->tfin);
     __threadfence_block();
-    c.S->issuer_done = 1;
+    atomicAdd((int*)&c.S->issuer_done, 1);
   }
 }
 
@@ -1289,10 +1298,13 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
  * then two P^T buffers [2 key tiles][RP rows][128 B], then the Q terms
  * [3][RP rows][128 B].  TMEM: O^T at column 0, S^T buffers at 64 and 256.
  */
-/* The issuing warp's part of one layer's attention: this CTA's stages in
- * the consumers' order; lane 0 issues.  ait / aseg: stages and segments
- * issued so far (the consumers count the same). */
-MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg) {
+/* One issuing warp's part of one layer's attention (lane 0 issues): role 0
+ * issues every stage's QK products, role 1 its PV products, so the two
+ * streams of MMAs are issued by two threads at once (a single thread issues
+ * a tcgen05.mma about every 70 cycles, two together every 45).  ait / aseg:
+ * stages and segments this role issued so far (the consumers count the
+ * same). */
+MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& aseg) {
   const MskParams* P = c.P;
   const int lane = threadIdx.x & 31;
   if (!pwait_flag(c, &c.S->ag_ready, layer + 1, layer, PH_ATT)) return false;
@@ -1301,46 +1313,40 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg) {
   const uint32_t tb = c.S->tmem_base, ring = smem_u32(c.ring);
   const uint32_t qoff = ring + atc_q_off(RP), ptoff = ring + atc_pt_off(RP);
   const uint32_t id_qk = atc_idesc_qk(RP), id_pv = atc_idesc_pv(RP);
+  const uint64_t qb = umma_desc(qoff, 16, 1024, 2);
   bool ok = true;
-  auto qk = [&](uint32_t j) -> bool {
-    if (!pwait_bar(c, &c.S->afull[j % NS], (j / NS) & 1u, layer, PH_ATT)) return false;
-    if (j >= 2 && !pwait_bar(c, &c.S->s_free[j & 1u], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) return false;
-    if (lane == 0) {
-      tc_fence_after();
-      const uint32_t sk = ring + (j % NS) * ATC_STAGE, d = tb + ATC_TM_S + ATC_TM_SSTRIDE * (j & 1u);
-      const uint64_t ka = umma_desc(sk, 16, 1024, 2), qb = umma_desc(qoff, 16, 1024, 2);
-#pragma unroll
-      for (int s = 0; s < 4; ++s) tc_mma_f8(d, ka + (uint64_t)(2 * s), qb + (uint64_t)(2 * s), id_qk, s > 0 ? 1u : 0u);
-      tc_commit(&c.S->s_ready[j & 1u]);
-    }
-    __syncwarp();
-    return true;
-  };
-  auto pv = [&](uint32_t j, bool first) -> bool {
-    if (!pwait_bar(c, &c.S->p_ready[j & 1u], (j >> 1) & 1u, layer, PH_ATT)) return false;
-    if (first && aseg > 0 && !pwait_bar(c, &c.S->o_free, (aseg - 1u) & 1u, layer, PH_ATT)) return false;
-    if (lane == 0) {
-      tc_fence_after();
-      const uint32_t sv = ring + (j % NS) * ATC_STAGE, pt = ptoff + (j & 1u) * (uint32_t)RP * 256u;
-      const uint64_t va = umma_desc(sv, 1024, 16384, 2), pb0 = umma_desc(pt, 16, 1024, 2),
-                     pb1 = umma_desc(pt + (uint32_t)RP * 128u, 16, 1024, 2);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        tc_mma_f16(tb + ATC_TM_O, va + (uint64_t)(128 * kk), (kk < 4 ? pb0 : pb1) + (uint64_t)(2 * (kk & 3)), id_pv,
-                   (first && kk == 0) ? 0u : 1u);
-      tc_commit(&c.S->aempty[j % NS]);
-      tc_commit(&c.S->pv_done[j & 1u]);
-    }
-    __syncwarp();
-    return true;
-  };
   for_each_att_stage(c, g, [&](int, int, int64_t, int, bool first, bool last) {
-    if (first) {
-      if (!pwait_bar(c, &c.S->q_ready, aseg & 1u, layer, PH_ATT)) { ok = false; return false; }
-      if (!qk(ait)) { ok = false; return false; }
+    const uint32_t j = ait;
+    if (role == 0) {
+      if (first && !pwait_bar(c, &c.S->q_ready, aseg & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (!pwait_bar(c, &c.S->afull[j % NS], (j / NS) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (j >= 2 && !pwait_bar(c, &c.S->s_free[j & 1u], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (lane == 0) {
+        tc_fence_after();
+        const uint32_t d = tb + ATC_TM_S + ATC_TM_SSTRIDE * (j & 1u);
+        const uint64_t ka = umma_desc(ring + (j % NS) * ATC_STAGE, 16, 1024, 2);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) tc_mma_f8(d, ka + (uint64_t)(2 * s), qb + (uint64_t)(2 * s), id_qk, s > 0 ? 1u : 0u);
+        tc_commit(&c.S->s_ready[j & 1u]);
+      }
+      __syncwarp();
+    } else {
+      if (!pwait_bar(c, &c.S->p_ready[j & 1u], (j >> 1) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (first && aseg > 0 && !pwait_bar(c, &c.S->o_free, (aseg - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (lane == 0) {
+        tc_fence_after();
+        const uint32_t pt = ptoff + (j & 1u) * (uint32_t)RP * 256u;
+        const uint64_t va = umma_desc(ring + (j % NS) * ATC_STAGE, 1024, 16384, 2), pb0 = umma_desc(pt, 16, 1024, 2),
+                       pb1 = umma_desc(pt + (uint32_t)RP * 128u, 16, 1024, 2);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          tc_mma_f16(tb + ATC_TM_O, va + (uint64_t)(128 * kk), (kk < 4 ? pb0 : pb1) + (uint64_t)(2 * (kk & 3)), id_pv,
+                     (first && kk == 0) ? 0u : 1u);
+        tc_commit(&c.S->aempty[j % NS]);
+        tc_commit(&c.S->pv_done[j & 1u]);
+      }
+      __syncwarp();
     }
-    if (!last && !qk(ait + 1)) { ok = false; return false; }
-    if (!pv(ait, first)) { ok = false; return false; }
     ait++;
     if (last) aseg++;
     return true;
@@ -2276,7 +2282,7 @@ MSK_DEV bool expert_mma(Ctx& c, int layer, uint32_t& xpar) {
         xgemm<GU ? 2 : 1>(slot + cw * 16 * x.cpitch, slot + XROWS * x.cpitch + cw * 16 * x.spitch, x.mat_bytes,
                           x.cpitch, x.spitch, slot + x.b_off, x.bpitch, x.KC, acc, acc2);
       named_sync(BAR_CONS, NCT);
-      if (ok && ctid == 0) mbar_arrive(&c.S->xempty[s]);
+      if (ok && ctid < 2) mbar_arrive(&c.S->xempty[s]); /* the slot's two arrivals */
     }
     if (!ok) continue;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
@@ -2386,13 +2392,13 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     mbar_init(&c.S->rfull, 1);
     for (int i = 0; i < XNS_MAX; ++i) {
       mbar_init(&c.S->xfull[i], 1);
-      mbar_init(&c.S->xempty[i], 1);
+      mbar_init(&c.S->xempty[i], 2); /* two tensor-core commits, or two consumer threads */
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&c.S->dfull2[i], 1);
+      mbar_init(&c.S->dfull2[i], 2); /* both issuing roles commit */
       mbar_init(&c.S->dempty2[i], NCW);
     }
-    mbar_init(&c.S->tfin, 1);
+    mbar_init(&c.S->tfin, 2);
     for (int i = 0; i < 5; ++i) {
       mbar_init(&c.S->afull[i], 1);
       mbar_init(&c.S->aempty[i], 1);
@@ -2431,7 +2437,7 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
   if (threadIdx.x < CONS0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
     if (threadIdx.x < 32) producer(c);
-    else if (threadIdx.x < 64) issuer(c);
+    else if (threadIdx.x < 96) issuer(c, (threadIdx.x >> 5) - 1);
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_CONSUMER));
     const bool w0 = (threadIdx.x >> 5) == CONS_WARP0;
@@ -2447,7 +2453,7 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     named_sync(BAR_CONS, NCT);
     if (threadIdx.x == CONS0) {
       const uint64_t t0 = gtimer();
-      while (!c.S->issuer_done && gtimer() - t0 < 2 * (uint64_t)P->timeout_ns) __nanosleep(64);
+      while (c.S->issuer_done < 2 && gtimer() - t0 < 2 * (uint64_t)P->timeout_ns) __nanosleep(64);
       while (!mbar_try(&c.S->tfin, 0) && gtimer() - t0 < 4 * (uint64_t)P->timeout_ns) {
       }
     }
@@ -2471,30 +2477,92 @@ __global__ void msk_kv_encode_tail(const float* __restrict__ in, uint8_t* __rest
   if (i < n) out[i] = (uint8_t)f32x2_to_e4m3x2(in[i], 0.f);
 }
 
-/* NVFP4 block scales [rows][k16] (k16 = K/16, rows a multiple of 128, k16 a
- * multiple of 4) -> the block-scaled tensor cores' scale-factor atoms
- * [rows/128][k16/4][512 B]: byte 16 r + 4 m + b of atom (g, s) is the scale
- * of row 128 g + r + 32 m, block 4 s + b.  One 4-byte word per thread. */
-__global__ void msk_sf_repack_kernel(const uint8_t* __restrict__ in, uint32_t* __restrict__ out, int64_t nwords,
-                                     int k16) {
-  const int S = k16 / 4;
-  for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < nwords; w += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t a = w >> 7;
-    const int i = (int)(w & 127), r0 = i >> 2, m1 = i & 3;
-    const int64_t g = a / S, st = a - g * S;
-    const int64_t row = g * 128 + r0 + 32 * m1;
-    out[w] = *reinterpret_cast<const uint32_t*>(in + row * k16 + 4 * st);
+/* Expert weight tiles for whole-slot bulk copies (one contiguous copy per
+ * K chunk instead of a 2-D box per row: 2-D boxes of 128-byte rows stream at
+ * about 5.0 TB/s on this part, contiguous 32-48 KB bulk copies at 7.2-7.4).
+ * Gate/up for the block-scaled path, per (expert, 128-row group, 256-wide K
+ * chunk), 36 KB laid out as the slot: gate codes [128][128 B] and up codes,
+ * each as the 128-byte-swizzled image the tensor copy would have written
+ * (16-byte chunk c of row r at (c xor r mod 8)), then the gate and up
+ * scale-factor atoms of the chunk's four 64-wide K steps. */
+__global__ void msk_xtile_gu_kernel(const uint8_t* __restrict__ gc, const uint8_t* __restrict__ uc,
+                                    const uint8_t* __restrict__ gsc, const uint8_t* __restrict__ usc,
+                                    uint4* __restrict__ out, int64_t ntiles, int f, int d) {
+  const int nkc = d / 256, ng = f / 128, k16 = d / 16;
+  const int64_t nch = ntiles * (GU_SLOT - 8192) / 16; /* 2304 chunks of 16 bytes per tile */
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < nch; q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = q / 2304;
+    const int qi = (int)(q - t * 2304);
+    const int kc = (int)(t % nkc), g = (int)((t / nkc) % ng);
+    const int64_t e = t / ((int64_t)nkc * ng);
+    const int64_t row0 = e * f + (int64_t)g * 128;
+    uint4 v;
+    if (qi < 2048) { /* codes: matrix m, row r, physical chunk p */
+      const int m = qi >> 10, r = (qi >> 3) & 127, pch = qi & 7, lch = pch ^ (r & 7);
+      v = *reinterpret_cast<const uint4*>((m ? uc : gc) + (row0 + r) * (d / 2) + kc * 128 + lch * 16);
+    } else { /* scale atoms: matrix m, step st, atom row r: rows r + 32 m1, four blocks */
+      const int ai = qi - 2048, m = ai >> 7, st = (ai >> 5) & 3, r = ai & 31;
+      const uint8_t* sc = m ? usc : gsc;
+      uint32_t w[4];
+#pragma unroll
+      for (int m1 = 0; m1 < 4; ++m1)
+        w[m1] = *reinterpret_cast<const uint32_t*>(sc + (row0 + r + 32 * m1) * k16 + (kc * 4 + st) * 4);
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    out[q] = v;
+  }
+}
+
+/* Down projection tiles for the CUDA-core path, per (expert, 128-row group,
+ * K chunk of KC = min(K, 512)), laid out as its slot: codes [128][KC/2 + 32]
+ * (the 32 padding bytes zero) then scales [128][KC/16]. */
+__global__ void msk_xtile_dn_kernel(const uint8_t* __restrict__ dc, const uint8_t* __restrict__ dsc,
+                                    uint4* __restrict__ out, int64_t ntiles, int rows_per_expert, int K) {
+  const int KC = K < 512 ? K : 512, nkc = K / KC, ng = rows_per_expert / 128;
+  const int cp = KC / 2 + 32, sp = KC / 16;
+  const int tile16 = 128 * (cp + sp) / 16;
+  const int64_t nch = ntiles * tile16;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < nch; q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = q / tile16;
+    const int qi = (int)(q - t * tile16);
+    const int kc = (int)(t % nkc), g = (int)((t / nkc) % ng);
+    const int64_t e = t / ((int64_t)nkc * ng);
+    const int64_t row0 = e * rows_per_expert + (int64_t)g * 128;
+    uint4 v = make_uint4(0, 0, 0, 0);
+    const int off = qi * 16;
+    if (off < 128 * cp) {
+      const int r = off / cp, c = off - r * cp;
+      if (c < KC / 2) v = *reinterpret_cast<const uint4*>(dc + (row0 + r) * (K / 2) + kc * (KC / 2) + c);
+    } else {
+      const int so = off - 128 * cp, r = so / sp, c = so - r * sp;
+      v = *reinterpret_cast<const uint4*>(dsc + (row0 + r) * (K / 16) + kc * sp + c);
+    }
+    out[q] = v;
   }
 }
 
 /* ---- launch ---------------------------------------------------------------------------- */
 extern "C" size_t msk_kernel_smem_bytes() { return SMEM_BYTES; }
 
-extern "C" cudaError_t msk_kernel_sf_repack(const uint8_t* in, uint8_t* out, int64_t rows, int k16, cudaStream_t st) {
-  const int64_t nwords = rows * k16 / 4;
-  const int64_t blocks = (nwords + 255) / 256;
-  msk_sf_repack_kernel<<<(unsigned)(blocks < 148 * 32 ? blocks : 148 * 32), 256, 0, st>>>(
-      in, reinterpret_cast<uint32_t*>(out), nwords, k16);
+extern "C" size_t msk_kernel_xtile_gu_bytes(int E, int f, int d) { return (size_t)E * (f / 128) * (d / 256) * (GU_SLOT - 8192); }
+extern "C" size_t msk_kernel_xtile_dn_bytes(int E, int rows_per_expert, int K) {
+  const int KC = K < 512 ? K : 512;
+  return (size_t)E * (rows_per_expert / 128) * (K / KC) * 128 * (KC / 2 + 32 + KC / 16);
+}
+extern "C" cudaError_t msk_kernel_xtile(int kind, const uint8_t* c0, const uint8_t* c1, const uint8_t* s0, const uint8_t* s1,
+                                        uint8_t* out, int E, int rows_per_expert, int K, cudaStream_t st) {
+  if (kind == 0) {
+    const int64_t ntiles = (int64_t)E * (rows_per_expert / 128) * (K / 256);
+    const int64_t n = ntiles * 2304;
+    msk_xtile_gu_kernel<<<(unsigned)((n + 255) / 256 < 148 * 64 ? (n + 255) / 256 : 148 * 64), 256, 0, st>>>(
+        c0, c1, s0, s1, reinterpret_cast<uint4*>(out), ntiles, rows_per_expert, K);
+  } else {
+    const int KC = K < 512 ? K : 512;
+    const int64_t ntiles = (int64_t)E * (rows_per_expert / 128) * (K / KC);
+    const int64_t n = ntiles * 128 * (KC / 2 + 32 + KC / 16) / 16;
+    msk_xtile_dn_kernel<<<(unsigned)((n + 255) / 256 < 148 * 64 ? (n + 255) / 256 : 148 * 64), 256, 0, st>>>(
+        c0, s0, reinterpret_cast<uint4*>(out), ntiles, rows_per_expert, K);
+  }
   return cudaGetLastError();
 }
 
