@@ -93,7 +93,8 @@ struct Smem {
   uint4 sfb_one[64];        /* per issuing role: 128 rows x 4 ue4m3 scales of 1.0, the activation terms' scales */
   volatile int issuer_done; /* MMA-issuing warps that have committed their last work */
   uint64_t xfull[XNS_MAX];  /* expert slot landed (producer's expect-tx) */
-  uint64_t xempty[XNS_MAX]; /* expert slot consumed (two arrivals: both issuing roles' commits, or two consumer threads) */
+  uint64_t xempty[XNS_MAX]; /* block-scaled expert slot consumed (both issuing roles' commits) */
+  uint64_t xempty_cc[XNS_MAX]; /* CUDA-core expert slot consumed (each consumer warp arrives) */
   volatile int kv_ready;    /* layer+1 whose KV writes all CTAs finished */
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
@@ -106,8 +107,8 @@ struct Smem {
   uint64_t aempty[5];       /* the stage's P.V products completed (tensor-core commit) */
   uint64_t s_ready[2];      /* scores S^T of buffer b computed */
   uint64_t s_free[2];       /* S^T of buffer b read by every consumer warp */
-  uint64_t p_ready[2];      /* P^T of buffer b and the stage's bf16 V written by every consumer warp */
-  uint64_t pv_done[2];      /* the P.V products of buffer b completed */
+  uint64_t p_ready[3];      /* P^T of buffer b (stage mod 3) and the stage's bf16 V written by every consumer warp */
+  uint64_t pv_done[3];      /* the P.V products of P^T buffer b completed */
   uint64_t q_ready;         /* the segment's Q terms written */
   uint64_t o_free;          /* the segment's output accumulator read */
   volatile int ag_ready;    /* layer+1 whose attention key split (ag) the consumers computed */
@@ -408,10 +409,10 @@ constexpr uint32_t ATC_STAGE = 32768;
 constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64, ATC_TM_SSTRIDE = 192;
 MSK_DEV int atc_ns(int RP) { return RP > 32 ? 4 : 5; }
 MSK_DEV uint32_t atc_pt_off(int RP) { return (uint32_t)atc_ns(RP) * ATC_STAGE; }
-MSK_DEV uint32_t atc_q_off(int RP) { return atc_pt_off(RP) + 2u * (uint32_t)RP * 256u; }
+MSK_DEV uint32_t atc_q_off(int RP) { return atc_pt_off(RP) + 3u * (uint32_t)RP * 256u; }
 MSK_DEV int atc_rp(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 64); }
-static_assert(4 * ATC_STAGE + 2 * 64 * 256 + 3 * 64 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
-static_assert(5 * ATC_STAGE + 2 * 32 * 256 + 3 * 32 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
+static_assert(4 * ATC_STAGE + 3 * 64 * 256 + 3 * 64 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
+static_assert(5 * ATC_STAGE + 3 * 32 * 256 + 3 * 32 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
 /* instruction descriptors: fp32 accumulators, M = 128, N = RP; QK e4m3 x e4m3
  * both K-major; PV bf16 x bf16 with A MN-major */
 MSK_DEV uint32_t atc_idesc_qk(int RP) { return (1u << 4) | ((uint32_t)((3 * RP) >> 3) << 17) | ((128u >> 4) << 24); }
@@ -426,6 +427,9 @@ struct Prod {
   uint32_t ait;   /* tensor-core attention stages issued */
   uint32_t xpar;  /* bit s: parity of the fills of expert slot s so far */
   uint32_t xused; /* bit s: expert slot s filled at least once */
+  uint32_t xptc;  /* bit s: parity of its block-scaled fills (released by the issuers' commits) */
+  uint32_t xpcc;  /* bit s: parity of its CUDA-core fills (released by the eight consumer warps) */
+  uint32_t xlast; /* bit s: its last fill was a block-scaled one */
   uint32_t dpar;  /* bit 2w+s: parity of the fills of warp w's dense slot s */
   uint32_t dused; /* bit 2w+s: that slot filled at least once */
   bool ok;
@@ -529,6 +533,8 @@ MSK_DEV void prefetch_dense(const Ctx& c, int layer, bool qkv) {
 /* Fill the expert ring for one phase: for each of this CTA's items and
  * each K chunk, the 128-row tiles of the unit's expert (gate and up, or
  * down) and the unit's activation rows, all on the slot's full barrier. */
+MSK_DEV bool prod_xslot(Prod& p, int s, bool tc, int layer, int phase);
+
 MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
   Ctx& c = *p.c;
   const MskParams* P = c.P;
@@ -555,11 +561,7 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
       const uint32_t bytes = (uint32_t)(2 * 16384 + 2 * XROWS * (GU_KC / 16) + n * 8 * (GU_KC / 2));
       for (int kc = 0; kc < x.nkc; ++kc, ++j) {
         const int s = j % x.ns;
-        if ((p.xused >> s) & 1u) {
-          if (!pwait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, phase)) return false;
-        }
-        p.xpar ^= 1u << s;
-        p.xused |= 1u << s;
+        if (!prod_xslot(p, s, true, layer, phase)) return false;
         uint8_t* dst = c.ring + (size_t)s * x.slot_bytes;
         uint64_t* bar = &c.S->xfull[s];
         if (lane == 0) mbar_arrive_tx(bar, bytes);
@@ -588,11 +590,7 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
     }
     for (int kc = 0; kc < x.nkc; ++kc, ++j) {
       const int s = j % x.ns;
-      if ((p.xused >> s) & 1u) {
-        if (!pwait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, phase)) return false;
-      }
-      p.xpar ^= 1u << s;
-      p.xused |= 1u << s;
+      if (!prod_xslot(p, s, false, layer, phase)) return false;
       uint8_t* dst = c.ring + (size_t)s * x.slot_bytes;
       uint64_t* bar = &c.S->xfull[s];
       if (lane == 0) mbar_arrive_tx(bar, x.b_off + (uint32_t)n * brow);
@@ -619,11 +617,38 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
   return true;
 }
 
+/* Before filling expert slot s: wait (if it was filled before) until its
+ * last fill was released, by the barrier of that fill's kind, then record
+ * this fill (tc: a block-scaled fill). */
+MSK_DEV bool prod_xslot(Prod& p, int s, bool tc, int layer, int phase) {
+  Ctx& c = *p.c;
+  if ((p.xused >> s) & 1u) {
+    const bool ltc = (p.xlast >> s) & 1u;
+    if (!pwait_bar(c, ltc ? &c.S->xempty[s] : &c.S->xempty_cc[s], (((ltc ? p.xptc : p.xpcc) >> s) & 1u) ^ 1u, layer,
+                   phase))
+      return false;
+  }
+  p.xpar ^= 1u << s;
+  p.xused |= 1u << s;
+  if (tc) {
+    p.xptc ^= 1u << s;
+    p.xlast |= 1u << s;
+  } else {
+    p.xpcc ^= 1u << s;
+    p.xlast &= ~(1u << s);
+  }
+  return true;
+}
+
 /* wait until the last fill of every expert slot has been released */
 MSK_DEV bool prod_xdrain(Prod& p, int layer) {
   Ctx& c = *p.c;
   for (int s = 0; s < XNS_MAX; ++s)
-    if (((p.xused >> s) & 1u) && !pwait_bar(c, &c.S->xempty[s], ((p.xpar >> s) & 1u) ^ 1u, layer, PH_GU)) return false;
+    if ((p.xused >> s) & 1u) {
+      const bool tc = (p.xlast >> s) & 1u;
+      if (!pwait_bar(c, tc ? &c.S->xempty[s] : &c.S->xempty_cc[s], (((tc ? p.xptc : p.xpcc) >> s) & 1u) ^ 1u, layer, PH_GU))
+        return false;
+    }
   return true;
 }
 
@@ -728,6 +753,9 @@ MSK_DEV void producer(Ctx& c) {
   p.ait = 0;
   p.xpar = 0;
   p.xused = 0;
+  p.xptc = 0;
+  p.xpcc = 0;
+  p.xlast = 0;
   p.dpar = 0;
   p.dused = 0;
   p.ok = true;
@@ -1265,6 +1293,60 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
   return R <= 16 ? attention_phase_mt<HD, 1>(q, layer) : attention_phase_mt<HD, 2>(q, layer);
 }
 
+/* One (token t, head hh) item of the projections' output, by one warp
+ * (heads: q heads, then k, then v): its K slices' split-K partials added
+ * in slice order into v[0..per), per = hd / 32 values per lane; q and k
+ * heads then RMS-normalised with their gains (QK-norm). */
+MSK_DEV void qkv_head(const Ctx& c, const MskLayer& Ly, int t, int hh, float* v) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31;
+  const int hd = P->hd, nqkv = P->qd + 2 * P->kvd, per = hd / 32;
+  const int S = P->d <= DKS_MAX ? 1 : P->d / DKS_MAX;
+  v[0] = v[1] = v[2] = v[3] = 0.f;
+#pragma unroll 4
+  for (int sl = 0; sl < S; ++sl) {
+    const float* raw = P->qkv + ((size_t)sl * c.st.T + t) * nqkv + hh * hd + lane * per;
+    if (per == 4) {
+      const float4 q = *reinterpret_cast<const float4*>(raw);
+      v[0] += q.x; v[1] += q.y; v[2] += q.z; v[3] += q.w;
+    } else {
+      const float2 q = *reinterpret_cast<const float2*>(raw);
+      v[0] += q.x; v[1] += q.y;
+    }
+  }
+  if (hh < P->hq + P->hkv) {
+    float ss = 0.f;
+    for (int i = 0; i < per; ++i) ss += v[i] * v[i];
+    ss = warp_sum(ss);
+    const float r = 1.0f / sqrtf(ss / hd + P->eps);
+    const float* gain = (hh < P->hq ? Ly.g_q : Ly.g_k) + lane * per;
+    for (int i = 0; i < per; ++i) v[i] = v[i] * r * gain[i];
+  }
+}
+
+/* This step's key or value of (token t, kv head kvh) as fp8 e4m3 into the
+ * cache (and, if captured, its fp32 value before the encode). */
+MSK_DEV void kv_store(const Ctx& c, int layer, int t, int kvh, bool isv, const float* v) {
+  const MskParams* P = c.P;
+  const int lane = threadIdx.x & 31, hd = P->hd, per = hd / 32;
+  const int b = t / c.st.Tq, ti = t % c.st.Tq;
+  float* pre = isv ? P->dbg_vpre : P->dbg_kpre;
+  if (pre) {
+    pre += ((size_t)layer * c.st.T + t) * P->kvd + kvh * hd + lane * per;
+    for (int i = 0; i < per; ++i) pre[i] = v[i];
+  }
+  const int64_t pos = c.S->pos0[b] + ti;
+  int64_t row = (((int64_t)layer * c.st.kv_seqs + b) * P->hkv + kvh) * c.st.kv_cap + pos;
+  if (isv) row += c.st.kv_half_rows;
+  uint8_t* dst = c.st.kv_base + row * hd + lane * per;
+  if (per == 4) {
+    uint32_t lo = f32x2_to_e4m3x2(v[0], v[1]), hi = f32x2_to_e4m3x2(v[2], v[3]);
+    *reinterpret_cast<uint32_t*>(dst) = lo | (hi << 16);
+  } else {
+    *reinterpret_cast<uint16_t*>(dst) = (uint16_t)f32x2_to_e4m3x2(v[0], v[1]);
+  }
+}
+
 /* ---- attention on the 5th-generation tensor cores (head dim 128) ------------------------ */
 /*
  * Per (sequence, kv head) segment of keys, with R = Tq * G query rows padded
@@ -1289,13 +1371,13 @@ MSK_DEV bool attention_phase(Cons& q, int layer) {
  * probabilities.  Parties and barriers per stage j (buffer b = j mod 2):
  *   producer -> afull -> issuer: QK(j) -> s_ready[b] -> consumers: widen V,
  *   read S^T -> s_free[b] -> issuer (QK(j+2)); consumers: write P^T ->
- *   p_ready[b] -> issuer: PV(j) -> aempty (stage refill) and pv_done[b]
+ *   p_ready[b3] -> issuer: PV(j) -> aempty (stage refill) and pv_done[b3]
  *   (P^T buffer reuse; the segment's output read).
  * Shared memory (from the ring base): NS stages of 32 KB (K at 0, V at 16 KB;
  * after widening, bf16 V: 8-key group g at 2 KB (g / 2) + 16 KB (g mod 2),
  * each [hd/64][key%8][128 B] with 128-byte swizzle, read MN-major with the
  * head-dim halves 1 KB apart and the two groups of an MMA 16 KB apart),
- * then two P^T buffers [2 key tiles][RP rows][128 B], then the Q terms
+ * then three P^T buffers (stage mod 3) [2 key tiles][RP rows][128 B], then the Q terms
  * [3][RP rows][128 B].  TMEM: O^T at column 0, S^T buffers at 64 and 256.
  */
 /* One issuing warp's part of one layer's attention (lane 0 issues): role 0
@@ -1331,11 +1413,11 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
       }
       __syncwarp();
     } else {
-      if (!pwait_bar(c, &c.S->p_ready[j & 1u], (j >> 1) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (!pwait_bar(c, &c.S->p_ready[j % 3u], (j / 3u) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (first && aseg > 0 && !pwait_bar(c, &c.S->o_free, (aseg - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t pt = ptoff + (j & 1u) * (uint32_t)RP * 256u;
+        const uint32_t pt = ptoff + (j % 3u) * (uint32_t)RP * 256u;
         const uint64_t va = umma_desc(ring + (j % NS) * ATC_STAGE, 1024, 16384, 2), pb0 = umma_desc(pt, 16, 1024, 2),
                        pb1 = umma_desc(pt + (uint32_t)RP * 128u, 16, 1024, 2);
 #pragma unroll
@@ -1343,7 +1425,7 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
           tc_mma_f16(tb + ATC_TM_O, va + (uint64_t)(128 * kk), (kk < 4 ? pb0 : pb1) + (uint64_t)(2 * (kk & 3)), id_pv,
                      (first && kk == 0) ? 0u : 1u);
         tc_commit(&c.S->aempty[j % NS]);
-        tc_commit(&c.S->pv_done[j & 1u]);
+        tc_commit(&c.S->pv_done[j % 3u]);
       }
       __syncwarp();
     }
@@ -1396,8 +1478,9 @@ MSK_DEV bool prod_att_tc_drain(Prod& p, int layer, uint32_t ait) {
   return true;
 }
 
-/* Q of the pair's R rows as three e4m3 terms (B operand rows t RP + rho,
- * 128-byte swizzle) and each row's softmax factor; one warp per row. */
+/* Q of the pair's R rows (QK-normed, f16) as three e4m3 terms (B operand
+ * rows t RP + rho, 128-byte swizzle) and each row's softmax factor; one
+ * warp per row. */
 MSK_DEV void atc_q_terms(const Ctx& c, int pair, int RP, uint32_t qoff) {
   const MskParams* P = c.P;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
@@ -1480,7 +1563,8 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
       for (int x = k0; x < k1; x += 128) {
         const uint32_t j = ait, bf = j & 1u, slot = j % NS;
         const int nkeys = min(128, k1 - x);
-        if (ok && j >= 2 && !wait_bar(c, &c.S->pv_done[bf], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) ok = false;
+        const uint32_t pb = j % 3u; /* P^T buffer: three, so a stage waits for the products of stage j - 3 */
+        if (ok && j >= 3 && !wait_bar(c, &c.S->pv_done[pb], ((j / 3u) - 1u) & 1u, layer, PH_ATT)) ok = false;
         if (ok && !wait_bar(c, &c.S->afull[slot], (j / NS) & 1u, layer, PH_ATT)) ok = false;
         if (ok && !wait_bar(c, &c.S->s_ready[bf], (j >> 1) & 1u, layer, PH_ATT)) ok = false;
         ok = __all_sync(0xffffffffu, ok) != 0; /* warp-uniform: the TMEM loads below are warp-collective */
@@ -1539,7 +1623,7 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
           /* P^T element (row rho, key): tile key / 64, row rho (rho mod 8 = i mod 8
            * since NR is a multiple of 8), 16-byte chunk (key mod 64) / 8 xor rho mod 8 */
           const uint32_t kk = (uint32_t)(key & 63), c8 = kk >> 3;
-          const uint32_t pt = ptoff + bf * (uint32_t)RP * 256u + (uint32_t)(key >> 6) * (uint32_t)RP * 128u +
+          const uint32_t pt = ptoff + pb * (uint32_t)RP * 256u + (uint32_t)(key >> 6) * (uint32_t)RP * 128u +
                               (uint32_t)(hh * NR) * 128u + 2u * (kk & 7u);
           float pv[NR];
           if (full) {
@@ -1562,12 +1646,12 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
         }
         fence_proxy_async_shared();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&c.S->p_ready[bf]);
+        if (lane == 0) mbar_arrive(&c.S->p_ready[pb]);
         ait++;
       }
       /* segment end: the output accumulator after the last stage's products */
       const uint32_t jl = ait - 1u;
-      if (ok && !wait_bar(c, &c.S->pv_done[jl & 1u], (jl >> 1) & 1u, layer, PH_ATT)) ok = false;
+      if (ok && !wait_bar(c, &c.S->pv_done[jl % 3u], (jl / 3u) & 1u, layer, PH_ATT)) ok = false;
       ok = __all_sync(0xffffffffu, ok) != 0;
       tc_fence_after();
       const int slotp = c.cta + pr;
@@ -1737,54 +1821,17 @@ MSK_DEV void phase_qknorm(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
   const int lane = threadIdx.x & 31;
-  const int hd = P->hd, nh = P->hq + 2 * P->hkv, nqkv = P->qd + 2 * P->kvd;
-  const int per = hd / 32; /* 4 or 2 values per lane */
+  const int hd = P->hd, nh = P->hq + 2 * P->hkv, per = hd / 32;
   for (int item = gwarp(c); item < c.st.T * nh; item += nwarps(c)) {
     const int t = item / nh, hh = item % nh;
-    /* the projection: its K slices' partials added in slice order */
-    const int S = P->d <= DKS_MAX ? 1 : P->d / DKS_MAX;
-    float v[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 4
-    for (int sl = 0; sl < S; ++sl) {
-      const float* raw = P->qkv + ((size_t)sl * c.st.T + t) * nqkv + hh * hd + lane * per;
-      if (per == 4) {
-        const float4 q = *reinterpret_cast<const float4*>(raw);
-        v[0] += q.x; v[1] += q.y; v[2] += q.z; v[3] += q.w;
-      } else {
-        const float2 q = *reinterpret_cast<const float2*>(raw);
-        v[0] += q.x; v[1] += q.y;
-      }
-    }
-    const int b = t / c.st.Tq, ti = t % c.st.Tq;
-    if (hh < P->hq + P->hkv) {
-      float ss = 0.f;
-      for (int i = 0; i < per; ++i) ss += v[i] * v[i];
-      ss = warp_sum(ss);
-      const float r = 1.0f / sqrtf(ss / hd + P->eps);
-      const float* gain = (hh < P->hq ? Ly.g_q : Ly.g_k) + lane * per;
-      for (int i = 0; i < per; ++i) v[i] = v[i] * r * gain[i];
-    }
+    float v[4];
+    qkv_head(c, Ly, t, hh, v);
     if (hh < P->hq) {
       uint16_t* dst = P->qs + (size_t)t * P->qd + hh * hd + lane * per;
       for (int i = 0; i < per; ++i) dst[i] = f32_to_f16(v[i]);
     } else {
       const int isv = hh >= P->hq + P->hkv;
-      const int kvh = hh - P->hq - (isv ? P->hkv : 0);
-      float* pre = isv ? P->dbg_vpre : P->dbg_kpre;
-      if (pre) {
-        pre += ((size_t)layer * c.st.T + t) * P->kvd + kvh * hd + lane * per;
-        for (int i = 0; i < per; ++i) pre[i] = v[i];
-      }
-      const int64_t pos = c.S->pos0[b] + ti;
-      int64_t row = (((int64_t)layer * c.st.kv_seqs + b) * P->hkv + kvh) * c.st.kv_cap + pos;
-      if (isv) row += c.st.kv_half_rows;
-      uint8_t* dst = c.st.kv_base + row * hd + lane * per;
-      if (per == 4) {
-        uint32_t lo = f32x2_to_e4m3x2(v[0], v[1]), hi = f32x2_to_e4m3x2(v[2], v[3]);
-        *reinterpret_cast<uint32_t*>(dst) = lo | (hi << 16);
-      } else {
-        *reinterpret_cast<uint16_t*>(dst) = (uint16_t)f32x2_to_e4m3x2(v[0], v[1]);
-      }
+      kv_store(c, layer, t, hh - P->hq - (isv ? P->hkv : 0), isv, v);
     }
   }
   fence_proxy_async_global();
@@ -2259,7 +2306,6 @@ MSK_DEV bool expert_mma(Ctx& c, int layer, uint32_t& xpar) {
   const MskLayer& Ly = P->layers[layer];
   const Route& R = c.S->route;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
-  const int ctid = threadIdx.x - CONS0;
   const int phase = GU ? PH_GU : PH_DN;
   XGeo x;
   xgeo(c, GU ? XP_CC : XP_DN, x);
@@ -2281,8 +2327,10 @@ MSK_DEV bool expert_mma(Ctx& c, int layer, uint32_t& xpar) {
       if (ok)
         xgemm<GU ? 2 : 1>(slot + cw * 16 * x.cpitch, slot + XROWS * x.cpitch + cw * 16 * x.spitch, x.mat_bytes,
                           x.cpitch, x.spitch, slot + x.b_off, x.bpitch, x.KC, acc, acc2);
-      named_sync(BAR_CONS, NCT);
-      if (ok && ctid < 2) mbar_arrive(&c.S->xempty[s]); /* the slot's two arrivals */
+      /* each warp releases the slot when it is done with it: no CTA barrier
+       * per chunk; the producer refills once all eight have arrived */
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&c.S->xempty_cc[s]);
     }
     if (!ok) continue;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
@@ -2392,7 +2440,8 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     mbar_init(&c.S->rfull, 1);
     for (int i = 0; i < XNS_MAX; ++i) {
       mbar_init(&c.S->xfull[i], 1);
-      mbar_init(&c.S->xempty[i], 2); /* two tensor-core commits, or two consumer threads */
+      mbar_init(&c.S->xempty[i], 2);  /* two tensor-core commits */
+      mbar_init(&c.S->xempty_cc[i], NCW);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.S->dfull2[i], 2); /* both issuing roles commit */
@@ -2406,6 +2455,8 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.S->s_ready[i], 1);
       mbar_init(&c.S->s_free[i], NCW);
+    }
+    for (int i = 0; i < 3; ++i) {
       mbar_init(&c.S->p_ready[i], NCW);
       mbar_init(&c.S->pv_done[i], 1);
     }
