@@ -406,18 +406,26 @@ MSK_DEV void for_each_att_stage(const Ctx& c, const AttGeo& g, F&& f) {
 
 /* tensor-core attention geometry (see attention_phase_tc) */
 constexpr uint32_t ATC_STAGE = 32768;
-constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64, ATC_TM_SSTRIDE = 192;
+/* TMEM columns: O^T, two S^T buffers, the V scale factors (all 1), and three
+ * buffers of the P^T scale factors (two terms, 4 columns each: a block-scaled
+ * MMA takes scale-factor addresses that are multiples of 4 columns) */
+constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64, ATC_TM_SSTRIDE = 192, ATC_TM_SFA = 448, ATC_TM_SFB = 452;
+static_assert(ATC_TM_S + 2 * ATC_TM_SSTRIDE <= ATC_TM_SFA && ATC_TM_SFB + 3 * 8 <= 512 && ATC_TM_SFB % 4 == 0, "TMEM");
 MSK_DEV int atc_ns(int RP) { return RP > 32 ? 4 : 5; }
 MSK_DEV uint32_t atc_pt_off(int RP) { return (uint32_t)atc_ns(RP) * ATC_STAGE; }
 MSK_DEV uint32_t atc_q_off(int RP) { return atc_pt_off(RP) + 3u * (uint32_t)RP * 256u; }
+/* scale-factor atoms: [3 buffers][2 terms][32 rows][16 B], then 512 B of ue8m0 1.0 */
+MSK_DEV uint32_t atc_sf_off(int RP) { return atc_q_off(RP) + 3u * (uint32_t)RP * 128u; }
+constexpr uint32_t ATC_SF_BYTES = 3 * 1024 + 512;
 MSK_DEV int atc_rp(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 64); }
-static_assert(4 * ATC_STAGE + 3 * 64 * 256 + 3 * 64 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
-static_assert(5 * ATC_STAGE + 3 * 32 * 256 + 3 * 32 * 128 <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
-/* instruction descriptors: fp32 accumulators, M = 128, N = RP; QK e4m3 x e4m3
- * both K-major; PV bf16 x bf16 with A MN-major */
+static_assert(4 * ATC_STAGE + 3 * 64 * 256 + 3 * 64 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
+static_assert(5 * ATC_STAGE + 3 * 32 * 256 + 3 * 32 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
+/* instruction descriptors, M = 128, fp32 accumulators.  QK: kind::f8f6f4,
+ * e4m3 x e4m3, both K-major, N = 3 RP.  PV: kind::mxf8f6f4 block32, e4m3 x
+ * e4m3, both MN-major, ue8m0 scales, N = RP, scale byte kk of B's words. */
 MSK_DEV uint32_t atc_idesc_qk(int RP) { return (1u << 4) | ((uint32_t)((3 * RP) >> 3) << 17) | ((128u >> 4) << 24); }
-MSK_DEV uint32_t atc_idesc_pv(int RP) {
-  return (1u << 4) | (1u << 7) | (1u << 10) | (1u << 15) | ((uint32_t)(RP >> 3) << 17) | ((128u >> 4) << 24);
+MSK_DEV uint32_t atc_idesc_pv(int RP, uint32_t kk) {
+  return (kk << 4) | (1u << 15) | (1u << 16) | ((uint32_t)(RP >> 3) << 17) | (1u << 23) | ((128u >> 4) << 24);
 }
 
 /* ---- producer ---------------------------------------------------------------------- */
@@ -1360,25 +1368,33 @@ MSK_DEV void kv_store(const Ctx& c, int layer, int t, int kvh, bool isv, const f
  *     costs about the same up to N = 128, and K is read once); the consumer
  *     adds a row's three term columns.
  *   p = exp(s - M) under the key windows, on CUDA cores: each consumer
- *     lane holds one key (TMEM lane), its rows' scores; l += p per lane;
- *     P^T is written to shared memory as bf16 scaled by 2^120.
- *   O^T[128 hd][RP] += V^T P^T: kind::f16 (bf16), A = the stage's V widened
- *     in place to bf16 x 2^-120 (an exact bit move) and read MN-major
- *     (head-dim contiguous, no transpose), B = P^T (K-major); 8 MMAs of
- *     K = 16 keys per stage, accumulated in TMEM over the segment.
- * The MMA-issuing warp runs one stage ahead: the QK products of stage j+1
- * are in flight while the consumer warps turn the scores of stage j into
- * probabilities.  Parties and barriers per stage j (buffer b = j mod 2):
- *   producer -> afull -> issuer: QK(j) -> s_ready[b] -> consumers: widen V,
- *   read S^T -> s_free[b] -> issuer (QK(j+2)); consumers: write P^T ->
- *   p_ready[b3] -> issuer: PV(j) -> aempty (stage refill) and pv_done[b3]
- *   (P^T buffer reuse; the segment's output read).
- * Shared memory (from the ring base): NS stages of 32 KB (K at 0, V at 16 KB;
- * after widening, bf16 V: 8-key group g at 2 KB (g / 2) + 16 KB (g mod 2),
- * each [hd/64][key%8][128 B] with 128-byte swizzle, read MN-major with the
- * head-dim halves 1 KB apart and the two groups of an MMA 16 KB apart),
- * then three P^T buffers (stage mod 3) [2 key tiles][RP rows][128 B], then the Q terms
- * [3][RP rows][128 B].  TMEM: O^T at column 0, S^T buffers at 64 and 256.
+ *     lane holds one key (TMEM lane), its rows' scores; l += p per lane.
+ *     P^T goes to shared memory as two e4m3 terms per value under one ue8m0
+ *     scale per (row, 32-key block): the block's largest p sets the scale
+ *     so that p / scale lies below 256; t0 = e4m3(p / scale) and t1 =
+ *     e4m3(16 (p / scale - t0)) with scale / 16 (about 9 significant bits,
+ *     as bf16; p spans up to 2^-116 .. 1, which one fixed e4m3 scale cannot).
+ *   O^T[128 hd][RP] += V^T P^T: kind::mxf8f6f4 block32, A = the stage's V
+ *     exactly as the tensor copy lands it (e4m3, key rows of 128 bytes,
+ *     128-byte swizzle), read MN-major (head-dim contiguous); B = a P^T term,
+ *     MN-major without swizzle (core matrices [8 keys][16 rows]); V's
+ *     scales all 1.  8 MMAs of K = 32 keys per stage (2 terms x 4 key
+ *     blocks), accumulated in TMEM over the segment.
+ * The QK issuer runs one stage ahead: the QK products of stage j+1 are in
+ * flight while the consumer warps turn the scores of stage j into
+ * probabilities.  Parties and barriers per stage j (b = j mod 2, b3 = j mod 3):
+ *   producer -> afull -> issuer: QK(j) -> s_ready[b] -> consumers: read S^T
+ *   -> s_free[b] -> issuer (QK(j+2)); consumers: write P^T terms and their
+ *   scales -> p_ready[b3] -> issuer: scales into TMEM, PV(j) -> aempty
+ *   (stage refill) and pv_done[b3] (P^T buffer reuse; the segment's output
+ *   read).  The consumers never touch a stage's K or V.
+ * Shared memory (from the ring base): NS stages of 32 KB (K at 0, V at 16 KB),
+ * then three P^T buffers (stage mod 3) [2 terms][16 key groups][RP / 16 row
+ * groups][8 keys][16 rows] e4m3, the Q terms [3][RP rows][128 B], then the
+ * scale-factor atoms [3][2 terms][32 rows][16 B] (row n: atom row n mod 32,
+ * word n / 32, byte = key block) and 512 bytes of ue8m0 1.0 for V.  TMEM:
+ * O^T at column 0, S^T buffers at 64 and 256, V scales at 448, P^T scales
+ * at 452 + 8 b3 + 4 term.
  */
 /* One issuing warp's part of one layer's attention (lane 0 issues): role 0
  * issues every stage's QK products, role 1 its PV products, so the two
@@ -1393,10 +1409,10 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
   const AttGeo& g = c.S->ag;
   const int RP = atc_rp(c.st.Tq * P->G), NS = atc_ns(RP);
   const uint32_t tb = c.S->tmem_base, ring = smem_u32(c.ring);
-  const uint32_t qoff = ring + atc_q_off(RP), ptoff = ring + atc_pt_off(RP);
-  const uint32_t id_qk = atc_idesc_qk(RP), id_pv = atc_idesc_pv(RP);
+  const uint32_t qoff = ring + atc_q_off(RP), ptoff = ring + atc_pt_off(RP), sfoff = ring + atc_sf_off(RP);
+  const uint32_t id_qk = atc_idesc_qk(RP);
   const uint64_t qb = umma_desc(qoff, 16, 1024, 2);
-  bool ok = true;
+  bool ok = true, sfa = false;
   for_each_att_stage(c, g, [&](int, int, int64_t, int, bool first, bool last) {
     const uint32_t j = ait;
     if (role == 0) {
@@ -1417,16 +1433,27 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
       if (first && aseg > 0 && !pwait_bar(c, &c.S->o_free, (aseg - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (lane == 0) {
         tc_fence_after();
-        const uint32_t pt = ptoff + (j % 3u) * (uint32_t)RP * 256u;
-        const uint64_t va = umma_desc(ring + (j % NS) * ATC_STAGE, 1024, 16384, 2), pb0 = umma_desc(pt, 16, 1024, 2),
-                       pb1 = umma_desc(pt + (uint32_t)RP * 128u, 16, 1024, 2);
+        const uint32_t b3 = j % 3u, pt = ptoff + b3 * (uint32_t)RP * 256u, sfb = tb + ATC_TM_SFB + 8u * b3;
+        /* the scale factors into TMEM (V's once per layer), in issue order
+         * before the MMAs that read them */
+        if (!sfa) tc_cp_sf(tb + ATC_TM_SFA, umma_desc(sfoff + 3072u, 16, 128, 0));
+        tc_cp_sf(sfb, umma_desc(sfoff + b3 * 1024u, 16, 128, 0));
+        tc_cp_sf(sfb + 4u, umma_desc(sfoff + b3 * 1024u + 512u, 16, 128, 0));
+        /* A: V, one 128-byte atom along the head dim, 8-key groups 1 KB apart;
+         * B: term t, key groups RP * 8 bytes apart, 16-row groups 128 bytes */
+        const uint64_t va = umma_desc(ring + (j % NS) * ATC_STAGE + 16384u, 8192, 1024, 2);
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          tc_mma_f16(tb + ATC_TM_O, va + (uint64_t)(128 * kk), (kk < 4 ? pb0 : pb1) + (uint64_t)(2 * (kk & 3)), id_pv,
-                     (first && kk == 0) ? 0u : 1u);
+        for (int t = 0; t < 2; ++t) {
+          const uint64_t pbt = umma_desc(pt + (uint32_t)(t * RP * 128), (uint32_t)RP * 8u, 128, 0);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            tc_mma_mx8(tb + ATC_TM_O, va + (uint64_t)(256 * kk), pbt + (uint64_t)(2 * RP * kk), atc_idesc_pv(RP, (uint32_t)kk),
+                       (first && t == 0 && kk == 0) ? 0u : 1u, tb + ATC_TM_SFA, sfb + 4u * (uint32_t)t);
+        }
         tc_commit(&c.S->aempty[j % NS]);
-        tc_commit(&c.S->pv_done[j % 3u]);
+        tc_commit(&c.S->pv_done[b3]);
       }
+      sfa = true;
       __syncwarp();
     }
     ait++;
@@ -1522,7 +1549,6 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
   const MskParams* P = c.P;
   const MskLayer& Ly = P->layers[layer];
   constexpr int NR = RP / 2; /* query rows per consumer warp */
-  constexpr int NS = RP > 32 ? 4 : 5;
   att_geo_shared(c, layer);
   if (threadIdx.x == CONS0) {
     __threadfence_block();
@@ -1533,12 +1559,13 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
   const int qd = cw & 3, hh = cw >> 2; /* TMEM lane quadrant (keys 32 qd ..), row half */
   const int R = c.st.Tq * P->G;
   const uint32_t ring = smem_u32(c.ring), tb = c.S->tmem_base;
-  const uint32_t ptoff = ring + atc_pt_off(RP), qoff = ring + atc_q_off(RP);
+  const uint32_t ptoff = ring + atc_pt_off(RP), qoff = ring + atc_q_off(RP), sfoff = ring + atc_sf_off(RP);
   const float bound_log2 = Ly.bound_log2;
-  const float two120 = 1.329227995784916e36f; /* 2^120 */
   const bool sliding = Ly.sliding != 0;
   float* lred = reinterpret_cast<float*>(c.S->lbuf); /* [4 quadrants][64 rows] */
   bool ok = true;
+  /* V's block scales, ue8m0 1.0 (published with the first segment's Q terms) */
+  if (ctid < 128) sts32(sfoff + 3072u + 4u * (uint32_t)ctid, 0x7F7F7F7Fu);
   if (c.cta < g.nparts) {
     const int64_t A0 = g.N * c.cta / g.nparts, B0 = g.N * (c.cta + 1) / g.nparts;
     for (int pr = 0; pr < g.npairs; ++pr) {
@@ -1561,57 +1588,34 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
       }
       const int nvalid = min(NR, max(0, R - hh * NR)); /* this warp's rows below R */
       for (int x = k0; x < k1; x += 128) {
-        const uint32_t j = ait, bf = j & 1u, slot = j % NS;
+        const uint32_t j = ait, bf = j & 1u, pb = j % 3u;
         const int nkeys = min(128, k1 - x);
-        const uint32_t pb = j % 3u; /* P^T buffer: three, so a stage waits for the products of stage j - 3 */
+        /* P^T buffer pb and its scale atoms: free once the products of stage j - 3 completed */
         if (ok && j >= 3 && !wait_bar(c, &c.S->pv_done[pb], ((j / 3u) - 1u) & 1u, layer, PH_ATT)) ok = false;
-        if (ok && !wait_bar(c, &c.S->afull[slot], (j / NS) & 1u, layer, PH_ATT)) ok = false;
         if (ok && !wait_bar(c, &c.S->s_ready[bf], (j >> 1) & 1u, layer, PH_ATT)) ok = false;
         ok = __all_sync(0xffffffffu, ok) != 0; /* warp-uniform: the TMEM loads below are warp-collective */
         tc_fence_after();
-        /* V of the stage, widened in place: warp w owns keys 16 w .. 16 w + 15,
-         * whose fp8 V (2 KB at 16 KB + 2 KB w) and fp8 K (2 KB at 2 KB w, free
-         * once the QK products are done) it overwrites with their bf16 V, so
-         * no other warp's bytes are touched and a warp barrier suffices.  Its
-         * lanes read 16-byte chunks (key 16 w + lane / 8 + 4 u, head-dim chunk
-         * lane mod 8). */
-        const uint32_t sb = ring + slot * ATC_STAGE;
-        uint4 vv[4];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int k = 16 * cw + (lane >> 3) + 4 * u, ch = lane & 7;
-          vv[u] = ok ? lds128(sb + 16384u + (uint32_t)k * 128u + ((uint32_t)(ch ^ (k & 7)) << 4)) : make_uint4(0, 0, 0, 0);
-        }
-        __syncwarp();
-        if (ok) {
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int kl = (lane >> 3) + 4 * u, k = 16 * cw + kl, ch = lane & 7;
-            /* 8-key group 2 w (keys 16 w ..) in the K bytes, group 2 w + 1 in
-             * the V bytes; then [hd / 64][key mod 8][128 B], 128-byte swizzle */
-            const uint32_t dst = sb + (kl < 8 ? 0u : 16384u) + (uint32_t)cw * 2048u + (uint32_t)(ch >> 2) * 1024u +
-                                 (uint32_t)(k & 7) * 128u;
-            const uint32_t c0 = (uint32_t)(2 * (ch & 3)), c1 = c0 + 1u, sw = (uint32_t)(k & 7);
-            sts128(dst + ((c0 ^ sw) << 4), e4m3x2_to_bf16x2_scaled(vv[u].x, 0), e4m3x2_to_bf16x2_scaled(vv[u].x, 1),
-                   e4m3x2_to_bf16x2_scaled(vv[u].y, 0), e4m3x2_to_bf16x2_scaled(vv[u].y, 1));
-            sts128(dst + ((c1 ^ sw) << 4), e4m3x2_to_bf16x2_scaled(vv[u].z, 0), e4m3x2_to_bf16x2_scaled(vv[u].z, 1),
-                   e4m3x2_to_bf16x2_scaled(vv[u].w, 0), e4m3x2_to_bf16x2_scaled(vv[u].w, 1));
-          }
-        }
         /* this warp's scores: its quadrant's 32 keys, its NR rows, the sum
          * of each row's three term columns */
         float sr[NR];
         if (ok) {
           const uint32_t ta = tb + ATC_TM_S + ATC_TM_SSTRIDE * bf + (uint32_t)(hh * NR) + ((uint32_t)(qd * 32) << 16);
+          constexpr int NB = NR < 16 ? NR : 16;
 #pragma unroll
-          for (int i = 0; i < NR; i += 8) {
-            uint32_t t0[8], t1[8], t2[8];
-            tc_ld8(ta + (uint32_t)i, t0);
-            tc_ld8(ta + (uint32_t)(RP + i), t1);
-            tc_ld8(ta + (uint32_t)(2 * RP + i), t2);
+          for (int i = 0; i < NR; i += NB) {
+            uint32_t t0[NB], t1[NB], t2[NB];
+            if constexpr (NB == 16) {
+              tc_ld16(ta + (uint32_t)i, t0);
+              tc_ld16(ta + (uint32_t)(RP + i), t1);
+              tc_ld16(ta + (uint32_t)(2 * RP + i), t2);
+            } else {
+              tc_ld8(ta + (uint32_t)i, t0);
+              tc_ld8(ta + (uint32_t)(RP + i), t1);
+              tc_ld8(ta + (uint32_t)(2 * RP + i), t2);
+            }
             tc_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 8; ++e) sr[i + e] = __uint_as_float(t0[e]) + __uint_as_float(t1[e]) + __uint_as_float(t2[e]);
+            for (int e = 0; e < NB; ++e) sr[i + e] = __uint_as_float(t0[e]) + __uint_as_float(t1[e]) + __uint_as_float(t2[e]);
           }
         }
         tc_fence_before();
@@ -1620,11 +1624,6 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
         if (ok) {
           const int key = qd * 32 + lane, kp = x + key;
           const bool full = nkeys == 128 && x >= lo_max && x + 127 <= hi_min;
-          /* P^T element (row rho, key): tile key / 64, row rho (rho mod 8 = i mod 8
-           * since NR is a multiple of 8), 16-byte chunk (key mod 64) / 8 xor rho mod 8 */
-          const uint32_t kk = (uint32_t)(key & 63), c8 = kk >> 3;
-          const uint32_t pt = ptoff + pb * (uint32_t)RP * 256u + (uint32_t)(key >> 6) * (uint32_t)RP * 128u +
-                              (uint32_t)(hh * NR) * 128u + 2u * (kk & 7u);
           float pv[NR];
           if (full) {
 #pragma unroll
@@ -1638,10 +1637,54 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
               pv[i] = valid ? fast_exp2(fmaf(sr[i], qf[i], -bound_log2)) : 0.f;
             }
           }
+          /* each row's block scale from its largest p over the warp's 32 keys
+           * (one key block): biased exponent E of the maximum, p 2^(134 - E)
+           * below 256, ue8m0 code E - 7 (E >= 11 keeps the second term's code
+           * E - 11 valid; p >= 2^-116 under the bound wherever it is not 0) */
+          uint32_t code = 0; /* lane i < NR: row hh NR + i */
 #pragma unroll
           for (int i = 0; i < NR; ++i) {
             l[i] += pv[i];
-            sts16(pt + (uint32_t)i * 128u + ((c8 ^ (uint32_t)(i & 7)) << 4), f32_to_bf16(pv[i] * two120));
+            const uint32_t m = __reduce_max_sync(0xffffffffu, __float_as_uint(pv[i]));
+            const int E = max((int)(m >> 23), 11);
+            pv[i] *= __uint_as_float((uint32_t)(261 - E) << 23);
+            if (lane == i) code = (uint32_t)(E - 7);
+          }
+          /* t0 = e4m3(x), t1 = e4m3(16 (x - t0)), x via f16 (exact differences) */
+          uint32_t w0[NR / 4], w1[NR / 4];
+#pragma unroll
+          for (int i = 0; i < NR; i += 2) {
+            const uint32_t h = f32x2_to_f16x2(pv[i], pv[i + 1]);
+            const uint32_t a = f16x2_to_e4m3x2(h);
+            const uint32_t r = f16x2_to_e4m3x2(hmul2(hsub2(h, e4m3x2_to_f16x2(a)), 0x4C004C00u)); /* x 16 */
+            if ((i & 2) == 0) {
+              w0[i >> 2] = a;
+              w1[i >> 2] = r;
+            } else {
+              w0[i >> 2] |= a << 16;
+              w1[i >> 2] |= r << 16;
+            }
+          }
+          /* the key's 16-byte row in its core matrices: key group key / 8,
+           * row group, key mod 8 */
+          const uint32_t pt = ptoff + pb * (uint32_t)RP * 256u + (uint32_t)(key >> 3) * (uint32_t)RP * 8u + (uint32_t)(key & 7) * 16u;
+          const uint32_t p1 = (uint32_t)RP * 128u; /* term 1 */
+          if constexpr (NR == 8) {
+            sts64(pt + 8u * (uint32_t)hh, w0[0], w0[1]);
+            sts64(pt + p1 + 8u * (uint32_t)hh, w1[0], w1[1]);
+          } else {
+#pragma unroll
+            for (int gq = 0; gq < NR / 16; ++gq) {
+              const uint32_t o = (uint32_t)(hh * (NR / 16) + gq) * 128u;
+              sts128(pt + o, w0[4 * gq], w0[4 * gq + 1], w0[4 * gq + 2], w0[4 * gq + 3]);
+              sts128(pt + p1 + o, w1[4 * gq], w1[4 * gq + 1], w1[4 * gq + 2], w1[4 * gq + 3]);
+            }
+          }
+          if (lane < NR) { /* the scales of row hh NR + lane: atom row n mod 32, word n / 32, byte qd */
+            const int n = hh * NR + lane;
+            const uint32_t sa = sfoff + pb * 1024u + (uint32_t)(n & 31) * 16u + (uint32_t)(n >> 5) * 4u + (uint32_t)qd;
+            sts8(sa, code);
+            sts8(sa + 512u, code - 4u);
           }
         }
         fence_proxy_async_shared();
