@@ -507,12 +507,19 @@ msk_status_t msk_kv_create(msk_handle_t* h, int n_seqs, int64_t capacity, msk_kv
     cudaSetDevice(prev);
     return MSK_ERR_CUDA;
   }
+  /* head dim 64: one box per attention stage, C positions of one (layer,
+   * sequence, kv head) row range with K and V together (the third
+   * dimension steps from the K half of the cache to the V half), 32 KB.
+   * Head dim 128: one box is K or V of 128 positions (16 KB); the two go to
+   * separate rings. */
   const int C = P.hd == 128 ? 128 : 256;
-  cuuint64_t dims[2] = {(cuuint64_t)P.hd, (cuuint64_t)(2 * half_rows)};
-  cuuint64_t strides[1] = {(cuuint64_t)P.hd};
-  cuuint32_t box[2] = {(cuuint32_t)P.hd, (cuuint32_t)C};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&kv->map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kv->base, dims, strides, box, estr,
+  const cuuint32_t rank = P.hd == 128 ? 2 : 3;
+  cuuint64_t dims[3] = {(cuuint64_t)P.hd, (cuuint64_t)half_rows, 2};
+  cuuint64_t strides[2] = {(cuuint64_t)P.hd, (cuuint64_t)half_rows * (cuuint64_t)P.hd};
+  cuuint32_t box[3] = {(cuuint32_t)P.hd, (cuuint32_t)C, 2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (rank == 2) dims[1] = (cuuint64_t)(2 * half_rows);
+  CUresult r = enc(&kv->map, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, kv->base, dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE,
                    P.hd == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -103,8 +103,10 @@ struct Smem {
   volatile int abort;
   /* attention on the tensor cores (head dim 128): stage ring, score and
    * probability buffers, Q terms, output accumulator handoff */
-  uint64_t afull[5];        /* K and V of a stage landed (producer's expect-tx) */
-  uint64_t aempty[5];       /* the stage's P.V products completed (tensor-core commit) */
+  uint64_t kfull[6];        /* a stage's K landed (producer's expect-tx) */
+  uint64_t kempty[6];       /* its QK products completed (tensor-core commit) */
+  uint64_t vfull[6];        /* a stage's V landed */
+  uint64_t vempty[6];       /* its P.V products completed */
   uint64_t s_ready[2];      /* scores S^T of buffer b computed */
   uint64_t s_free[2];       /* S^T of buffer b read by every consumer warp */
   uint64_t p_ready[3];      /* P^T of buffer b (stage mod 3) and the stage's bf16 V written by every consumer warp */
@@ -146,21 +148,33 @@ MSK_DEV void raise_err(const Ctx& c, uint32_t code, int layer, int phase) {
   c.S->abort = 1;
 }
 
+/* Waits consult the abort word and the timer only every WAIT_POLL SM
+ * cycles (about 2 us): the abort word is in global memory, and a global
+ * load behind a full copy stream takes about a microsecond, during which a
+ * wait could not see its barrier complete.  A wait therefore runs up to
+ * WAIT_POLL cycles past its limit. */
+constexpr long long WAIT_POLL = 4096;
+
 /* bounded mbarrier wait; false on timeout or abort.  `mult` scales the
  * limit: the producer's waits on the consumers' progress take twice the
  * limit of the consumers' own waits, so that when a step stalls, the wait
  * nearest the cause gives up first and its site is the one recorded. */
 MSK_DEV bool wait_bar(const Ctx& c, uint64_t* bar, uint32_t parity, int layer, int phase, uint32_t mult = 1) {
   if (mbar_try(bar, parity)) return true;
-  uint64_t t0 = gtimer();
-  for (uint32_t it = 0;; ++it) {
+  long long next = clock64() + WAIT_POLL;
+  uint64_t t0 = 0;
+  for (;;) {
     if (mbar_try(bar, parity)) return true;
-    if ((it & 63) == 0) {
+    const long long now = clock64();
+    if (now >= next) {
       if (aborted(c)) return false;
-      if (gtimer() - t0 > mult * (uint64_t)c.P->timeout_ns) {
+      const uint64_t t = gtimer();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > mult * (uint64_t)c.P->timeout_ns) {
         raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
         return false;
       }
+      next = now + WAIT_POLL;
     }
   }
 }
@@ -405,21 +419,26 @@ MSK_DEV void for_each_att_stage(const Ctx& c, const AttGeo& g, F&& f) {
 }
 
 /* tensor-core attention geometry (see attention_phase_tc) */
-constexpr uint32_t ATC_STAGE = 32768;
+constexpr uint32_t ATC_HALF = 16384; /* K or V of a stage: 128 keys x 128 bytes */
 /* TMEM columns: O^T, two S^T buffers, the V scale factors (all 1), and three
  * buffers of the P^T scale factors (two terms, 4 columns each: a block-scaled
  * MMA takes scale-factor addresses that are multiples of 4 columns) */
 constexpr uint32_t ATC_TM_O = 0, ATC_TM_S = 64, ATC_TM_SSTRIDE = 192, ATC_TM_SFA = 448, ATC_TM_SFB = 452;
 static_assert(ATC_TM_S + 2 * ATC_TM_SSTRIDE <= ATC_TM_SFA && ATC_TM_SFB + 3 * 8 <= 512 && ATC_TM_SFB % 4 == 0, "TMEM");
-MSK_DEV int atc_ns(int RP) { return RP > 32 ? 4 : 5; }
-MSK_DEV uint32_t atc_pt_off(int RP) { return (uint32_t)atc_ns(RP) * ATC_STAGE; }
+/* K and V come in separate rings (K is free once its QK products are
+ * done, two stages before V): slots per ring by RP */
+MSK_DEV int atc_nk(int RP) { return RP > 32 ? 4 : (RP > 16 ? 4 : 5); }
+MSK_DEV int atc_nv(int RP) { return RP > 32 ? 4 : 6; }
+MSK_DEV uint32_t atc_v_off(int RP) { return (uint32_t)atc_nk(RP) * ATC_HALF; }
+MSK_DEV uint32_t atc_pt_off(int RP) { return (uint32_t)(atc_nk(RP) + atc_nv(RP)) * ATC_HALF; }
 MSK_DEV uint32_t atc_q_off(int RP) { return atc_pt_off(RP) + 3u * (uint32_t)RP * 256u; }
 /* scale-factor atoms: [3 buffers][2 terms][32 rows][16 B], then 512 B of ue8m0 1.0 */
 MSK_DEV uint32_t atc_sf_off(int RP) { return atc_q_off(RP) + 3u * (uint32_t)RP * 128u; }
 constexpr uint32_t ATC_SF_BYTES = 3 * 1024 + 512;
 MSK_DEV int atc_rp(int R) { return R <= 16 ? 16 : (R <= 32 ? 32 : 64); }
-static_assert(4 * ATC_STAGE + 3 * 64 * 256 + 3 * 64 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
-static_assert(5 * ATC_STAGE + 3 * 32 * 256 + 3 * 32 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
+static_assert(8 * ATC_HALF + 3 * 64 * 256 + 3 * 64 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 64 fits");
+static_assert(10 * ATC_HALF + 3 * 32 * 256 + 3 * 32 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 32 fits");
+static_assert(11 * ATC_HALF + 3 * 16 * 256 + 3 * 16 * 128 + ATC_SF_BYTES <= MSK_NST * MSK_STAGE + MSK_SCR, "RP 16 fits");
 /* instruction descriptors, M = 128, fp32 accumulators.  QK: kind::f8f6f4,
  * e4m3 x e4m3, both K-major, N = 3 RP.  PV: kind::mxf8f6f4 block32, e4m3 x
  * e4m3, both MN-major, ue8m0 scales, N = RP, scale byte kk of B's words. */
@@ -432,7 +451,8 @@ MSK_DEV uint32_t atc_idesc_pv(int RP, uint32_t kk) {
 struct Prod {
   Ctx* c;
   uint32_t it;
-  uint32_t ait;   /* tensor-core attention stages issued */
+  uint32_t ait;   /* tensor-core attention stages issued (their K boxes) */
+  uint32_t avt;   /* their V boxes issued */
   uint32_t xpar;  /* bit s: parity of the fills of expert slot s so far */
   uint32_t xused; /* bit s: expert slot s filled at least once */
   uint32_t xptc;  /* bit s: parity of its block-scaled fills (released by the issuers' commits) */
@@ -472,16 +492,21 @@ MSK_DEV bool prod_drain(Prod& p, int layer, int phase) {
 
 /* a flag the consumers set: twice the consumers' limit (see wait_bar) */
 MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, int phase) {
-  uint64_t t0 = gtimer();
-  for (uint32_t it = 0; *flag < want; ++it) {
-    if ((it & 15) == 0) {
+  long long next = clock64() + WAIT_POLL;
+  uint64_t t0 = 0;
+  while (*flag < want) {
+    const long long now = clock64();
+    if (now >= next) {
       if (aborted(c)) return false;
-      if (gtimer() - t0 > 2 * (uint64_t)c.P->timeout_ns) {
+      const uint64_t t = gtimer();
+      if (t0 == 0) t0 = t;
+      else if (t - t0 > 2 * (uint64_t)c.P->timeout_ns) {
         raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
         return false;
       }
+      next = now + WAIT_POLL;
     }
-    __nanosleep(32);
+    __nanosleep(20);
   }
   __threadfence_block();
   return true;
@@ -759,6 +784,7 @@ MSK_DEV void producer(Ctx& c) {
   p.c = &c;
   p.it = 0;
   p.ait = 0;
+  p.avt = 0;
   p.xpar = 0;
   p.xused = 0;
   p.xptc = 0;
@@ -783,7 +809,7 @@ MSK_DEV void producer(Ctx& c) {
       /* tensor-core attention: its own stage ring; W_o tiles once every
        * stage's products have completed */
       if (!prod_att_tc(p, l, p.ait) || !prod_att_tc_drain(p, l, p.ait)) { p.ok = false; break; }
-    } else
+    } else {
     for_each_att_stage(c, g, [&](int pr, int slot, int64_t k0, int n, bool, bool) {
       int b = pr / P->hkv, h = pr % P->hkv;
       if (k0 + C > c.S->pos0[b]) {
@@ -795,14 +821,16 @@ MSK_DEV void producer(Ctx& c) {
       if (!prod_acquire(p, l, PH_ATT, &stg, &bar)) { p.ok = false; return false; }
       int64_t row = (((int64_t)l * c.st.kv_seqs + b) * P->hkv + h) * c.st.kv_cap + k0;
       const int lane = threadIdx.x & 31;
-      if (lane == 0) mbar_arrive_tx(bar, (uint32_t)(2 * C * hd));
+      if (lane == 0) {
+        mbar_arrive_tx(bar, (uint32_t)(2 * C * hd));
+        tma_3d_g2s(stg, c.kvmap, 0, (int32_t)row, 0, bar); /* K at 0, V at C hd */
+      }
       __syncwarp();
-      if (lane == 0) tma_2d_g2s(stg, c.kvmap, 0, (int32_t)row, bar);
-      else if (lane == 1) tma_2d_g2s(stg + C * hd, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), bar);
       (void)slot;
       (void)n;
       return true;
     });
+    }
     if (!p.ok) break;
     /* W_o tiles once every attention stage has been read */
     if (!prod_drain(p, l, PH_WO) || !prod_dense(p, l, false)) { p.ok = false; break; }
@@ -854,12 +882,15 @@ MSK_DEV void producer(Ctx& c) {
         if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
       }
     }
-    if (hd == 128) {
-      const uint32_t ns = (uint32_t)atc_ns(atc_rp(c.st.Tq * P->G)), na = p.ait < ns ? p.ait : ns;
-      for (uint32_t i = p.ait - na; i < p.ait; ++i) {
-        uint64_t t0 = gtimer();
-        while (!mbar_try(&c.S->afull[i % ns], (i / ns) & 1)) {
-          if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+    if (hd == 128) { /* every K and V copy issued */
+      const int RP = atc_rp(c.st.Tq * P->G);
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint32_t ns = (uint32_t)(kv ? atc_nv(RP) : atc_nk(RP)), it = kv ? p.avt : p.ait, na = it < ns ? it : ns;
+        for (uint32_t i = it - na; i < it; ++i) {
+          uint64_t t0 = gtimer();
+          while (!mbar_try(kv ? &c.S->vfull[i % ns] : &c.S->kfull[i % ns], (i / ns) & 1)) {
+            if (gtimer() - t0 > 2 * (uint64_t)P->timeout_ns) break;
+          }
         }
       }
     }
@@ -1383,12 +1414,15 @@ MSK_DEV void kv_store(const Ctx& c, int layer, int t, int kvh, bool isv, const f
  * The QK issuer runs one stage ahead: the QK products of stage j+1 are in
  * flight while the consumer warps turn the scores of stage j into
  * probabilities.  Parties and barriers per stage j (b = j mod 2, b3 = j mod 3):
- *   producer -> afull -> issuer: QK(j) -> s_ready[b] -> consumers: read S^T
- *   -> s_free[b] -> issuer (QK(j+2)); consumers: write P^T terms and their
- *   scales -> p_ready[b3] -> issuer: scales into TMEM, PV(j) -> aempty
- *   (stage refill) and pv_done[b3] (P^T buffer reuse; the segment's output
- *   read).  The consumers never touch a stage's K or V.
- * Shared memory (from the ring base): NS stages of 32 KB (K at 0, V at 16 KB),
+ *   producer -> kfull -> issuer: QK(j) -> s_ready[b] (consumers) and kempty
+ *   (K refill) -> consumers: read S^T -> s_free[b] -> issuer (QK(j+2));
+ *   consumers: write P^T terms and their scales -> p_ready[b3], producer ->
+ *   vfull -> issuer: scales into TMEM, PV(j) -> vempty (V refill) and
+ *   pv_done[b3] (P^T buffer reuse; the segment's output read).  The
+ *   consumers never touch K or V.  K and V have rings of their own because
+ *   K is released two stages before V: with one 32 KB stage per slot, too
+ *   few bytes were left in flight to cover the copy latency.
+ * Shared memory (from the ring base): NK K slots and NV V slots of 16 KB,
  * then three P^T buffers (stage mod 3) [2 terms][16 key groups][RP / 16 row
  * groups][8 keys][16 rows] e4m3, the Q terms [3][RP rows][128 B], then the
  * scale-factor atoms [3][2 terms][32 rows][16 B] (row n: atom row n mod 32,
@@ -1407,8 +1441,9 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
   const int lane = threadIdx.x & 31;
   if (!pwait_flag(c, &c.S->ag_ready, layer + 1, layer, PH_ATT)) return false;
   const AttGeo& g = c.S->ag;
-  const int RP = atc_rp(c.st.Tq * P->G), NS = atc_ns(RP);
-  const uint32_t tb = c.S->tmem_base, ring = smem_u32(c.ring);
+  const int RP = atc_rp(c.st.Tq * P->G);
+  const uint32_t NK = (uint32_t)atc_nk(RP), NV = (uint32_t)atc_nv(RP);
+  const uint32_t tb = c.S->tmem_base, ring = smem_u32(c.ring), vring = ring + atc_v_off(RP);
   const uint32_t qoff = ring + atc_q_off(RP), ptoff = ring + atc_pt_off(RP), sfoff = ring + atc_sf_off(RP);
   const uint32_t id_qk = atc_idesc_qk(RP);
   const uint64_t qb = umma_desc(qoff, 16, 1024, 2);
@@ -1417,19 +1452,21 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
     const uint32_t j = ait;
     if (role == 0) {
       if (first && !pwait_bar(c, &c.S->q_ready, aseg & 1u, layer, PH_ATT)) { ok = false; return false; }
-      if (!pwait_bar(c, &c.S->afull[j % NS], (j / NS) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (!pwait_bar(c, &c.S->kfull[j % NK], (j / NK) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (j >= 2 && !pwait_bar(c, &c.S->s_free[j & 1u], ((j >> 1) - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (lane == 0) {
         tc_fence_after();
         const uint32_t d = tb + ATC_TM_S + ATC_TM_SSTRIDE * (j & 1u);
-        const uint64_t ka = umma_desc(ring + (j % NS) * ATC_STAGE, 16, 1024, 2);
+        const uint64_t ka = umma_desc(ring + (j % NK) * ATC_HALF, 16, 1024, 2);
 #pragma unroll
         for (int s = 0; s < 4; ++s) tc_mma_f8(d, ka + (uint64_t)(2 * s), qb + (uint64_t)(2 * s), id_qk, s > 0 ? 1u : 0u);
         tc_commit(&c.S->s_ready[j & 1u]);
+        tc_commit(&c.S->kempty[j % NK]);
       }
       __syncwarp();
     } else {
       if (!pwait_bar(c, &c.S->p_ready[j % 3u], (j / 3u) & 1u, layer, PH_ATT)) { ok = false; return false; }
+      if (!pwait_bar(c, &c.S->vfull[j % NV], (j / NV) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (first && aseg > 0 && !pwait_bar(c, &c.S->o_free, (aseg - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
       if (lane == 0) {
         tc_fence_after();
@@ -1437,20 +1474,33 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
         /* the scale factors into TMEM (V's once per layer), in issue order
          * before the MMAs that read them */
         if (!sfa) tc_cp_sf(tb + ATC_TM_SFA, umma_desc(sfoff + 3072u, 16, 128, 0));
-        tc_cp_sf(sfb, umma_desc(sfoff + b3 * 1024u, 16, 128, 0));
-        tc_cp_sf(sfb + 4u, umma_desc(sfoff + b3 * 1024u + 512u, 16, 128, 0));
-        /* A: V, one 128-byte atom along the head dim, 8-key groups 1 KB apart;
-         * B: term t, key groups RP * 8 bytes apart, 16-row groups 128 bytes */
-        const uint64_t va = umma_desc(ring + (j % NS) * ATC_STAGE + 16384u, 8192, 1024, 2);
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          const uint64_t pbt = umma_desc(pt + (uint32_t)(t * RP * 128), (uint32_t)RP * 8u, 128, 0);
+        /* A: V, one 128-byte atom along the head dim, 8-key groups 1 KB apart */
+        const uint64_t va = umma_desc(vring + (j % NV) * ATC_HALF, 8192, 1024, 2);
+        if (RP <= 32) {
+          /* B: both terms stacked along N (2 RP rows), key groups 2 RP * 8
+           * bytes apart, 16-row groups 128 bytes; one scale atom */
+          tc_cp_sf(sfb, umma_desc(sfoff + b3 * 1024u, 16, 128, 0));
+          const uint64_t pbs = umma_desc(pt, 16u * (uint32_t)RP, 128, 0);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            tc_mma_mx8(tb + ATC_TM_O, va + (uint64_t)(256 * kk), pbt + (uint64_t)(2 * RP * kk), atc_idesc_pv(RP, (uint32_t)kk),
-                       (first && t == 0 && kk == 0) ? 0u : 1u, tb + ATC_TM_SFA, sfb + 4u * (uint32_t)t);
+            tc_mma_mx8(tb + ATC_TM_O, va + (uint64_t)(256 * kk), pbs + (uint64_t)(4 * RP * kk),
+                       atc_idesc_pv(2 * RP, (uint32_t)kk), (first && kk == 0) ? 0u : 1u, tb + ATC_TM_SFA, sfb);
+        } else {
+          /* B: term t, key groups RP * 8 bytes apart, 16-row groups 128
+           * bytes; a scale atom per term; both terms into the same columns */
+          tc_cp_sf(sfb, umma_desc(sfoff + b3 * 1024u, 16, 128, 0));
+          tc_cp_sf(sfb + 4u, umma_desc(sfoff + b3 * 1024u + 512u, 16, 128, 0));
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            const uint64_t pbt = umma_desc(pt + (uint32_t)(t * RP * 128), (uint32_t)RP * 8u, 128, 0);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              tc_mma_mx8(tb + ATC_TM_O, va + (uint64_t)(256 * kk), pbt + (uint64_t)(2 * RP * kk),
+                         atc_idesc_pv(RP, (uint32_t)kk), (first && t == 0 && kk == 0) ? 0u : 1u, tb + ATC_TM_SFA,
+                         sfb + 4u * (uint32_t)t);
+          }
         }
-        tc_commit(&c.S->aempty[j % NS]);
+        tc_commit(&c.S->vempty[j % NV]);
         tc_commit(&c.S->pv_done[b3]);
       }
       sfa = true;
@@ -1463,45 +1513,62 @@ MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& as
   return ok;
 }
 
-/* The producer's part: this CTA's K and V boxes into the stage ring. */
+/* The producer's part: this CTA's K and V boxes (16 KB each) into their
+ * rings, K of stage j before V of stage j - 1, so that K, which is needed
+ * first, runs a stage ahead.  p.avt counts the V boxes issued. */
 MSK_DEV bool prod_att_tc(Prod& p, int layer, uint32_t& ait) {
   Ctx& c = *p.c;
   const MskParams* P = c.P;
   const AttGeo& g = c.S->agp;
-  const int RP = atc_rp(c.st.Tq * P->G), NS = atc_ns(RP);
+  const int RP = atc_rp(c.st.Tq * P->G);
+  const uint32_t NK = (uint32_t)atc_nk(RP), NV = (uint32_t)atc_nv(RP);
+  uint8_t* vring = c.ring + atc_v_off(RP);
   const int lane = threadIdx.x & 31;
   bool ok = true;
+  int64_t vrow = -1; /* the V row of the previous stage, still to issue */
+  auto issue_v = [&](int64_t row) -> bool {
+    const uint32_t j = p.avt, s = j % NV;
+    if (j >= NV && !pwait_bar(c, &c.S->vempty[s], ((j / NV) - 1u) & 1u, layer, PH_ATT)) return false;
+    if (lane == 0) {
+      mbar_arrive_tx(&c.S->vfull[s], ATC_HALF);
+      tma_2d_g2s(vring + (size_t)s * ATC_HALF, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), &c.S->vfull[s]);
+    }
+    __syncwarp();
+    p.avt++;
+    return true;
+  };
   for_each_att_stage(c, g, [&](int pr, int, int64_t k0, int, bool, bool) {
     const int b = pr / P->hkv, h = pr % P->hkv;
     if (k0 + 128 > c.S->pos0[b]) {
       if (!pwait_flag(c, &c.S->kv_ready, layer + 1, layer, PH_ATT)) { ok = false; return false; }
       fence_proxy_async_global();
     }
-    const uint32_t slot = ait % NS;
-    if (ait >= (uint32_t)NS && !pwait_bar(c, &c.S->aempty[slot], ((ait / NS) - 1u) & 1u, layer, PH_ATT)) {
-      ok = false;
-      return false;
-    }
-    uint8_t* stg = c.ring + (size_t)slot * ATC_STAGE;
-    uint64_t* bar = &c.S->afull[slot];
+    const uint32_t j = ait, s = j % NK;
+    if (j >= NK && !pwait_bar(c, &c.S->kempty[s], ((j / NK) - 1u) & 1u, layer, PH_ATT)) { ok = false; return false; }
     const int64_t row = (((int64_t)layer * c.st.kv_seqs + b) * P->hkv + h) * c.st.kv_cap + k0;
-    if (lane == 0) mbar_arrive_tx(bar, 2u * 128u * 128u);
+    if (lane == 0) {
+      mbar_arrive_tx(&c.S->kfull[s], ATC_HALF);
+      tma_2d_g2s(c.ring + (size_t)s * ATC_HALF, c.kvmap, 0, (int32_t)row, &c.S->kfull[s]);
+    }
     __syncwarp();
-    if (lane == 0) tma_2d_g2s(stg, c.kvmap, 0, (int32_t)row, bar);
-    else if (lane == 1) tma_2d_g2s(stg + 16384, c.kvmap, 0, (int32_t)(row + c.st.kv_half_rows), bar);
     ait++;
+    if (vrow >= 0 && !issue_v(vrow)) { ok = false; return false; }
+    vrow = row;
     return true;
   });
+  if (ok && vrow >= 0 && !issue_v(vrow)) ok = false;
   return ok;
 }
 
-/* wait (bounded) until every tc attention stage issued so far is free again */
+/* wait (bounded) until every K and V slot issued so far is free again */
 MSK_DEV bool prod_att_tc_drain(Prod& p, int layer, uint32_t ait) {
   Ctx& c = *p.c;
-  const int NS = atc_ns(atc_rp(c.st.Tq * c.P->G));
-  const uint32_t n = ait < (uint32_t)NS ? ait : (uint32_t)NS;
-  for (uint32_t i = ait - n; i < ait; ++i)
-    if (!pwait_bar(c, &c.S->aempty[i % NS], (i / NS) & 1u, layer, PH_WO)) return false;
+  const int RP = atc_rp(c.st.Tq * c.P->G);
+  const uint32_t NK = (uint32_t)atc_nk(RP), NV = (uint32_t)atc_nv(RP);
+  for (uint32_t i = ait - (ait < NK ? ait : NK); i < ait; ++i)
+    if (!pwait_bar(c, &c.S->kempty[i % NK], (i / NK) & 1u, layer, PH_WO)) return false;
+  for (uint32_t i = p.avt - (p.avt < NV ? p.avt : NV); i < p.avt; ++i)
+    if (!pwait_bar(c, &c.S->vempty[i % NV], (i / NV) & 1u, layer, PH_WO)) return false;
   return true;
 }
 
@@ -1666,25 +1733,34 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
             }
           }
           /* the key's 16-byte row in its core matrices: key group key / 8,
-           * row group, key mod 8 */
-          const uint32_t pt = ptoff + pb * (uint32_t)RP * 256u + (uint32_t)(key >> 3) * (uint32_t)RP * 8u + (uint32_t)(key & 7) * 16u;
-          const uint32_t p1 = (uint32_t)RP * 128u; /* term 1 */
+           * row group, key mod 8.  RP <= 32: the terms stacked as rows
+           * (term t, row n at t RP + n), key groups 2 RP * 8 bytes apart;
+           * RP = 64: a block of RP * 128 bytes per term. */
+          constexpr bool STK = RP <= 32;
+          constexpr uint32_t LBO = STK ? 16u * RP : 8u * RP, P1 = STK ? 8u * RP : 128u * RP; /* term 1 */
+          const uint32_t pt = ptoff + pb * (uint32_t)RP * 256u + (uint32_t)(key >> 3) * LBO + (uint32_t)(key & 7) * 16u;
           if constexpr (NR == 8) {
             sts64(pt + 8u * (uint32_t)hh, w0[0], w0[1]);
-            sts64(pt + p1 + 8u * (uint32_t)hh, w1[0], w1[1]);
+            sts64(pt + P1 + 8u * (uint32_t)hh, w1[0], w1[1]);
           } else {
 #pragma unroll
             for (int gq = 0; gq < NR / 16; ++gq) {
               const uint32_t o = (uint32_t)(hh * (NR / 16) + gq) * 128u;
               sts128(pt + o, w0[4 * gq], w0[4 * gq + 1], w0[4 * gq + 2], w0[4 * gq + 3]);
-              sts128(pt + p1 + o, w1[4 * gq], w1[4 * gq + 1], w1[4 * gq + 2], w1[4 * gq + 3]);
+              sts128(pt + P1 + o, w1[4 * gq], w1[4 * gq + 1], w1[4 * gq + 2], w1[4 * gq + 3]);
             }
           }
-          if (lane < NR) { /* the scales of row hh NR + lane: atom row n mod 32, word n / 32, byte qd */
+          if (lane < NR) { /* the scales of row n' (t RP + n stacked, n per term): atom row n' mod 32, word n' / 32, byte qd */
             const int n = hh * NR + lane;
-            const uint32_t sa = sfoff + pb * 1024u + (uint32_t)(n & 31) * 16u + (uint32_t)(n >> 5) * 4u + (uint32_t)qd;
-            sts8(sa, code);
-            sts8(sa + 512u, code - 4u);
+            const uint32_t sa = sfoff + pb * 1024u + (uint32_t)qd;
+            if constexpr (STK) {
+              const int n1 = RP + n;
+              sts8(sa + (uint32_t)(n & 31) * 16u + (uint32_t)(n >> 5) * 4u, code);
+              sts8(sa + (uint32_t)(n1 & 31) * 16u + (uint32_t)(n1 >> 5) * 4u, code - 4u);
+            } else {
+              sts8(sa + (uint32_t)(n & 31) * 16u + (uint32_t)(n >> 5) * 4u, code);
+              sts8(sa + 512u + (uint32_t)(n & 31) * 16u + (uint32_t)(n >> 5) * 4u, code - 4u);
+            }
           }
         }
         fence_proxy_async_shared();
@@ -1700,15 +1776,21 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
       const int slotp = c.cta + pr;
       float* base = P->part + (size_t)slotp * P->part_stride;
       if (ok) {
-        uint32_t orr[NR];
+        /* O^T: with the terms stacked (RP <= 32) the sum of the two term columns */
+        uint32_t orr[NR], or1[RP <= 32 ? NR : 1];
         const uint32_t ta = tb + ATC_TM_O + (uint32_t)(hh * NR) + ((uint32_t)(qd * 32) << 16);
 #pragma unroll
-        for (int i = 0; i < NR; i += 8) tc_ld8(ta + (uint32_t)i, orr + i);
+        for (int i = 0; i < NR; i += 8) {
+          tc_ld8(ta + (uint32_t)i, orr + i);
+          if constexpr (RP <= 32) tc_ld8(ta + (uint32_t)(RP + i), or1 + i);
+        }
         tc_wait_ld();
 #pragma unroll
         for (int i = 0; i < NR; ++i) {
           const int rho = hh * NR + i;
-          if (rho < R) base[(size_t)rho * (128 + 4) + qd * 32 + lane] = __uint_as_float(orr[i]);
+          float o = __uint_as_float(orr[i]);
+          if constexpr (RP <= 32) o += __uint_as_float(or1[i]);
+          if (rho < R) base[(size_t)rho * (128 + 4) + qd * 32 + lane] = o;
         }
       }
       /* row sums: over the warp's 32 keys, then the four quadrants */
@@ -2491,9 +2573,11 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
       mbar_init(&c.S->dempty2[i], NCW);
     }
     mbar_init(&c.S->tfin, 2);
-    for (int i = 0; i < 5; ++i) {
-      mbar_init(&c.S->afull[i], 1);
-      mbar_init(&c.S->aempty[i], 1);
+    for (int i = 0; i < 6; ++i) {
+      mbar_init(&c.S->kfull[i], 1);
+      mbar_init(&c.S->kempty[i], 1);
+      mbar_init(&c.S->vfull[i], 1);
+      mbar_init(&c.S->vempty[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&c.S->s_ready[i], 1);
