@@ -314,6 +314,8 @@ static_assert(XNS_MAX * GU_SLOT <= MSK_NST * MSK_STAGE, "four gate/up slots fit 
  * warp i mod 8, through that warp's 2-slot ring).  Each unit writes its
  * fp32 partial; the next phase adds the slices in order. */
 constexpr int DKS_MAX = 512;
+constexpr int MAX_KS = 8; /* K slices of a projection of K <= 4096 */
+constexpr int TOPK_MAX = 8; /* experts per token */
 constexpr int DNS = 2;
 constexpr uint32_t DB_BYTES = MSK_MAX_TOKENS * (2 * DKS_MAX + 16);   /* activation slice */
 constexpr uint32_t DSLOT = 16 * (DKS_MAX / 2 + 32 + DKS_MAX / 16); /* one weight m-tile */
@@ -1342,17 +1344,24 @@ MSK_DEV void qkv_head(const Ctx& c, const MskLayer& Ly, int t, int hh, float* v)
   const int hd = P->hd, nqkv = P->qd + 2 * P->kvd, per = hd / 32;
   const int S = P->d <= DKS_MAX ? 1 : P->d / DKS_MAX;
   v[0] = v[1] = v[2] = v[3] = 0.f;
-#pragma unroll 4
-  for (int sl = 0; sl < S; ++sl) {
+  /* every slice's load issued before the first add (S <= 8 for d <= 4096) */
+  float4 q[MAX_KS];
+#pragma unroll
+  for (int sl = 0; sl < MAX_KS; ++sl) {
     const float* raw = P->qkv + ((size_t)sl * c.st.T + t) * nqkv + hh * hd + lane * per;
-    if (per == 4) {
-      const float4 q = *reinterpret_cast<const float4*>(raw);
-      v[0] += q.x; v[1] += q.y; v[2] += q.z; v[3] += q.w;
-    } else {
-      const float2 q = *reinterpret_cast<const float2*>(raw);
-      v[0] += q.x; v[1] += q.y;
+    q[sl] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (sl < S) {
+      if (per == 4) {
+        q[sl] = *reinterpret_cast<const float4*>(raw);
+      } else {
+        const float2 h2 = *reinterpret_cast<const float2*>(raw);
+        q[sl].x = h2.x; q[sl].y = h2.y;
+      }
     }
   }
+#pragma unroll
+  for (int sl = 0; sl < MAX_KS; ++sl)
+    if (sl < S) { v[0] += q[sl].x; v[1] += q[sl].y; v[2] += q[sl].z; v[3] += q[sl].w; }
   if (hh < P->hq + P->hkv) {
     float ss = 0.f;
     for (int i = 0; i < per; ++i) ss += v[i] * v[i];
@@ -1580,13 +1589,22 @@ MSK_DEV void atc_q_terms(const Ctx& c, int pair, int RP, uint32_t qoff) {
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
   const int b = pair / P->hkv, kvh = pair % P->hkv;
   const int R = c.st.Tq * P->G;
-  for (int rho = cw; rho < RP; rho += NCW) {
-    float x[4] = {0.f, 0.f, 0.f, 0.f};
-    if (rho < R) {
+  /* this warp's rows (at most 64 / 8): every load issued first */
+  uint2 wq[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int rho = cw + u * NCW;
+    wq[u] = make_uint2(0u, 0u);
+    if (rho < R && rho < RP) {
       const int t = b * c.st.Tq + rho / P->G, h = kvh * P->G + rho % P->G;
-      const uint2 w = *reinterpret_cast<const uint2*>(P->qs + (size_t)t * P->qd + h * 128 + lane * 4);
-      x[0] = f16lo_f32(w.x); x[1] = f16hi_f32(w.x); x[2] = f16lo_f32(w.y); x[3] = f16hi_f32(w.y);
+      wq[u] = *reinterpret_cast<const uint2*>(P->qs + (size_t)t * P->qd + h * 128 + lane * 4);
     }
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) {
+    const int rho = cw + u * NCW;
+    if (rho >= RP) break;
+    float x[4] = {f16lo_f32(wq[u].x), f16hi_f32(wq[u].x), f16lo_f32(wq[u].y), f16hi_f32(wq[u].y)};
     float mx = fmaxf(fmaxf(fabsf(x[0]), fabsf(x[1])), fmaxf(fabsf(x[2]), fabsf(x[3])));
 #pragma unroll
     for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -2004,20 +2022,33 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
   for (int t = c.cta; t < c.st.T; t += c.ncta) {
     float4 v[ROWV];
     float ss = 0.f;
+    /* residual + W_o o, the projection's K slices added in order; all loads
+     * issued before the first store */
 #pragma unroll
     for (int u = 0; u < ROWV; ++u) {
       const int i = base + u * 128;
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i < (cw + 1) * sl) {
-        /* residual + W_o o, the projection's K slices added in order */
-        float4* hp = reinterpret_cast<float4*>(P->h + (size_t)t * d + i);
-        v[u] = *hp;
-#pragma unroll 4
-        for (int s = 0; s < So; ++s) {
-          const float4 q = *reinterpret_cast<const float4*>(P->qkv + ((size_t)s * c.st.T + t) * d + i);
-          v[u].x += q.x; v[u].y += q.y; v[u].z += q.z; v[u].w += q.w;
+      if (i < (cw + 1) * sl) v[u] = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
+    }
+#pragma unroll
+    for (int s = 0; s < MAX_KS; ++s) {
+      if (s < So) {
+        float4 q[ROWV];
+#pragma unroll
+        for (int u = 0; u < ROWV; ++u) {
+          const int i = base + u * 128;
+          q[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < (cw + 1) * sl) q[u] = *reinterpret_cast<const float4*>(P->qkv + ((size_t)s * c.st.T + t) * d + i);
         }
-        *hp = v[u];
+#pragma unroll
+        for (int u = 0; u < ROWV; ++u) { v[u].x += q[u].x; v[u].y += q[u].y; v[u].z += q[u].z; v[u].w += q[u].w; }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      if (i < (cw + 1) * sl) {
+        *reinterpret_cast<float4*>(P->h + (size_t)t * d + i) = v[u];
         ss += v[u].x * v[u].x + v[u].y * v[u].y + v[u].z * v[u].z + v[u].w * v[u].w;
       }
     }
@@ -2027,29 +2058,43 @@ MSK_DEV void phase_moenorm(const Ctx& c, int layer) {
   }
 }
 
-/* router logits in fp32: warp items (8 tokens, 2 experts); the warps of a
- * CTA take consecutive expert pairs of the same tokens (shared in L1) */
+/* router logits in fp32: CTA items of 8 tokens x 16 experts.  The 8
+ * tokens' normed rows are staged in the ring (idle between the W_o products
+ * and the expert phases), read once from L2 per item; warp w takes experts
+ * 2w, 2w+1 of the item, its lanes 4 consecutive elements of every 128. */
 MSK_DEV void phase_router(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const float* Wr = P->layers[layer].router;
-  const int lane = threadIdx.x & 31, d = P->d;
-  const int ntg = (c.st.T + 7) / 8, nep = P->E / 2;
-  for (int item = gwarp(c); item < ntg * nep; item += nwarps(c)) {
-    const int tg = item / nep, e0 = (item % nep) * 2;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31, ctid = threadIdx.x - CONS0, d = P->d;
+  const int ntg = (c.st.T + 7) / 8, neg = (P->E + 15) / 16;
+  float* xs = reinterpret_cast<float*>(c.ring);
+  int staged = -1;
+  for (int item = c.cta; item < ntg * neg; item += c.ncta) {
+    const int tg = item / neg, e0 = (item % neg) * 16 + 2 * cw;
     const int nt = min(8, c.st.T - tg * 8);
+    if (tg != staged) {
+      named_sync(BAR_CONS, NCT); /* every warp done with the previous rows */
+      const float4* src = reinterpret_cast<const float4*>(P->x2f + (size_t)tg * 8 * d);
+      float4* dst = reinterpret_cast<float4*>(xs);
+      const int n4 = nt * d / 4;
+#pragma unroll 8
+      for (int q = ctid; q < n4; q += NCT) dst[q] = src[q];
+      named_sync(BAR_CONS, NCT);
+      staged = tg;
+    }
+    if (e0 >= P->E) continue;
     float a0[8], a1[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) a0[j] = a1[j] = 0.f;
     const float* w0p = Wr + (size_t)e0 * d;
     const float* w1p = w0p + d;
-    const float* xp = P->x2f + (size_t)tg * 8 * d;
-#pragma unroll 2
+#pragma unroll 4
     for (int i = lane * 4; i < d; i += 128) {
       const float4 w0 = *reinterpret_cast<const float4*>(w0p + i), w1 = *reinterpret_cast<const float4*>(w1p + i);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         if (j < nt) {
-          const float4 x = *reinterpret_cast<const float4*>(xp + (size_t)j * d + i);
+          const float4 x = *reinterpret_cast<const float4*>(xs + (size_t)j * d + i);
           a0[j] += w0.x * x.x + w0.y * x.y + w0.z * x.z + w0.w * x.w;
           a1[j] += w1.x * x.x + w1.y * x.y + w1.z * x.z + w1.w * x.w;
         }
@@ -2065,6 +2110,7 @@ MSK_DEV void phase_router(const Ctx& c, int layer) {
     }
   }
 }
+static_assert(8 * 4096 * 4 <= MSK_NST * MSK_STAGE, "the router stages 8 rows of d <= 4096 floats in the ring");
 
 static_assert(MSK_MAX_TOKENS * 256 * 4 <= MSK_NST * MSK_STAGE, "top-k copies every logit into the stage ring");
 
@@ -2270,18 +2316,33 @@ MSK_DEV void phase_comb(const Ctx& c, int layer) {
     float4 v[ROWV];
     float ss = 0.f;
 #pragma unroll
+    /* all loads issued before the first store; slots added in order */
+#pragma unroll
     for (int u = 0; u < ROWV; ++u) {
       const int i = base + u * 128;
       v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i < (cw + 1) * sl) {
-        float4 acc = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
-#pragma unroll 4
-        for (int s = 0; s < k; ++s) {
-          const float w = R.w[t * k + s];
-          const float4 y = *reinterpret_cast<const float4*>(P->y + (size_t)(t * k + s) * d + i);
-          acc.x += w * y.x; acc.y += w * y.y; acc.z += w * y.z; acc.w += w * y.w;
+      if (i < (cw + 1) * sl) v[u] = *reinterpret_cast<const float4*>(P->h + (size_t)t * d + i);
+    }
+#pragma unroll
+    for (int s = 0; s < TOPK_MAX; ++s) {
+      if (s < k) {
+        const float w = R.w[t * k + s];
+        float4 y[ROWV];
+#pragma unroll
+        for (int u = 0; u < ROWV; ++u) {
+          const int i = base + u * 128;
+          y[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (i < (cw + 1) * sl) y[u] = *reinterpret_cast<const float4*>(P->y + (size_t)(t * k + s) * d + i);
         }
-        v[u] = acc;
+#pragma unroll
+        for (int u = 0; u < ROWV; ++u) { v[u].x += w * y[u].x; v[u].y += w * y[u].y; v[u].z += w * y[u].z; v[u].w += w * y[u].w; }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      if (i < (cw + 1) * sl) {
+        const float4 acc = v[u];
         *reinterpret_cast<float4*>(P->h + (size_t)t * d + i) = acc;
         ss += acc.x * acc.x + acc.y * acc.y + acc.z * acc.z + acc.w * acc.w;
         if (last) {
