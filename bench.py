@@ -457,7 +457,7 @@ def trace_step(args, w, eng, launch, stream, dev, rank):
     msk.msk_set_debug(eng.h)
     distinct = list(msk.msk_query(eng.h).n_distinct[:w.n_layers])
     t = trace.cpu().numpy()
-    order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 9, 10, 11)
+    order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11)
                         if not (l == w.n_layers - 1 and p == 11)]
     out = {PHASES[p]: 0.0 for p in range(12)}
     prev = None
@@ -469,7 +469,7 @@ def trace_step(args, w, eng, launch, stream, dev, rank):
     if rank == 0:
         print(json.dumps({"trace_us": {k: round(v, 1) for k, v in out.items()}, "total_us_after_in": round(total, 1),
                           "distinct_experts_per_layer": distinct,
-                          "note": "router phase includes top-k's predecessor barrier; gate_up includes top-k"}))
+                          "note": "each phase ends at its grid barrier; top-k ends when CTA 0 has its routing (no barrier), so gate_up starts there"}))
     eng.close()
     return 0
 

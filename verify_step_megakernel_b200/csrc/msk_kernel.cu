@@ -2212,8 +2212,11 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
     for (int e = lane; e < E; e += 32) R.cnt[e] = 0;
     __syncwarp();
     /* rank of each pair among same-expert pairs, in pair order */
-    int16_t rank_local[16];
-    for (int base = 0, ch = 0; base < np; base += 32, ++ch) {
+    int rank_local[MSK_MAX_TOKENS * 8 / 32]; /* registers: the chunk loops unroll */
+#pragma unroll
+    for (int ch = 0; ch < MSK_MAX_TOKENS * 8 / 32; ++ch) {
+      const int base = 32 * ch;
+      if (base >= np) break;
       const int pi = base + lane;
       const bool valid = pi < np;
       const int e = valid ? R.ids[pi] : -1 - lane;
@@ -2223,7 +2226,7 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
       __syncwarp();
       if (valid && rank == 0) R.cnt[e] = (int16_t)(before + __popc(peers));
       __syncwarp();
-      rank_local[ch] = (int16_t)(before + rank);
+      rank_local[ch] = before + rank;
     }
     /* exclusive scan of counts -> start */
     int run = 0;
@@ -2239,7 +2242,10 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
     }
     if (lane == 0) R.start[E] = (int16_t)run;
     __syncwarp();
-    for (int base = 0, ch = 0; base < np; base += 32, ++ch) {
+#pragma unroll
+    for (int ch = 0; ch < MSK_MAX_TOKENS * 8 / 32; ++ch) {
+      const int base = 32 * ch;
+      if (base >= np) break;
       const int pi = base + lane;
       if (pi < np) R.pairs[R.start[R.ids[pi]] + rank_local[ch]] = (int16_t)pi;
     }
@@ -2300,6 +2306,8 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
   if (threadIdx.x == CONS0) {
     __threadfence_block();
     c.S->route_ready = layer + 1;
+    /* trace: CTA 0 has its routing (top-k has no grid barrier of its own) */
+    if (c.P->dbg_trace && c.cta == 0) c.P->dbg_trace[layer * 16 + PH_TOPK] = gtimer();
   }
   return true;
 }
