@@ -2113,6 +2113,9 @@ MSK_DEV void phase_router(const Ctx& c, int layer) {
 static_assert(8 * 4096 * 4 <= MSK_NST * MSK_STAGE, "the router stages 8 rows of d <= 4096 floats in the ring");
 
 static_assert(MSK_MAX_TOKENS * 256 * 4 <= MSK_NST * MSK_STAGE, "top-k copies every logit into the stage ring");
+/* the counting sort's per-chunk counts [chunk][E] (int16) in the ring after the logits */
+constexpr uint32_t TOPK_CNT_OFF = MSK_MAX_TOKENS * 256 * 4;
+static_assert(TOPK_CNT_OFF + (MSK_MAX_TOKENS * 8 / 32) * 256 * 2 <= MSK_NST * MSK_STAGE, "top-k scratch fits the ring");
 
 /* order-preserving map of a non-NaN float to u32, -0 taken as +0 */
 MSK_DEV uint32_t ord_key(float x) {
@@ -2161,8 +2164,8 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         key[q][i] = 0u; /* below every real key: never picked while k <= E */
-        if (t < c.st.T && i < per) {
-          const float x = lg[(size_t)t * E + lane * per + i];
+        if (t < c.st.T && i < per) { /* lane holds experts lane + 32 i (conflict-free loads) */
+          const float x = lg[(size_t)t * E + lane + 32 * i];
           key[q][i] = ord_key(x == x ? x : -INFINITY); /* a NaN logit ranks last */
         }
       }
@@ -2185,7 +2188,7 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
 #pragma unroll
       for (int q = 0; q < TQ; ++q) wk[q] = __reduce_max_sync(0xffffffffu, bk[q]);
 #pragma unroll
-      for (int q = 0; q < TQ; ++q) cand[q] = bk[q] == wk[q] ? (uint32_t)(lane * per + bi[q]) : 0xFFFFFFFFu;
+      for (int q = 0; q < TQ; ++q) cand[q] = bk[q] == wk[q] ? (uint32_t)(lane + 32 * bi[q]) : 0xFFFFFFFFu;
 #pragma unroll
       for (int q = 0; q < TQ; ++q) {
         const uint32_t wi = __reduce_min_sync(0xffffffffu, cand[q]);
@@ -2197,58 +2200,81 @@ MSK_DEV bool phase_topk(Ctx& c, int layer, uint32_t& dpar) {
         }
       }
     }
-    __syncwarp(); /* lane 0's picks, read by lanes 0 .. TQ-1 */
-    if (lane < TQ && t0 + lane * NCW < c.st.T) { /* softmax of a token's k picks (the first is the largest) */
-      float* w = R.w + (t0 + lane * NCW) * k;
-      const float vmax = w[0];
-      float sum = 0.f;
-      for (int s = 0; s < k; ++s) { w[s] = expf(w[s] - vmax); sum += w[s]; }
-      for (int s = 0; s < k; ++s) w[s] = w[s] / sum;
-    }
   }
   named_sync(BAR_CONS, NCT);
-  if (cw == 0) {
-    const int np = c.st.T * k;
-    for (int e = lane; e < E; e += 32) R.cnt[e] = 0;
-    __syncwarp();
-    /* rank of each pair among same-expert pairs, in pair order */
-    int rank_local[MSK_MAX_TOKENS * 8 / 32]; /* registers: the chunk loops unroll */
+  /* softmax of each token's k picks (the first is the largest): eight lanes
+   * per token, lane s one pick, the sum by a fixed shuffle tree */
+  for (int base = cw * 32; base < c.st.T * 8; base += NCT) { /* whole warps: the shuffles take every lane */
+    const int i = base + lane, t = i >> 3, sl = i & 7;
+    const bool act = i < c.st.T * 8 && sl < k;
+    float* w = R.w + t * k;
+    const float e = act ? expf(w[sl] - w[0]) : 0.f;
+    float sum = e;
 #pragma unroll
-    for (int ch = 0; ch < MSK_MAX_TOKENS * 8 / 32; ++ch) {
-      const int base = 32 * ch;
-      if (base >= np) break;
-      const int pi = base + lane;
-      const bool valid = pi < np;
-      const int e = valid ? R.ids[pi] : -1 - lane;
-      const uint32_t peers = __match_any_sync(0xffffffffu, e);
-      const int rank = __popc(peers & ((1u << lane) - 1));
-      const int before = valid ? R.cnt[e] : 0;
-      __syncwarp();
-      if (valid && rank == 0) R.cnt[e] = (int16_t)(before + __popc(peers));
-      __syncwarp();
-      rank_local[ch] = before + rank;
-    }
-    /* exclusive scan of counts -> start */
-    int run = 0;
-    for (int base = 0; base < E; base += 32) {
-      int v = R.cnt[base + lane], x = v;
+    for (int o = 4; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o, 8);
+    if (act) w[sl] = e / sum;
+  }
+  named_sync(BAR_CONS, NCT);
+  /* Counting sort of the pairs (token * k + slot) by expert, stable in pair
+   * order.  Warp w takes the 32-pair chunks w, w + 8: per chunk, each pair's
+   * rank among the chunk's pairs of its expert (match_any) and the chunk's
+   * count per expert; then per expert the counts' prefix over chunks, the
+   * experts' starts, and every pair's place. */
+  {
+    const int np = c.st.T * k, nchunk = (np + 31) / 32;
+    int16_t* ccnt = reinterpret_cast<int16_t*>(c.ring + TOPK_CNT_OFF); /* [chunk][E] */
+    for (int i = ctid; i < nchunk * E; i += NCT) ccnt[i] = 0;
+    named_sync(BAR_CONS, NCT);
+    int myrank[2] = {0, 0};
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
+    for (int q = 0; q < 2; ++q) {
+      const int ch = cw + q * NCW;
+      if (ch < nchunk) {
+        const int pi = 32 * ch + lane;
+        const bool valid = pi < np;
+        const int e = valid ? R.ids[pi] : -1 - lane;
+        const uint32_t peers = __match_any_sync(0xffffffffu, e);
+        myrank[q] = __popc(peers & ((1u << lane) - 1));
+        if (valid && myrank[q] == 0) ccnt[ch * E + e] = (int16_t)__popc(peers);
       }
-      R.start[base + lane] = (int16_t)(run + x - v);
-      run += __shfl_sync(0xffffffffu, x, 31);
     }
-    if (lane == 0) R.start[E] = (int16_t)run;
-    __syncwarp();
+    named_sync(BAR_CONS, NCT);
+    for (int e = ctid; e < E; e += NCT) { /* per expert: exclusive prefix over the chunks */
+      int run = 0;
+      for (int ch = 0; ch < nchunk; ++ch) {
+        const int v = ccnt[ch * E + e];
+        ccnt[ch * E + e] = (int16_t)run;
+        run += v;
+      }
+      R.cnt[e] = (int16_t)run;
+    }
+    named_sync(BAR_CONS, NCT);
+    if (cw == 0) { /* exclusive scan of the counts -> start */
+      int run = 0;
+      for (int base = 0; base < E; base += 32) {
+        int v = R.cnt[base + lane], x = v;
 #pragma unroll
-    for (int ch = 0; ch < MSK_MAX_TOKENS * 8 / 32; ++ch) {
-      const int base = 32 * ch;
-      if (base >= np) break;
-      const int pi = base + lane;
-      if (pi < np) R.pairs[R.start[R.ids[pi]] + rank_local[ch]] = (int16_t)pi;
+        for (int o = 1; o < 32; o <<= 1) {
+          int y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        R.start[base + lane] = (int16_t)(run + x - v);
+        run += __shfl_sync(0xffffffffu, x, 31);
+      }
+      if (lane == 0) R.start[E] = (int16_t)run;
     }
+    named_sync(BAR_CONS, NCT);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const int ch = cw + q * NCW, pi = 32 * ch + lane;
+      if (ch < nchunk && pi < np) {
+        const int e = R.ids[pi];
+        R.pairs[R.start[e] + ccnt[ch * E + e] + myrank[q]] = (int16_t)pi;
+      }
+    }
+    named_sync(BAR_CONS, NCT);
+  }
+  if (cw == 0) {
     /* units: experts with tokens, split into groups of <= MSK_UNIT_TOK;
      * the units with at least tau tokens (block-scaled gate/up) first, in
      * expert order, then the others */
