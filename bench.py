@@ -459,6 +459,8 @@ def trace_step(args, w, eng, launch, stream, dev, rank):
     t = trace.cpu().numpy()
     order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11)
                         if not (l == w.n_layers - 1 and p == 11)]
+    # a phase folded into another (the attention combine at head dim 128) leaves no stamp
+    order = [(l, p) for (l, p) in order if t[l, p] != 0]
     out = {PHASES[p]: 0.0 for p in range(12)}
     prev = None
     for (l, p) in order:

@@ -114,6 +114,7 @@ struct Smem {
   uint64_t q_ready;         /* the segment's Q terms written */
   uint64_t o_free;          /* the segment's output accumulator read */
   volatile int ag_ready;    /* layer+1 whose attention key split (ag) the consumers computed */
+  volatile int attc_last;   /* this CTA wrote the last part of a pair: it combines the pair */
   float qfac[64];           /* per query row: softmax scale / its Q-term factor */
   int pos0[MSK_MAX_TOKENS];
   float lbuf[4][32][2];
@@ -1825,6 +1826,44 @@ MSK_DEV bool attention_phase_tc(Ctx& c, int layer, uint32_t& ait, uint32_t& aseg
         base[(size_t)ctid * (128 + 4) + 128] = lred[ctid] + lred[64 + ctid] + lred[128 + ctid] + lred[192 + ctid];
       if (ctid == 0) mbar_arrive(&c.S->o_free);
       aseg++;
+      /* the pair's parts are combined by the CTA that writes the last one
+       * (a counter per pair; the others' parts are visible to it after
+       * their fence and its acquire), so no separate phase and grid barrier
+       * is needed: o = sum of the parts' O / sum of their l, parts in CTA
+       * order, f16 into the W_o projection's input */
+      __threadfence();
+      named_sync(BAR_CONS, NCT);
+      if (ctid == 0) {
+        const int cf = att_owner(g, g.off[pr]), cl = att_owner(g, g.off[pr + 1] - 1);
+        const uint32_t old = atomicAdd(&P->ctrl[CTRL_PAIR0 + pr], 1u);
+        const int last = ok && (int)old + 1 == cl - cf + 1;
+        if (last) P->ctrl[CTRL_PAIR0 + pr] = 0u; /* every part arrived: ready for the next layer */
+        c.S->attc_last = last;
+      }
+      named_sync(BAR_CONS, NCT);
+      if (c.S->attc_last) {
+        __threadfence();
+        const int cf = att_owner(g, g.off[pr]), cl = att_owner(g, g.off[pr + 1] - 1);
+        for (int item = ctid; item < R * 32; item += NCT) {
+          const int rho = item >> 5, c4 = item & 31;
+          float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+          float lsum = 0.f;
+          for (int cc = cf; cc <= cl; ++cc) {
+            const float* row = P->part + (size_t)(cc + pr) * P->part_stride + (size_t)rho * (128 + 4);
+            const float4 q = *reinterpret_cast<const float4*>(row + 4 * c4);
+            acc.x += q.x; acc.y += q.y; acc.z += q.z; acc.w += q.w;
+            lsum += row[128];
+          }
+          const float inv = 1.0f / lsum;
+          const int t = b * c.st.Tq + rho / P->G, h = (pr % P->hkv) * P->G + rho % P->G;
+          uint16_t* dst = P->o + (size_t)t * P->qd + h * 128 + 4 * c4;
+          *reinterpret_cast<uint2*>(dst) = make_uint2(f32x2_to_f16x2(acc.x * inv, acc.y * inv), f32x2_to_f16x2(acc.z * inv, acc.w * inv));
+          if (P->dbg_attn) {
+            float* dbg = P->dbg_attn + ((size_t)layer * c.st.T + t) * P->qd + h * 128 + 4 * c4;
+            *reinterpret_cast<float4*>(dbg) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+          }
+        }
+      }
       named_sync(BAR_CONS, NCT); /* lred reused by the next segment */
     }
   }
@@ -2601,8 +2640,10 @@ MSK_DEV void consumer(Ctx& c) {
     }
     if (!ok) return;
     if (!grid_sync(c, l, PH_ATT)) return;
-    phase_attc(c, l);
-    if (!grid_sync(c, l, PH_ATTC)) return;
+    if constexpr (HD != 128) { /* head dim 128 combines inside its attention phase */
+      phase_attc(c, l);
+      if (!grid_sync(c, l, PH_ATTC)) return;
+    }
     if (!dense_phase<false>(c, l, dpar)) return;
     if (!grid_sync(c, l, PH_WO)) return;
     phase_moenorm(c, l);
