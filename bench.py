@@ -440,7 +440,7 @@ def run_sweep(args, w):
 
 
 PHASES = ["in", "qkv", "qknorm", "attention", "attn_combine", "wo", "moe_norm", "router", "topk", "gate_up",
-          "down", "combine"]
+          "down", "combine", "down_terms"]
 
 
 def trace_step(args, w, eng, launch, stream, dev, rank):
@@ -457,11 +457,11 @@ def trace_step(args, w, eng, launch, stream, dev, rank):
     msk.msk_set_debug(eng.h)
     distinct = list(msk.msk_query(eng.h).n_distinct[:w.n_layers])
     t = trace.cpu().numpy()
-    order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11)
+    order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 8, 9, 12, 10, 11)
                         if not (l == w.n_layers - 1 and p == 11)]
     # a phase folded into another (the attention combine at head dim 128) leaves no stamp
     order = [(l, p) for (l, p) in order if t[l, p] != 0]
-    out = {PHASES[p]: 0.0 for p in range(12)}
+    out = {PHASES[p]: 0.0 for p in range(len(PHASES))}
     prev = None
     for (l, p) in order:
         if prev is not None:

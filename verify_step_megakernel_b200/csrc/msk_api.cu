@@ -18,6 +18,7 @@ extern "C" size_t msk_kernel_smem_bytes();
 extern "C" cudaError_t msk_kernel_setup(int hd, int* ctas_per_sm);
 extern "C" size_t msk_kernel_xtile_gu_bytes(int E, int f, int d);
 extern "C" size_t msk_kernel_xtile_dn_bytes(int E, int rows_per_expert, int K);
+extern "C" size_t msk_kernel_xtile_dt_bytes(int E, int rows_per_expert, int K);
 extern "C" cudaError_t msk_kernel_xtile(int kind, const uint8_t* c0, const uint8_t* c1, const uint8_t* s0, const uint8_t* s1,
                                         uint8_t* out, int E, int rows_per_expert, int K, cudaStream_t st);
 extern "C" cudaError_t msk_kernel_kv_encode(const float* in, uint8_t* out, int64_t n, cudaStream_t stream);
@@ -127,7 +128,7 @@ static uint8_t* g_static_ptr[MSK_STATIC_MAX_DEVICES];
 
 /* where the step's buffers sit inside g_static_scratch */
 struct StaticLayout {
-  size_t params, h, x, qkv, qs, part, o, x2f, x2h, xq, logits, u, y, ctrl, total;
+  size_t params, h, x, qkv, qs, part, o, x2f, x2h, xq, logits, u, ut, y, ctrl, total;
 };
 
 static StaticLayout static_layout(const msk_handle_t* h) {
@@ -150,6 +151,7 @@ static StaticLayout static_layout(const msk_handle_t* h) {
   L.xq = take(T * MSK_XQ_BYTES(d));
   L.logits = take(T * P.E * 4);
   L.u = take(T * P.k * P.f * 2);
+  L.ut = take(T * P.k * MSK_XQ_BYTES(P.f));
   L.y = take(T * P.k * d * 4);
   L.ctrl = take(CTRL_WORDS * 4);
   L.total = at;
@@ -168,6 +170,7 @@ struct StaticPtrs {
   uint8_t* xq;
   float* logits;
   uint16_t* u;
+  uint8_t* ut;
   float* y;
   uint32_t* ctrl;
 };
@@ -192,6 +195,7 @@ __global__ void msk_static_params(const MskParams* src, MskParams* dst, StaticPt
     dst->xq = p.xq;
     dst->logits = p.logits;
     dst->u = p.u;
+    dst->ut = p.ut;
     dst->y = p.y;
     dst->ctrl = p.ctrl;
   }
@@ -308,13 +312,14 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
       T * MSK_XQ_BYTES(d),       /* xq */
       T * P.E * 4,               /* logits */
       T * P.k * P.f * 2,         /* u */
+      T * P.k * MSK_XQ_BYTES(P.f), /* ut */
       T * P.k * d * 4,           /* y */
       (CTRL_WORDS + ST_WORDS) * 4,
       (size_t)P.L * 4,           /* n_distinct */
       (2 + MSK_MAX_TOKENS) * 4,  /* last_shape */
   };
   const int nbuf = sizeof(sizes) / sizeof(sizes[0]);
-  size_t off[16], total = 0;
+  size_t off[20], total = 0;
   for (int i = 0; i < nbuf; ++i) { off[i] = total; total += (sizes[i] + 255) & ~(size_t)255; }
   if (cudaMalloc(&h->scratch, total) != cudaSuccess) { delete h; cudaSetDevice(prev); return MSK_ERR_OOM; }
   cudaMemset(h->scratch, 0, total);
@@ -331,11 +336,12 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   P.xq = b + off[8];
   P.logits = (float*)(b + off[9]);
   P.u = (uint16_t*)(b + off[10]);
-  P.y = (float*)(b + off[11]);
-  P.ctrl = (uint32_t*)(b + off[12]);
+  P.ut = b + off[11];
+  P.y = (float*)(b + off[12]);
+  P.ctrl = (uint32_t*)(b + off[13]);
   P.status = P.ctrl + CTRL_WORDS;
-  P.n_distinct = (int32_t*)(b + off[13]);
-  P.last_shape = (int32_t*)(b + off[14]);
+  P.n_distinct = (int32_t*)(b + off[14]);
+  P.last_shape = (int32_t*)(b + off[15]);
   h->words = P.ctrl;
   /* tensor maps of the expert tensors, for the K-chunked expert tiles */
   {
@@ -412,24 +418,31 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   /* the expert weights as slot images, one contiguous bulk copy per K
    * chunk (library-owned copies; the borrowed weights are not touched):
    * gate/up for the block-scaled path when some unit can take it, down for
-   * the CUDA-core path when its K is a multiple of 256 */
+   * that path too when f is a multiple of 512, and down for the CUDA-core
+   * path when some unit takes it and its K is a multiple of 256 */
   {
-    const bool gu = P.tau <= MSK_UNIT_TOK, dn = (P.f % 256) == 0;
+    const bool gu = P.tau <= MSK_UNIT_TOK, dt = gu && (P.f % 512) == 0 && P.f <= 4096;
+    const bool dn = (P.f % 256) == 0 && (!dt || P.tau > 1); /* tau 1: every unit (>= 1 token) is block-scaled */
     const size_t gub = gu ? msk_kernel_xtile_gu_bytes(P.E, P.f, P.d) : 0;
+    const size_t dtb = dt ? msk_kernel_xtile_dt_bytes(P.E, P.d, P.f) : 0;
     const size_t dnb = dn ? msk_kernel_xtile_dn_bytes(P.E, P.d, P.f) : 0;
-    h->repack_bytes = (gub + dnb) * P.L;
+    h->repack_bytes = (gub + dtb + dnb) * P.L;
     bool ok = h->repack_bytes == 0 || cudaMalloc(&h->repack, h->repack_bytes) == cudaSuccess;
     for (int l = 0; l < P.L && ok && h->repack_bytes; ++l) {
-      uint8_t* g = h->repack + (gub + dnb) * l;
+      uint8_t* g = h->repack + (gub + dtb + dnb) * l;
       const msk_layer_weights_t& w = layers[l];
       if (gu)
         ok = msk_kernel_xtile(0, w.w_gate.codes, w.w_up.codes, w.w_gate.scales, w.w_up.scales, g, P.E, P.f, P.d, 0) ==
              cudaSuccess;
+      if (ok && dt)
+        ok = msk_kernel_xtile(2, w.w_down.codes, nullptr, w.w_down.scales, nullptr, g + gub, P.E, P.d, P.f, 0) ==
+             cudaSuccess;
       if (ok && dn)
-        ok = msk_kernel_xtile(1, w.w_down.codes, nullptr, w.w_down.scales, nullptr, g + gub, P.E, P.d, P.f, 0) ==
+        ok = msk_kernel_xtile(1, w.w_down.codes, nullptr, w.w_down.scales, nullptr, g + gub + dtb, P.E, P.d, P.f, 0) ==
              cudaSuccess;
       P.layers[l].xtgu = gu ? g : nullptr;
-      P.layers[l].xtdn = dn ? g + gub : nullptr;
+      P.layers[l].xtdt = dt ? g + gub : nullptr;
+      P.layers[l].xtdn = dn ? g + gub + dtb : nullptr;
     }
     if (ok) ok = cudaDeviceSynchronize() == cudaSuccess;
     if (!ok) {
@@ -759,6 +772,7 @@ msk_status_t msk_step_static(msk_handle_t* h, const uint16_t* hidden_in, const i
     p.xq = b + Lo.xq;
     p.logits = (float*)(b + Lo.logits);
     p.u = (uint16_t*)(b + Lo.u);
+    p.ut = b + Lo.ut;
     p.y = (float*)(b + Lo.y);
     p.ctrl = (uint32_t*)(b + Lo.ctrl);
     MskParams* Pd = (MskParams*)(b + Lo.params);

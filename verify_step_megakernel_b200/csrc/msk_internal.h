@@ -61,6 +61,12 @@ typedef struct MskLayer {
    * multiple of 256: whole rows are copied then) */
   const uint8_t* xtgu;
   const uint8_t* xtdn;
+  /* down tiles of the block-scaled path [E][d/128][f/512][36 KB]: per 512-wide
+   * K chunk the swizzled codes of its two 256-wide halves, then their
+   * scale-factor atoms (the gate/up tile layout with the halves in place of
+   * the two matrices); null when no unit takes that path or f is not a
+   * multiple of 512 */
+  const uint8_t* xtdt;
   float bound_log2; /* M * log2(e), M = sqrt(hd) max|g_q| max|g_k| */
   int32_t sliding;
 } MskLayer;
@@ -85,6 +91,8 @@ typedef struct MskParams {
                        codes [d/32][8 term rows][16 B], then the fp32 factor */
   float* logits;    /* [T][E] */
   uint16_t* u;      /* [T*k][f] f16 SwiGLU activations */
+  uint8_t* ut;      /* [T*k] the same row as eight e2m1 terms for the down projection on the block-scaled
+                       tensor cores, MSK_XQ_BYTES(f) each (layout of xq) */
   float* y;         /* [T*k][d] expert outputs */
   uint32_t* ctrl;   /* CTRL_WORDS, zeroed per step */
   uint32_t* status; /* ST_WORDS */

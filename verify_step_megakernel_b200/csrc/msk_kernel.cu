@@ -46,7 +46,8 @@ constexpr int REGS_PRODUCER = 64;
 constexpr int REGS_CONSUMER = 208;
 
 enum Phase {
-  PH_IN = 0, PH_QKV, PH_QKNORM, PH_ATT, PH_ATTC, PH_WO, PH_MOENORM, PH_ROUTER, PH_TOPK, PH_GU, PH_DN, PH_COMB
+  PH_IN = 0, PH_QKV, PH_QKNORM, PH_ATT, PH_ATTC, PH_WO, PH_MOENORM, PH_ROUTER, PH_TOPK, PH_GU, PH_DN, PH_COMB,
+  PH_UT /* the SwiGLU rows as e2m1 terms (block-scaled down projection) */
 };
 
 struct Route {
@@ -99,6 +100,7 @@ struct Smem {
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
   volatile int dn_ready;    /* layer+1 whose gate/up outputs all CTAs finished */
+  volatile int ut_ready;    /* layer+1 whose SwiGLU term rows all CTAs finished */
   volatile int dense_done;  /* dense phases this CTA finished (2 per layer) */
   volatile int abort;
   /* attention on the tensor cores (head dim 128): stage ring, score and
@@ -242,6 +244,10 @@ MSK_DEV void item_range(int n, int cta, int ncta, int* a, int* b) {
 constexpr int GU_KC = 256;
 constexpr uint32_t GU_A = 0, GU_AS = 32768, GU_B = 36864, GU_SLOT = 45056;
 constexpr uint32_t GU_AS_END = GU_B; /* codes and scale atoms of a chunk: one repacked tile */
+/* block-scaled down slot: one repacked 512-wide K chunk (the gate/up tile
+ * layout, its halves in place of the matrices), then per half the unit's
+ * pairs' SwiGLU terms (8 pairs x 1 KB) */
+constexpr uint32_t DT_B = GU_AS_END, DT_SLOT = DT_B + 2 * 8192;
 /* TMEM columns: two buffers of gate and up accumulators (128 lanes x 64
  * each), then the scale factors of two chunks in flight */
 constexpr uint32_t TM_D = 0, TM_DU = 64, TM_SFA = 256, TM_SFB = 384, TM_COLS = 512;
@@ -259,13 +265,35 @@ struct XGeo {
 
 /* some expert unit can take the block-scaled gate/up path */
 MSK_DEV bool tc_experts(const MskParams* P) { return P->tau <= MSK_UNIT_TOK; }
+/* the block-scaled units take the block-scaled down projection too (the
+ * host repacked the down tiles for it) */
+MSK_DEV bool tc_down(const MskParams* P) { return P->layers[0].xtdt != nullptr; }
 
 /* the parts of an expert phase: gate/up of the block-scaled units, gate/up
- * of the CUDA-core units, the down projection of every unit */
-enum { XP_TC = 0, XP_CC = 1, XP_DN = 2 };
+ * of the CUDA-core units, the down projection on the CUDA-core path (every
+ * unit, or the CUDA-core units when tc_down), the block-scaled down
+ * projection of the block-scaled units */
+enum { XP_TC = 0, XP_CC = 1, XP_DN = 2, XP_DT = 3 };
 
 MSK_DEV void xgeo(const Ctx& c, int part, XGeo& x) {
   const MskParams* P = c.P;
+  const Route& R = c.S->route;
+  if (part == XP_DT) {
+    x.K = P->f;
+    x.rows_unit = P->d;
+    x.KC = 512;
+    x.nkc = x.K / x.KC;
+    x.tma = 1;
+    x.cpitch = x.spitch = x.bpitch = 0;
+    x.NM = 1;
+    x.mat_bytes = x.b_off = DT_B;
+    x.slot_bytes = DT_SLOT;
+    x.ns = min(XNS_MAX, (int)((uint32_t)(MSK_NST * MSK_STAGE) / DT_SLOT));
+    x.ngroups = x.rows_unit / XROWS;
+    x.u0 = 0;
+    item_range(R.n_units_tc * x.ngroups, c.cta, c.ncta, &x.a, &x.b);
+    return;
+  }
   const bool gu = part != XP_DN, tc = part == XP_TC;
   x.K = gu ? P->d : P->f;
   x.rows_unit = gu ? P->f : P->d;
@@ -281,9 +309,8 @@ MSK_DEV void xgeo(const Ctx& c, int part, XGeo& x) {
   x.slot_bytes = tc ? GU_SLOT : (x.b_off + MSK_UNIT_TOK * x.bpitch + 127) & ~127u;
   x.ns = min(XNS_MAX, (int)((uint32_t)(MSK_NST * MSK_STAGE) / x.slot_bytes));
   x.ngroups = x.rows_unit / XROWS;
-  const Route& R = c.S->route;
-  x.u0 = part == XP_CC ? R.n_units_tc : 0;
-  const int nu = part == XP_TC ? R.n_units_tc : (part == XP_CC ? R.n_units - R.n_units_tc : R.n_units);
+  x.u0 = (part == XP_CC || (part == XP_DN && tc_down(P))) ? R.n_units_tc : 0;
+  const int nu = part == XP_TC ? R.n_units_tc : R.n_units - x.u0;
   item_range(nu * x.ngroups, c.cta, c.ncta, &x.a, &x.b);
 }
 /* bit s set where the phase's fills of expert slot s are odd in number */
@@ -306,6 +333,7 @@ static_assert(2 * ((2 * XROWS * (XKC_MAX / 2 + 32 + XKC_MAX / 16) + MSK_UNIT_TOK
                   MSK_NST * MSK_STAGE,
               "two gate+up slots of the CUDA-core path fit the stage ring");
 static_assert(XNS_MAX * GU_SLOT <= MSK_NST * MSK_STAGE, "four gate/up slots fit the stage ring");
+static_assert(3 * DT_SLOT <= MSK_NST * MSK_STAGE && DT_SLOT % 1024 == 0, "three block-scaled down slots fit the ring");
 
 /* Dense projections (QKV, W_o) with T <= 64 tokens: split-K over CTAs.  A
  * unit is one 16-row m-tile of the output rows times one K slice of 512 (or
@@ -585,6 +613,33 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
   const CUtensorMap* smap[2] = {Ly.emap + (gu ? 1 : 5), Ly.emap + 3};
   const int lane = threadIdx.x & 31;
   int j = 0;
+  if (part == XP_DT) { /* block-scaled down: one repacked tile per 512-wide chunk, the pairs' SwiGLU terms */
+    const size_t utb = MSK_XQ_BYTES(P->f);
+    for (int item = x.a; item < x.b; ++item) {
+      const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups;
+      const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+      const int64_t tile0 = ((int64_t)R.unit_e[unit] * x.ngroups + grp) * x.nkc;
+      const int tl = lane - 8; /* lanes 8-15 copy pair tl's terms */
+      const uint8_t* tq = nullptr;
+      if (lane >= 8 && tl < n) tq = P->ut + (size_t)R.pairs[st0 + tl] * utb;
+      const uint32_t bytes = DT_B + (uint32_t)n * 2048u;
+      for (int kc = 0; kc < x.nkc; ++kc, ++j) {
+        const int s = j % x.ns;
+        if (!prod_xslot(p, s, true, layer, PH_DN)) return false;
+        uint8_t* dst = c.ring + (size_t)s * x.slot_bytes;
+        uint64_t* bar = &c.S->xfull[s];
+        if (lane == 0) mbar_arrive_tx(bar, bytes);
+        __syncwarp();
+        if (lane == 0) {
+          bulk_g2s(dst, Ly.xtdt + (tile0 + kc) * DT_B, DT_B, bar);
+        } else if (tq) { /* per 256-wide half: the pair's kilobyte of terms */
+          bulk_g2s(dst + DT_B + tl * 1024, tq + (size_t)(2 * kc) * 1024, 1024, bar);
+          bulk_g2s(dst + DT_B + 8192 + tl * 1024, tq + (size_t)(2 * kc + 1) * 1024, 1024, bar);
+        }
+      }
+    }
+    return true;
+  }
   if (part == XP_TC) { /* block-scaled tensor cores: swizzled code boxes, scale atoms, the tokens' terms */
     const size_t xqb = MSK_XQ_BYTES(P->d);
     for (int item = x.a; item < x.b; ++item) {
@@ -726,10 +781,12 @@ MSK_DEV void issuer(Ctx& c, int role) {
       tc_cp_sf(tb + TM_SFB + 4 * role, umma_desc(smem_u32(c.S->sfb_one + role * 32), 16, 128, 0));
     }
     __syncwarp();
-    XGeo x, xc, xd;
+    XGeo x, xc, xd, xt;
     xgeo(c, XP_TC, x);
     xgeo(c, XP_CC, xc); /* (read while this layer's routing is current) */
     xgeo(c, XP_DN, xd);
+    const bool dt = tc_down(P) && c.S->route.n_units_tc > 0;
+    xgeo(c, XP_DT, xt);
     const uint32_t ring = smem_u32(c.ring);
     int j = 0;
     for (int item = x.a; item < x.b && ok; ++item) {
@@ -767,9 +824,64 @@ MSK_DEV void issuer(Ctx& c, int role) {
       }
     }
     /* the producer fills the same slots for the CUDA-core units and the
-     * down projection: count those fills too, so the next layer's waits
-     * take the right parity */
-    bits ^= fill_parity(xc) ^ fill_parity(xd);
+     * down projection: count those fills too, so the later waits take the
+     * right parity */
+    bits ^= fill_parity(xc);
+    /* block-scaled down: the items alternate between the roles (item i on
+     * accumulator buffer i mod 2 and role i mod 2); a role issues both
+     * halves of each of its chunks and commits twice for the slot's and the
+     * buffer's two-arrival barriers; it follows the other role's slot fills
+     * and buffer releases in its parities without waiting on them */
+    int jr = 0; /* chunks this role issued */
+    /* a slot's full barrier only tells parities apart: wait until the
+     * CUDA-core fills counted above have all landed (every CTA is past
+     * gate/up once the term rows are ready) before waiting on the fills
+     * that follow them, so no wait can match a fill two phases early */
+    if (dt && ok && !pwait_flag(c, &c.S->ut_ready, l + 1, l, PH_UT)) ok = false;
+    for (int item = xt.a; dt && ok && item < xt.b; ++item) {
+      const int db = (item - xt.a) & 1;
+      const bool mine = db == role;
+      for (int kc = 0; kc < xt.nkc; ++kc) {
+        const int s = ((item - xt.a) * xt.nkc + kc) % xt.ns;
+        if (mine && !pwait_bar(c, &c.S->xfull[s], (bits >> s) & 1u, l, PH_DN)) { ok = false; break; }
+        bits ^= 1u << s;
+        if (kc == 0 && ((bits >> (6 + db)) & 1u)) {
+          if (mine && !pwait_bar(c, &c.S->dempty2[db], (bits >> (4 + db)) & 1u, l, PH_DN)) { ok = false; break; }
+          bits ^= 1u << (4 + db);
+        }
+        if (mine) {
+          if (lane == 0) {
+            tc_fence_after();
+            const uint32_t slot = ring + (uint32_t)s * xt.slot_bytes;
+            const uint64_t sd = umma_desc(slot + GU_AS, 16, 128, 0), ad = umma_desc(slot + GU_A, 16, 1024, 2);
+            /* two scale buffers per role, alternating by chunk */
+            const uint32_t sbuf = tb + TM_SFA + (uint32_t)(2 * (jr & 1) + role) * TM_SFA_BUF;
+            const uint32_t dg = tb + TM_D + db * 128, sfb = tb + TM_SFB + 4 * role;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t sfa = sbuf + 16 * h;
+              const uint64_t bd = umma_desc(slot + DT_B + 8192 * h, 128, 8 * GU_KC / 2, 0);
+#pragma unroll
+              for (int st = 0; st < GU_KC / 64; ++st) tc_cp_sf(sfa + 4 * st, sd + (uint64_t)(128 * h + st * 32));
+#pragma unroll
+              for (int st = 0; st < GU_KC / 64; ++st)
+                tc_mma_nvf4(dg, ad + (uint64_t)(1024 * h + 2 * st), bd + (uint64_t)(16 * st), idesc,
+                            (kc > 0 || h > 0 || st > 0) ? 1u : 0u, sfa + 4 * st, sfb);
+            }
+            tc_commit(&c.S->xempty[s]);
+            tc_commit(&c.S->xempty[s]);
+            if (kc == xt.nkc - 1) {
+              tc_commit(&c.S->dfull2[db]);
+              tc_commit(&c.S->dfull2[db]);
+            }
+          }
+          __syncwarp();
+          ++jr;
+        }
+        if (kc == xt.nkc - 1) bits |= 1u << (6 + db);
+      }
+    }
+    bits ^= fill_parity(xd);
   }
   if (lane == 0) {
     tc_commit(&c.S->tfin);
@@ -856,7 +968,19 @@ MSK_DEV void producer(Ctx& c) {
     }
     if (!pwait_flag(c, &c.S->dn_ready, l + 1, l, PH_DN)) { p.ok = false; break; }
     fence_proxy_async_global();
-    if (!prod_experts(p, l, XP_DN)) { p.ok = false; break; }
+    {
+      const Route& R = c.S->route;
+      const bool dt = tc_down(P) && R.n_units_tc > 0;
+      if (dt) { /* every previous slot released, then the block-scaled down units once their terms exist */
+        if (!prod_xdrain(p, l) || !pwait_flag(c, &c.S->ut_ready, l + 1, l, PH_UT)) { p.ok = false; break; }
+        fence_proxy_async_global();
+        if (!prod_experts(p, l, XP_DT)) { p.ok = false; break; }
+      }
+      if (R.n_units > (dt ? R.n_units_tc : 0)) {
+        if (dt && !prod_xdrain(p, l)) { p.ok = false; break; }
+        if (!prod_experts(p, l, XP_DN)) { p.ok = false; break; }
+      }
+    }
     if (!pwait_flag(c, &c.S->ring_free, l + 1, l, PH_DN)) { p.ok = false; break; }
   }
   if (!p.ok && (threadIdx.x & 31) == 0) {
@@ -1941,7 +2065,7 @@ MSK_DEV void row_quant8(const Ctx& c, const float4* v, int d, float r, const flo
     const int i = base + u * 128;
     x[u][0] = x[u][1] = x[u][2] = x[u][3] = 0.f;
     if (i < (cw + 1) * sl) {
-      const float4 gg = *reinterpret_cast<const float4*>(gain + i);
+      const float4 gg = gain ? *reinterpret_cast<const float4*>(gain + i) : make_float4(1.f, 1.f, 1.f, 1.f);
       x[u][0] = v[u].x * r * gg.x;
       x[u][1] = v[u].y * r * gg.y;
       x[u][2] = v[u].z * r * gg.z;
@@ -1972,6 +2096,31 @@ MSK_DEV void row_quant8(const Ctx& c, const float4* v, int d, float r, const flo
     fj *= 4.0f;
   }
   if (cw == 0 && lane == 0) *reinterpret_cast<float*>(xq + (size_t)4 * d) = finv;
+}
+
+/* The SwiGLU rows of the step's (token, expert) pairs as eight e2m1 terms
+ * for the block-scaled down projection (row_quant8 with unit gains: the
+ * same encoding as the gate/up activations), pair p by CTA p mod ncta. */
+MSK_DEV void phase_ut(const Ctx& c, int layer) {
+  const MskParams* P = c.P;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  const int f = P->f, sl = f / NCW, base = cw * sl + lane * 4, npairs = c.st.T * P->k;
+  const size_t utb = MSK_XQ_BYTES(f);
+  (void)layer;
+  for (int pr = c.cta; pr < npairs; pr += c.ncta) {
+    const uint16_t* ur = P->u + (size_t)pr * f;
+    float4 v[ROWV];
+#pragma unroll
+    for (int u = 0; u < ROWV; ++u) {
+      const int i = base + u * 128;
+      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (i < (cw + 1) * sl) {
+        const uint2 w = *reinterpret_cast<const uint2*>(ur + i);
+        v[u] = make_float4(f16lo_f32(w.x), f16hi_f32(w.x), f16lo_f32(w.y), f16hi_f32(w.y));
+      }
+    }
+    row_quant8(c, v, f, 1.0f, nullptr, P->ut + (size_t)pr * utb);
+  }
 }
 
 MSK_DEV void phase_in(const Ctx& c) {
@@ -2553,6 +2702,59 @@ MSK_DEV bool expert_gu_tc(Ctx& c, int layer, uint32_t& xpar) {
   return !named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
 }
 
+/* Down projection of the block-scaled units on the block-scaled tensor
+ * cores (tcgen05.mma kind::mxf4nvf4, M = 128 weight rows, N = 8 pairs x 8
+ * term rows, K = 64 per instruction): the issuing warps walk the items (see
+ * issuer); the consumer warps run the epilogue, as for gate/up: read the
+ * item's accumulators (TMEM lane = output row), sum each pair's eight term
+ * columns, undo the pair's power-of-two factor and apply the global scale. */
+MSK_DEV bool expert_dt_tc(Ctx& c, int layer, uint32_t& xpar) {
+  const MskParams* P = c.P;
+  const MskLayer& Ly = P->layers[layer];
+  const Route& R = c.S->route;
+  const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
+  XGeo x;
+  xgeo(c, XP_DT, x);
+  const int d = P->d;
+  const float gs = Ly.wd.gs;
+  const size_t utb = MSK_XQ_BYTES(P->f);
+  const uint32_t tb = c.S->tmem_base;
+  const int q = (threadIdx.x >> 5) & 3, th = cw >> 2; /* TMEM lane quadrant, pair half of the epilogue */
+  bool ok = true;
+  for (int item = x.a; item < x.b; ++item) {
+    const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups, db = (item - x.a) & 1;
+    const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+    xpar ^= fill_parity_run(x, item - x.a);
+    const uint32_t dp = (xpar >> (12 + db)) & 1u;
+    xpar ^= 1u << (12 + db);
+    if (ok && !wait_bar(c, &c.S->dfull2[db], dp, layer, PH_DN)) ok = false;
+    ok = __all_sync(0xffffffffu, ok) != 0; /* warp-uniform: the TMEM loads below are warp-collective */
+    if (!ok) continue;
+    tc_fence_after();
+    uint32_t yr[32];
+    tc_ld32(tb + TM_D + db * 128 + ((uint32_t)(q * 32) << 16) + th * 32, yr);
+    tc_wait_ld();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&c.S->dempty2[db]); /* the buffer may take the item after next */
+    const int row = grp * XROWS + q * 32 + lane;
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+      const int tt = th * 4 + t;
+      if (tt < n) {
+        const int pair = R.pairs[st0 + tt];
+        const float fi = *reinterpret_cast<const float*>(P->ut + (size_t)pair * utb + utb - 16);
+        float ysum = 0.f;
+#pragma unroll
+        for (int jt = 7; jt >= 0; --jt) ysum = ysum * 0.25f + __uint_as_float(yr[8 * t + jt]); /* smallest first */
+        P->y[(size_t)pair * d + row] = ysum * fi * gs;
+      }
+    }
+  }
+  if (!ok) c.S->abort = 1;
+  return !named_sync_or(BAR_CONS, NCT, c.S->abort != 0);
+}
+
 /* Gate/up (GU) or down projection of the selected experts on the CUDA-core
  * tensor path (mma.sync, weights decoded in registers): this CTA's items,
  * 16 rows per warp, weight chunks and the unit's activation rows from the
@@ -2655,6 +2857,12 @@ MSK_DEV void consumer(Ctx& c) {
     if (!expert_mma<true>(c, l, xpar)) return;
     if (!grid_sync(c, l, PH_GU)) return;
     if (threadIdx.x == CONS0) c.S->dn_ready = l + 1;
+    if (tc_down(P) && c.S->route.n_units_tc > 0) {
+      phase_ut(c, l);
+      if (!grid_sync(c, l, PH_UT)) return;
+      if (threadIdx.x == CONS0) c.S->ut_ready = l + 1;
+      if (!expert_dt_tc(c, l, xpar)) return;
+    }
     if (!expert_mma<false>(c, l, xpar)) return;
     named_sync(BAR_CONS, NCT);
     if (threadIdx.x == CONS0) c.S->ring_free = l + 1;
@@ -2691,6 +2899,7 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     c.S->ring_free = 0;
     c.S->abort = 0;
     c.S->dn_ready = 0;
+    c.S->ut_ready = 0;
     c.S->dense_done = 0;
     for (int w = 0; w < MSK_NCW; ++w)
       for (int i = 0; i < DNS; ++i) {
@@ -2827,6 +3036,36 @@ __global__ void msk_xtile_gu_kernel(const uint8_t* __restrict__ gc, const uint8_
   }
 }
 
+/* Down projection tiles for the block-scaled path, per (expert, 128-row
+ * group, 512-wide K chunk): the gate/up tile layout with the chunk's two
+ * 256-wide halves in place of the two matrices (swizzled codes of half 0,
+ * of half 1, then each half's four scale-factor atoms). */
+__global__ void msk_xtile_dt_kernel(const uint8_t* __restrict__ dc, const uint8_t* __restrict__ dsc,
+                                    uint4* __restrict__ out, int64_t ntiles, int rows_per_expert, int K) {
+  const int nkc = K / 512, ng = rows_per_expert / 128, k16 = K / 16;
+  const int64_t nch = ntiles * 2304;
+  for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < nch; q += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = q / 2304;
+    const int qi = (int)(q - t * 2304);
+    const int kc = (int)(t % nkc), g = (int)((t / nkc) % ng);
+    const int64_t e = t / ((int64_t)nkc * ng);
+    const int64_t row0 = e * rows_per_expert + (int64_t)g * 128;
+    uint4 v;
+    if (qi < 2048) { /* codes: half h, row r, physical chunk p */
+      const int h = qi >> 10, r = (qi >> 3) & 127, pch = qi & 7, lch = pch ^ (r & 7);
+      v = *reinterpret_cast<const uint4*>(dc + (row0 + r) * (K / 2) + (2 * kc + h) * 128 + lch * 16);
+    } else { /* scale atoms: half h, step st, atom row r: rows r + 32 m1, four blocks */
+      const int ai = qi - 2048, h = ai >> 7, st = (ai >> 5) & 3, r = ai & 31;
+      uint32_t w[4];
+#pragma unroll
+      for (int m1 = 0; m1 < 4; ++m1)
+        w[m1] = *reinterpret_cast<const uint32_t*>(dsc + (row0 + r + 32 * m1) * k16 + ((2 * kc + h) * 4 + st) * 4);
+      v = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    out[q] = v;
+  }
+}
+
 /* Down projection tiles for the CUDA-core path, per (expert, 128-row group,
  * K chunk of KC = min(K, 512)), laid out as its slot: codes [128][KC/2 + 32]
  * (the 32 padding bytes zero) then scales [128][KC/16]. */
@@ -2863,6 +3102,9 @@ extern "C" size_t msk_kernel_xtile_dn_bytes(int E, int rows_per_expert, int K) {
   const int KC = K < 512 ? K : 512;
   return (size_t)E * (rows_per_expert / 128) * (K / KC) * 128 * (KC / 2 + 32 + KC / 16);
 }
+extern "C" size_t msk_kernel_xtile_dt_bytes(int E, int rows_per_expert, int K) {
+  return (size_t)E * (rows_per_expert / 128) * (K / 512) * 36864;
+}
 extern "C" cudaError_t msk_kernel_xtile(int kind, const uint8_t* c0, const uint8_t* c1, const uint8_t* s0, const uint8_t* s1,
                                         uint8_t* out, int E, int rows_per_expert, int K, cudaStream_t st) {
   if (kind == 0) {
@@ -2870,6 +3112,11 @@ extern "C" cudaError_t msk_kernel_xtile(int kind, const uint8_t* c0, const uint8
     const int64_t n = ntiles * 2304;
     msk_xtile_gu_kernel<<<(unsigned)((n + 255) / 256 < 148 * 64 ? (n + 255) / 256 : 148 * 64), 256, 0, st>>>(
         c0, c1, s0, s1, reinterpret_cast<uint4*>(out), ntiles, rows_per_expert, K);
+  } else if (kind == 2) {
+    const int64_t ntiles = (int64_t)E * (rows_per_expert / 128) * (K / 512);
+    const int64_t n = ntiles * 2304;
+    msk_xtile_dt_kernel<<<(unsigned)((n + 255) / 256 < 148 * 64 ? (n + 255) / 256 : 148 * 64), 256, 0, st>>>(
+        c0, s0, reinterpret_cast<uint4*>(out), ntiles, rows_per_expert, K);
   } else {
     const int KC = K < 512 ? K : 512;
     const int64_t ntiles = (int64_t)E * (rows_per_expert / 128) * (K / KC);
