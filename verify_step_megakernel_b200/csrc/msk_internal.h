@@ -27,11 +27,13 @@
 #define MSK_NMAPS 16
 #define MSK_XQ_BYTES(d) ((size_t)(d) * 4 + 16)
 
-/* per-step control words (zeroed before every launch) */
 /* control words, zeroed per step: the grid barrier's counter, the abort
- * word, and from CTRL_PAIR0 one counter per attention pair (the CTAs that
- * have written their part of the pair's attention in the current layer) */
-enum { CTRL_BARRIER = 0, CTRL_ABORT = 1, CTRL_PAIR0 = 32, CTRL_WORDS = 32 + MSK_MAX_PAIRS };
+ * word, from CTRL_PAIR0 one counter per attention pair (the CTAs that have
+ * written their part of the pair's attention in the current layer), and
+ * from CTRL_UT0 one word per (token, expert) pair: the last layer + 1 whose
+ * SwiGLU term row of the pair is written */
+enum { CTRL_BARRIER = 0, CTRL_ABORT = 1, CTRL_PAIR0 = 32, CTRL_UT0 = 32 + MSK_MAX_PAIRS,
+       CTRL_WORDS = CTRL_UT0 + MSK_MAX_TOKENS * 8 };
 /* persistent status words (cleared by msk_step_status) */
 enum { ST_CODE = 0, ST_WHERE = 1, ST_WORDS = 4 };
 

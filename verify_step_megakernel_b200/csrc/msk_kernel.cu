@@ -100,7 +100,6 @@ struct Smem {
   volatile int route_ready; /* layer+1 whose routing this CTA resolved */
   volatile int ring_free;   /* layer+1 whose expert phases released the ring */
   volatile int dn_ready;    /* layer+1 whose gate/up outputs all CTAs finished */
-  volatile int ut_ready;    /* layer+1 whose SwiGLU term rows all CTAs finished */
   volatile int dense_done;  /* dense phases this CTA finished (2 per layer) */
   volatile int abort;
   /* attention on the tensor cores (head dim 128): stage ring, score and
@@ -542,6 +541,24 @@ MSK_DEV bool wait_flag(const Ctx& c, volatile int* flag, int want, int layer, in
   __threadfence_block();
   return true;
 }
+/* wait until a global ready word reaches want (acquire), the abort word and
+ * the clock checked now and then; false on abort or timeout (recorded) */
+MSK_DEV bool wait_gword(const Ctx& c, const uint32_t* word, uint32_t want, int layer, int phase) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0; ld_acquire_u32(word) < want; ++it) {
+    if ((it & 15) == 15) {
+      if (ld_volatile_u32(&c.P->ctrl[CTRL_ABORT])) return false;
+      if (t0 == 0) {
+        t0 = gtimer();
+      } else if (gtimer() - t0 > (uint64_t)c.P->timeout_ns) {
+        raise_err(c, MSK_ERR_TIMEOUT, layer, phase);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
 MSK_DEV bool pwait_flag(const Ctx& c, volatile int* flag, int want, int layer, int phase) {
   return __all_sync(0xffffffffu, wait_flag(c, flag, want, layer, phase)) != 0;
 }
@@ -615,6 +632,7 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
   int j = 0;
   if (part == XP_DT) { /* block-scaled down: one repacked tile per 512-wide chunk, the pairs' SwiGLU terms */
     const size_t utb = MSK_XQ_BYTES(P->f);
+    int wunit = -1; /* the unit whose pairs' terms were last waited for */
     for (int item = x.a; item < x.b; ++item) {
       const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups;
       const int n = R.unit_n[unit], st0 = R.unit_start[unit];
@@ -630,12 +648,21 @@ MSK_DEV bool prod_experts(Prod& p, int layer, int part) {
         uint64_t* bar = &c.S->xfull[s];
         if (lane == 0) mbar_arrive_tx(bar, bytes);
         __syncwarp();
+        bool ok = true;
         if (lane == 0) {
           bulk_g2s(dst, Ly.xtdt + (tile0 + kc) * DT_B, DT_B, bar);
-        } else if (tq) { /* per 256-wide half: the pair's kilobyte of terms */
-          bulk_g2s(dst + DT_B + tl * 1024, tq + (size_t)(2 * kc) * 1024, 1024, bar);
-          bulk_g2s(dst + DT_B + 8192 + tl * 1024, tq + (size_t)(2 * kc + 1) * 1024, 1024, bar);
+        } else if (tq) { /* per 256-wide half: the pair's kilobyte of terms, once some CTA has written them */
+          if (unit != wunit) {
+            ok = wait_gword(c, &P->ctrl[CTRL_UT0 + R.pairs[st0 + tl]], (uint32_t)(layer + 1), layer, PH_UT);
+            fence_proxy_async_global();
+          }
+          if (ok) {
+            bulk_g2s(dst + DT_B + tl * 1024, tq + (size_t)(2 * kc) * 1024, 1024, bar);
+            bulk_g2s(dst + DT_B + 8192 + tl * 1024, tq + (size_t)(2 * kc + 1) * 1024, 1024, bar);
+          }
         }
+        if (!__all_sync(0xffffffffu, ok)) return false;
+        wunit = unit;
       }
     }
     return true;
@@ -835,9 +862,9 @@ MSK_DEV void issuer(Ctx& c, int role) {
     int jr = 0; /* chunks this role issued */
     /* a slot's full barrier only tells parities apart: wait until the
      * CUDA-core fills counted above have all landed (every CTA is past
-     * gate/up once the term rows are ready) before waiting on the fills
-     * that follow them, so no wait can match a fill two phases early */
-    if (dt && ok && !pwait_flag(c, &c.S->ut_ready, l + 1, l, PH_UT)) ok = false;
+     * gate/up) before waiting on the fills that follow them, so no wait can
+     * match a fill two phases early */
+    if (dt && ok && !pwait_flag(c, &c.S->dn_ready, l + 1, l, PH_DN)) ok = false;
     for (int item = xt.a; dt && ok && item < xt.b; ++item) {
       const int db = (item - xt.a) & 1;
       const bool mine = db == role;
@@ -971,10 +998,8 @@ MSK_DEV void producer(Ctx& c) {
     {
       const Route& R = c.S->route;
       const bool dt = tc_down(P) && R.n_units_tc > 0;
-      if (dt) { /* every previous slot released, then the block-scaled down units once their terms exist */
-        if (!prod_xdrain(p, l) || !pwait_flag(c, &c.S->ut_ready, l + 1, l, PH_UT)) { p.ok = false; break; }
-        fence_proxy_async_global();
-        if (!prod_experts(p, l, XP_DT)) { p.ok = false; break; }
+      if (dt) { /* every previous slot released, then the block-scaled down units (each pair's terms waited for) */
+        if (!prod_xdrain(p, l) || !prod_experts(p, l, XP_DT)) { p.ok = false; break; }
       }
       if (R.n_units > (dt ? R.n_units_tc : 0)) {
         if (dt && !prod_xdrain(p, l)) { p.ok = false; break; }
@@ -2099,27 +2124,74 @@ MSK_DEV void row_quant8(const Ctx& c, const float4* v, int d, float r, const flo
 }
 
 /* The SwiGLU rows of the step's (token, expert) pairs as eight e2m1 terms
- * for the block-scaled down projection (row_quant8 with unit gains: the
- * same encoding as the gate/up activations), pair p by CTA p mod ncta. */
+ * for the block-scaled down projection: the encoding of row_quant8 with
+ * unit gains (the same terms, bit for bit), one warp per pair (pair p by
+ * warp p mod (ncta NCW)); lane l codes the 32-value core columns l, l + 32,
+ * ... of the row, one 16-byte row per term.  Each pair's ready word is
+ * released once its row and factor are written. */
 MSK_DEV void phase_ut(const Ctx& c, int layer) {
   const MskParams* P = c.P;
   const int cw = (threadIdx.x >> 5) - CONS_WARP0, lane = threadIdx.x & 31;
-  const int f = P->f, sl = f / NCW, base = cw * sl + lane * 4, npairs = c.st.T * P->k;
+  const int f = P->f, nkk = f / 32, npairs = c.st.T * P->k;
   const size_t utb = MSK_XQ_BYTES(f);
-  (void)layer;
-  for (int pr = c.cta; pr < npairs; pr += c.ncta) {
+  for (int pr = c.cta * NCW + cw; pr < npairs; pr += c.ncta * NCW) {
     const uint16_t* ur = P->u + (size_t)pr * f;
-    float4 v[ROWV];
+    uint8_t* xq = P->ut + (size_t)pr * utb;
+    float mx = 0.f;
+    for (int kk = lane; kk < nkk; kk += 32) {
+      const uint4* s4 = reinterpret_cast<const uint4*>(ur + kk * 32);
 #pragma unroll
-    for (int u = 0; u < ROWV; ++u) {
-      const int i = base + u * 128;
-      v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (i < (cw + 1) * sl) {
-        const uint2 w = *reinterpret_cast<const uint2*>(ur + i);
-        v[u] = make_float4(f16lo_f32(w.x), f16hi_f32(w.x), f16lo_f32(w.y), f16hi_f32(w.y));
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w = s4[q];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) mx = fmaxf(mx, fmaxf(fabsf(f16lo_f32(ws[e])), fabsf(f16hi_f32(ws[e]))));
       }
     }
-    row_quant8(c, v, f, 1.0f, nullptr, P->ut + (size_t)pr * utb);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    int pe = 0;
+    if (mx > 0.f) pe = max(-100, min(100, (int)floorf(log2f(6.0f / mx))));
+    const float f0 = __int_as_float((127 + pe) << 23), finv = __int_as_float((127 - pe) << 23);
+    for (int kk = lane; kk < nkk; kk += 32) {
+      float x[32];
+      const uint4* s4 = reinterpret_cast<const uint4*>(ur + kk * 32);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w = s4[q];
+        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          x[8 * q + 2 * e] = f16lo_f32(ws[e]);
+          x[8 * q + 2 * e + 1] = f16hi_f32(ws[e]);
+        }
+      }
+      float fj = f0;
+#pragma unroll 1
+      for (int t = 0; t < 8; ++t) {
+        const float inv = 1.0f / fj; /* powers of two: exact */
+        uint32_t wd[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t word = 0;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int i = 8 * q + 2 * e;
+            const uint32_t cb = f32x2_to_e2m1x2(x[i] * fj, x[i + 1] * fj), h = e2m1x2_to_f16x2(cb);
+            x[i] -= f16lo_f32(h) * inv;
+            x[i + 1] -= f16hi_f32(h) * inv;
+            word |= cb << (8 * e);
+          }
+          wd[q] = word;
+        }
+        *reinterpret_cast<uint4*>(xq + (size_t)kk * 128 + t * 16) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+        fj *= 4.0f;
+      }
+    }
+    if (lane == 0) *reinterpret_cast<float*>(xq + (size_t)4 * f) = finv;
+    __threadfence();
+    __syncwarp();
+    if (lane == 0) st_release_u32(&P->ctrl[CTRL_UT0 + pr], (uint32_t)(layer + 1));
   }
 }
 
@@ -2721,9 +2793,23 @@ MSK_DEV bool expert_dt_tc(Ctx& c, int layer, uint32_t& xpar) {
   const uint32_t tb = c.S->tmem_base;
   const int q = (threadIdx.x >> 5) & 3, th = cw >> 2; /* TMEM lane quadrant, pair half of the epilogue */
   bool ok = true;
+  int funit = -1;  /* the unit whose pair factors fiv holds */
+  float fiv[4] = {0.f, 0.f, 0.f, 0.f};
   for (int item = x.a; item < x.b; ++item) {
     const int unit = x.u0 + item / x.ngroups, grp = item % x.ngroups, db = (item - x.a) & 1;
     const int n = R.unit_n[unit], st0 = R.unit_start[unit];
+    if (unit != funit) { /* the factors of this warp's four pairs (their words are set: the terms went into the products) */
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int tt = th * 4 + t;
+        if (tt < n) {
+          const int pair = R.pairs[st0 + tt];
+          if (!wait_gword(c, &P->ctrl[CTRL_UT0 + pair], (uint32_t)(layer + 1), layer, PH_DN)) ok = false;
+          fiv[t] = *reinterpret_cast<const float*>(P->ut + (size_t)pair * utb + utb - 16);
+        }
+      }
+      funit = unit;
+    }
     xpar ^= fill_parity_run(x, item - x.a);
     const uint32_t dp = (xpar >> (12 + db)) & 1u;
     xpar ^= 1u << (12 + db);
@@ -2743,11 +2829,10 @@ MSK_DEV bool expert_dt_tc(Ctx& c, int layer, uint32_t& xpar) {
       const int tt = th * 4 + t;
       if (tt < n) {
         const int pair = R.pairs[st0 + tt];
-        const float fi = *reinterpret_cast<const float*>(P->ut + (size_t)pair * utb + utb - 16);
         float ysum = 0.f;
 #pragma unroll
         for (int jt = 7; jt >= 0; --jt) ysum = ysum * 0.25f + __uint_as_float(yr[8 * t + jt]); /* smallest first */
-        P->y[(size_t)pair * d + row] = ysum * fi * gs;
+        P->y[(size_t)pair * d + row] = ysum * fiv[t] * gs;
       }
     }
   }
@@ -2859,8 +2944,6 @@ MSK_DEV void consumer(Ctx& c) {
     if (threadIdx.x == CONS0) c.S->dn_ready = l + 1;
     if (tc_down(P) && c.S->route.n_units_tc > 0) {
       phase_ut(c, l);
-      if (!grid_sync(c, l, PH_UT)) return;
-      if (threadIdx.x == CONS0) c.S->ut_ready = l + 1;
       if (!expert_dt_tc(c, l, xpar)) return;
     }
     if (!expert_mma<false>(c, l, xpar)) return;
@@ -2899,7 +2982,6 @@ __global__ void __launch_bounds__(MSK_NTHREADS, 1)
     c.S->ring_free = 0;
     c.S->abort = 0;
     c.S->dn_ready = 0;
-    c.S->ut_ready = 0;
     c.S->dense_done = 0;
     for (int w = 0; w < MSK_NCW; ++w)
       for (int i = 0; i < DNS; ++i) {
