@@ -68,10 +68,6 @@ MSK_DEV void tma_3d_g2s(void* dst, const CUtensorMap* map, int32_t x, int32_t y,
       "l"(map), "r"(x), "r"(y), "r"(z), "r"(smem_u32(bar))
       : "memory");
 }
-MSK_DEV void tma_prefetch_3d(const CUtensorMap* map, int32_t x, int32_t y, int32_t z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];" ::"l"(map), "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
 MSK_DEV void tma_prefetch_2d(const CUtensorMap* map, int32_t x, int32_t y) {
   asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(map), "r"(x), "r"(y) : "memory");
 }
@@ -126,14 +122,6 @@ MSK_DEV void tc_mma_f8(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
-      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-/* D (+)= A B^T with 16-bit operands (kind::f16: f16 or bf16, fp32 accumulate) */
-MSK_DEV void tc_mma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
-      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
@@ -216,7 +204,6 @@ MSK_DEV void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t 
   asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d));
 }
 MSK_DEV void sts32(uint32_t addr, uint32_t v) { asm volatile("st.shared.u32 [%0], %1;" ::"r"(addr), "r"(v)); }
-MSK_DEV void sts16(uint32_t addr, uint16_t v) { asm volatile("st.shared.u16 [%0], %1;" ::"r"(addr), "h"(v)); }
 MSK_DEV void sts8(uint32_t addr, uint32_t v) { asm volatile("st.shared.u8 [%0], %1;" ::"r"(addr), "r"(v)); }
 MSK_DEV void sts64(uint32_t addr, uint32_t a, uint32_t b) {
   asm volatile("st.shared.v2.u32 [%0], {%1,%2};" ::"r"(addr), "r"(a), "r"(b));
@@ -264,12 +251,6 @@ MSK_DEV uint32_t e4m3x2_to_f16x2(uint32_t two) {
  * sign stays on top. */
 MSK_DEV uint32_t e4m3pair_to_bf16x2_scaled(uint32_t w0, uint32_t w1, uint32_t sel) {
   uint32_t t = __byte_perm(w0, w1, sel); /* [b, b, b', b'] */
-  return (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
-}
-/* bytes 2i and 2i+1 (i = half) of a word of e4m3 codes -> bf16x2 of value *
- * 2^-120 (exact; the same bit move as e4m3pair_to_bf16x2_scaled) */
-MSK_DEV uint32_t e4m3x2_to_bf16x2_scaled(uint32_t w, int half) {
-  const uint32_t t = __byte_perm(w, w, half ? 0x3322u : 0x1100u); /* [b, b, b', b'] */
   return (t & 0x80008000u) | ((t >> 4) & 0x07F007F0u);
 }
 /* the low / high f16 of an f16x2 word as fp32 (exact) */
@@ -328,11 +309,6 @@ MSK_DEV uint32_t hmul2(uint32_t a, uint32_t b) {
   uint32_t r;
   asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
   return r;
-}
-MSK_DEV float f16_to_f32(uint16_t h) {
-  float f;
-  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"(h));
-  return f;
 }
 MSK_DEV uint16_t f32_to_f16(float f) {
   uint16_t h;

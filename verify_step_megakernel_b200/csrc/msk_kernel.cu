@@ -3,24 +3,29 @@
  *
  * One launch runs every layer of the step (the pages' "one program replaces
  * many kernel boundaries"): one CTA per SM, each with one producer warp that
- * streams weight tiles (cp.async.bulk) and KV chunks (2-D tensor copies,
- * 128-byte swizzle) into a ring of shared-memory stages guarded by
- * mbarriers, and eight consumer warps that run the math.  The producer runs
- * ahead across phase and layer boundaries: the next phase's dense weights
- * and the past keys are in flight while the consumers wait at a grid
- * barrier; expert tiles are issued as soon as this CTA has resolved the
- * top-k routing (the pages' "dense weights are streamed through a ring of
- * tiles, selected expert weights are requested as soon as routing
- * finishes").
+ * streams weight tiles (cp.async.bulk), KV stages (tensor copies, 128-byte
+ * swizzle) and expert tiles into shared-memory rings guarded by mbarriers,
+ * two warps that issue the tcgen05 tensor-core products (attention at head
+ * dim 128, the block-scaled experts), and eight consumer warps that run the
+ * rest of the math.  The producer runs ahead across phase and layer
+ * boundaries: the next phase's dense weights and the past keys are in
+ * flight while the consumers wait at a grid barrier; expert tiles are
+ * issued as soon as this CTA has resolved the top-k routing (the pages'
+ * "dense weights are streamed through a ring of tiles, selected expert
+ * weights are requested as soon as routing finishes").
  *
  * Per layer (grid barriers marked |):
  *   QKV projection | QK-norm + fp8 KV write | split-sequence attention with
- *   the fixed softmax bound | chunk combine | W_o + residual | MoE RMSNorm |
- *   router logits | top-k (every CTA, redundantly) + gate/up + SwiGLU |
- *   down projection | weighted combine + next RMSNorm |
- * NVFP4 products run on the tensor cores (mma.sync m16n8k16, f16 operands,
- * fp32 accumulate): each e2m1 code times its e4m3 block scale is exact in
- * f16, the fp32 global scale is applied to the accumulator.
+ *   the fixed softmax bound (at head dim 128 with its chunk combine) |
+ *   (head dim 64: chunk combine |) W_o + residual | MoE RMSNorm | router
+ *   logits | top-k (every CTA, redundantly) + gate/up + SwiGLU | SwiGLU
+ *   terms + down projection | weighted combine + next RMSNorm |
+ * NVFP4 products: the experts of units with at least tau tokens on the
+ * block-scaled tensor cores (tcgen05.mma kind::mxf4nvf4, the activations as
+ * eight e2m1 terms), the projections and the other units on mma.sync
+ * m16n8k16 (f16 operands, fp32 accumulate: each e2m1 code times its e4m3
+ * block scale is exact in f16); the fp32 global scale is applied to the
+ * accumulator.
  *
  * Every wait is bounded by params.timeout_ns; a wait that gives up records
  * MSK_ERR_TIMEOUT and sets an abort word every other wait polls, so the
@@ -770,18 +775,18 @@ MSK_DEV bool prod_xdrain(Prod& p, int layer) {
   return true;
 }
 
-/* The MMA-issuing warp (one elected lane does the issuing): walks the same
- * gate/up chunk sequence as the consumers; per chunk it waits for the
- * consumers' scale staging, copies the scales into TMEM, issues the
- * block-scaled MMAs into the item's accumulator buffer (after the
- * consumers released that buffer) and commits (see expert_gu_tc). */
+/* The attention products of one layer at head dim 128 (QK for role 0, P.V
+ * for role 1), defined with the attention phase. */
 MSK_DEV bool issuer_att(Ctx& c, int layer, int role, uint32_t& ait, uint32_t& aseg);
 
 /* The two MMA-issuing warps (warps 1 and 2; lane 0 issues), role 0 and 1:
- * attention QK and PV products respectively, and the gate and the up
- * matrix of the block-scaled expert path respectively (each copies its
- * matrix's scale atoms into TMEM and issues its MMAs; the slot and the
- * accumulator buffer complete when both have committed). */
+ * attention QK and PV products respectively; the gate and the up matrix of
+ * the block-scaled gate/up items respectively (each copies its matrix's
+ * scale atoms into TMEM and issues its MMAs; the slot and the accumulator
+ * buffer complete when both have committed); and every other item of the
+ * block-scaled down projection each.  Per chunk: wait for the slot's fill
+ * and (first chunk of an item) for the consumers' release of the item's
+ * accumulator buffer, copy the scales, issue the MMAs, commit. */
 MSK_DEV void issuer(Ctx& c, int role) {
   const MskParams* P = c.P;
   const int lane = threadIdx.x & 31;
