@@ -440,7 +440,7 @@ def run_sweep(args, w):
 
 
 PHASES = ["in", "qkv", "qknorm", "attention", "attn_combine", "wo", "moe_norm", "router", "topk", "gate_up",
-          "down", "combine", "down_terms"]
+          "down", "combine"]
 
 
 def trace_step(args, w, eng, launch, stream, dev, rank):
@@ -457,7 +457,7 @@ def trace_step(args, w, eng, launch, stream, dev, rank):
     msk.msk_set_debug(eng.h)
     distinct = list(msk.msk_query(eng.h).n_distinct[:w.n_layers])
     t = trace.cpu().numpy()
-    order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 8, 9, 12, 10, 11)
+    order = [(0, 0)] + [(l, p) for l in range(w.n_layers) for p in (1, 2, 3, 4, 5, 6, 7, 8, 9, 10, 11)
                         if not (l == w.n_layers - 1 and p == 11)]
     # a phase folded into another (the attention combine at head dim 128) leaves no stamp
     order = [(l, p) for (l, p) in order if t[l, p] != 0]
@@ -471,7 +471,7 @@ def trace_step(args, w, eng, launch, stream, dev, rank):
     if rank == 0:
         print(json.dumps({"trace_us": {k: round(v, 1) for k, v in out.items()}, "total_us_after_in": round(total, 1),
                           "distinct_experts_per_layer": distinct,
-                          "note": "each phase ends at its grid barrier; top-k ends when CTA 0 has its routing (no barrier), so gate_up starts there"}))
+                          "note": "each phase ends at its grid barrier; top-k ends when CTA 0 has its routing (no barrier), so gate_up starts there; down includes the encoding of the SwiGLU rows as e2m1 terms"}))
     eng.close()
     return 0
 

@@ -268,8 +268,9 @@ msk_status_t msk_step_status(msk_handle_t* h);
 /* msk_step_status, plus where the device recorded its first error: the
  * layer, the phase (0 input norm, 1 QKV projection, 2 QK-norm and KV write,
  * 3 attention, 4 attention combine, 5 W_o, 6 MoE norm, 7 router, 8 top-k,
- * 9 gate/up, 10 down, 11 combine, 12 the SwiGLU rows as e2m1 terms for
- * the block-scaled down projection) and the CTA; all -1 when the status is
+ * 9 gate/up, 10 down, 11 combine, 12 the wait for a (token, expert) pair's
+ * SwiGLU row as e2m1 terms, read by the block-scaled down projection) and
+ * the CTA; all -1 when the status is
  * MSK_OK or the error carries no site (positions refused before the layer
  * loop).  Any out pointer may be NULL.  Clears the status like
  * msk_step_status. */
