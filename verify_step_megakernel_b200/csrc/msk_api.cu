@@ -418,10 +418,14 @@ msk_status_t msk_create(const msk_config_t* config, const msk_layer_weights_t* l
   /* the expert weights as slot images, one contiguous bulk copy per K
    * chunk (library-owned copies; the borrowed weights are not touched):
    * gate/up for the block-scaled path when some unit can take it, down for
-   * that path too when f is a multiple of 512, and down for the CUDA-core
-   * path when some unit takes it and its K is a multiple of 256 */
+   * that path too when f is 512 or 1024, and down for the CUDA-core path
+   * when some unit takes it and its K is a multiple of 256.  (With at most
+   * two 512-wide chunks per down item, an issuing warp reuses a chunk's
+   * scale-factor columns four fills later, after the slot chain has seen
+   * that chunk's products complete; longer items would reuse them within
+   * one item, ordered only by the tensor pipe's issue order.) */
   {
-    const bool gu = P.tau <= MSK_UNIT_TOK, dt = gu && (P.f % 512) == 0 && P.f <= 4096;
+    const bool gu = P.tau <= MSK_UNIT_TOK, dt = gu && (P.f == 512 || P.f == 1024);
     const bool dn = (P.f % 256) == 0 && (!dt || P.tau > 1); /* tau 1: every unit (>= 1 token) is block-scaled */
     const size_t gub = gu ? msk_kernel_xtile_gu_bytes(P.E, P.f, P.d) : 0;
     const size_t dtb = dt ? msk_kernel_xtile_dt_bytes(P.E, P.d, P.f) : 0;
