@@ -21,6 +21,13 @@ expert_mma and expert_dt_tc.  The issuing warps' wait for the gate/up phase
 to end before the block-scaled down fills is what keeps their first down
 wait from matching a CUDA-core gate/up fill two phases earlier; the second
 test shows the model finds that mistake when the wait is left out.
+
+The tensor-core products complete asynchronously, after their issue, and
+the commits that follow them arrive only then.  A scale-factor copy into
+TMEM is not ordered after earlier products that read the same columns, so
+the model also checks that every such copy comes after those products have
+completed, as seen through the slot chain; the third test shows that this
+needs down items of at most two K chunks.
 """
 import random
 
@@ -57,8 +64,11 @@ def fill_parity_run(nkc, ns, i):
     return m
 
 
-def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
-    """Returns None when every wait matched its fill, else a description."""
+def simulate(seed, layers=4, issuer_waits_for_gate_up=True, dt_chunks=(1, 2)):
+    """Returns None when every wait matched its fill and every scale buffer
+    was reused only after the products that read it completed, else a
+    description.  dt_chunks: the K chunks per block-scaled down item to draw
+    from (512-wide chunks: f / 512)."""
     rnd = random.Random(seed)
     xfull = [Barrier(f"xfull{i}", 1) for i in range(4)]
     xempty = [Barrier(f"xempty{i}", 2) for i in range(4)]
@@ -71,7 +81,7 @@ def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
     geo = []
     for _ in range(layers):
         g = {"tc": (rnd.randint(0, 3), 8, 4), "cc": (rnd.randint(0, 3), 4, 2),
-             "dt": (rnd.randint(0, 4), rnd.choice([1, 2]), 3), "dn": (rnd.randint(0, 3), 1, 3)}
+             "dt": (rnd.randint(0, 4), rnd.choice(dt_chunks), 3), "dn": (rnd.randint(0, 3), 1, 3)}
         # whether the layer has block-scaled units / CUDA-core units at all
         # (the same on every CTA; a CTA's share of a part may still be empty)
         g["tc_on"], g["cc_on"] = rnd.random() < 0.9, rnd.random() < 0.7
@@ -81,6 +91,34 @@ def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
                 g[name] = (0,) + g[name][1:]
         geo.append(g)
     errors = []
+    # the tensor pipe: per issuing warp, its issued chunks' products in issue
+    # order, completing later; the commits after them arrive on completion
+    pipe = {0: [], 1: []}
+    # scale-factor TMEM columns in units of (buffer 0-3, half 0-1) of 16
+    # columns: gate/up chunk j uses buffer j mod 4, half = the warp's role;
+    # a down chunk uses both halves of buffer 2 (its warp's chunk count mod 2)
+    # + role.  scale_user: the products that read a unit last
+    scale_user = {}
+
+    def issue(role, key, units, arrivals):
+        op = {"key": key, "done": False, "arrivals": arrivals}
+        for u in units:
+            prev = scale_user.get(u)
+            if prev is not None and not prev["done"]:
+                errors.append(f"issuer {role}: scale columns {u} copied for {key} while the products of "
+                              f"{prev['key']} may still read them")
+            scale_user[u] = op
+        pipe[role].append(op)
+
+    def tensor_pipe():
+        while True:
+            busy = [r for r in (0, 1) if pipe[r]]
+            if busy:
+                op = pipe[rnd.choice(busy)].pop(0)
+                op["done"] = True
+                for bar, n in op["arrivals"]:
+                    bar.arrive(n)
+            yield
 
     def check_fill(s, key, who):
         idx = fills[s].index(key) if key in fills[s] else None
@@ -164,9 +202,9 @@ def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
                     while not dempty[db].ready((bits >> (4 + db)) & 1):
                         yield
                     bits ^= 1 << (4 + db)
-                xempty[s].arrive()
+                issue(role, (l, "tc", it, kc), [(j & 3, role)],
+                      [(xempty[s], 1)] + ([(dfull[db], 1)] if kc == nkc - 1 else []))
                 if kc == nkc - 1:
-                    dfull[db].arrive()
                     bits |= 1 << (6 + db)
                 yield
             bits ^= fill_parity(*g["cc"])
@@ -174,6 +212,7 @@ def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
                 while state["gu_done"] <= l:
                     yield
             n_items, nkc, ns = g["dt"]
+            jr = 0  # chunks this warp issued
             for j in range(n_items * nkc):
                 it, kc, s = j // nkc, j % nkc, j % ns
                 db = it & 1
@@ -189,9 +228,10 @@ def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
                             yield
                     bits ^= 1 << (4 + db)
                 if mine:
-                    xempty[s].arrive(2)
-                    if kc == nkc - 1:
-                        dfull[db].arrive(2)
+                    b = 2 * (jr & 1) + role
+                    issue(role, (l, "dt", it, kc), [(b, 0), (b, 1)],
+                          [(xempty[s], 2)] + ([(dfull[db], 2)] if kc == nkc - 1 else []))
+                    jr += 1
                 if kc == nkc - 1:
                     bits |= 1 << (6 + db)
                 yield
@@ -243,15 +283,19 @@ def simulate(seed, layers=4, issuer_waits_for_gate_up=True):
             yield
 
     agents = [producer(), issuer(0), issuer(1), consumers()]
+    tp = tensor_pipe()
     steps = 0
     while agents and not errors:
-        a = rnd.choice(agents)
-        try:
-            next(a)
-        except StopIteration:
-            agents.remove(a)
+        a = rnd.choice(agents + [tp])
+        if a is tp:
+            next(tp)
+        else:
+            try:
+                next(a)
+            except StopIteration:
+                agents.remove(a)
         steps += 1
-        if steps > 200_000:
+        if steps > 400_000:
             return "no progress"
     return errors[0] if errors else None
 
@@ -264,3 +308,12 @@ def test_every_wait_matches_its_fill():
 def test_model_finds_the_early_wait_without_the_gate_up_wait():
     found = [seed for seed in range(400) if simulate(seed, issuer_waits_for_gate_up=False) is not None]
     assert found, "the model should find a down wait matching a gate/up fill"
+
+
+def test_scale_buffers_need_items_of_at_most_two_chunks():
+    # four 512-wide chunks per down item (f = 2048): a warp reuses a scale
+    # buffer two chunks later within one item, before the slot chain has
+    # seen those products complete (why msk_create keeps such shapes on the
+    # CUDA-core down path)
+    found = [seed for seed in range(400) if simulate(seed, dt_chunks=(4,)) is not None]
+    assert found and all("scale columns" in simulate(s, dt_chunks=(4,)) for s in found[:5])
